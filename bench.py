@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark: quantized GEMV / MoE weight-stream GB/s on B200.
+
+Headline workload (one "step"): one decode step's projections at TinyLlama-1.1B shape,
+batch 1 — 22 layers of Q4_0 q/o 2048x2048, k/v 256x2048, gate/up 5632x2048, down
+2048x5632 plus a Q8_0 LM head 32000x2048 (614,629,376 weight bytes), all streamed by ONE
+qgemv_batched launch.  Inputs are seeded synthetic tensors resident in HBM; the weights of
+a step (615 MB) are larger than L2 (126 MB), so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  Under torchrun (N > 1) every rank runs an independent
+replica on its own GPU (no data-path collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantized GEMV/MoE weight-stream GB/s (% of HBM peak); us per MoE layer"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["common.cuh", "qgemv.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "block_quant_gemv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """Per-launch DRAM bytes of the headline kernel from the committed ncu summary, or None
+    when the summary is missing or was taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "k_qgemv_tinyllama_decode.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu(logical: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if not vis:
+        return str(logical)
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    return ids[logical] if logical < len(ids) else str(logical)
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample(seconds: float, seed: int):
+    """Time the float64 oracle (single thread) on whole matrices of the decode step, in
+    execution order, until the time budget is used.  Returns (bytes, seconds, n_matrices)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import synth
+    from oracle import qgemv as oq
+    from synth import workloads as wl
+
+    specs = wl.decode_step_specs()
+    done_bytes, t_total, n = 0, 0.0, 0
+    xs = {}
+    with threadpool_limits(1):
+        for s in specs:
+            if s.x_name not in xs:
+                xs[s.x_name] = wl.x_host(specs, s.x_name, seed).numpy().astype(np.float64)
+            W = synth.matrix(s.fmt, s.rows, s.cols, seed, s.name).numpy()
+            t0 = time.perf_counter()
+            oq.qgemv(s.fmt, W, xs[s.x_name], s.rows, s.cols)
+            t_total += time.perf_counter() - t0
+            done_bytes += synth.weight_bytes(s.fmt, s.rows, s.cols) + 4 * (s.rows + s.cols)
+            n += 1
+            if t_total >= seconds:
+                break
+    return done_bytes, t_total, n
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step a bounded sample of the decode step."""
+    if rank != 0:
+        return
+    from synth import workloads as wl
+    per_step_budget = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(per_step_budget / 4, args.seed)
+    tot_b, tot_t, tot_n = 0, 0.0, 0
+    for _ in range(args.steps):
+        b, t, n = oracle_sample(per_step_budget, args.seed)
+        tot_b, tot_t, tot_n = tot_b + b, tot_t + t, tot_n + n
+    gbs = tot_b / tot_t / 1e9
+    specs = wl.decode_step_specs()
+    step_bytes = sum(synth_bytes(s) for s in specs)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_bytes / (gbs * 1e9) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"float64 oracle, single thread, on the first whole matrices of the decode step "
+                                   f"in order ({tot_n // max(1, args.steps)} matrices, ~{per_step_budget:.1f} s per step)"},
+        "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def synth_bytes(s):
+    import synth
+    return synth.weight_bytes(s.fmt, s.rows, s.cols)
+
+
+def workload_config():
+    return {"workload": "tinyllama_decode: 22 layers x Q4_0 (q,o 2048x2048; k,v 256x2048; gate,up 5632x2048; "
+                        "down 2048x5632) + Q8_0 LM head 32000x2048, batch 1, x ~ N(0,1)",
+            "weight_bytes_per_step": 614629376, "launch": "one qgemv_batched launch per step",
+            "l2": "inputs larger than L2 (615 MB of weights per step vs 126 MB L2); no flush",
+            "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------- GPU legs
+def time_decode_step(args, world, dev):
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+
+    specs = wl.decode_step_specs()
+    W = wl.build_gemv_workload(specs, seed=args.seed, device=dev)
+    batch = bqg.GemvBatch(W.items())
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        batch.run()
+    torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(physical_gpu(torch.cuda.current_device()))
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.2)
+    t_begin.record(stream)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        batch.run()
+        ends[i].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    total_ms = t_begin.elapsed_time(t_end)
+    launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(total_ms, world)
+
+    # end to end through the public API: pinned host x -> device, step, device y -> pinned host
+    x_host = torch.empty(W.x_all.shape, dtype=torch.float32, pin_memory=True)
+    x_host.copy_(W.x_all.cpu())
+    y_host = torch.empty(W.y_all.shape, dtype=torch.float32, pin_memory=True)
+    e_steps = max(10, min(args.steps, 500))
+    for _ in range(3):
+        W.x_all.copy_(x_host, non_blocking=True)
+        batch.run()
+        y_host.copy_(W.y_all, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        W.x_all.copy_(x_host, non_blocking=True)
+        batch.run()
+        y_host.copy_(W.y_all, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e_steps
+    barrier(world)
+    return dict(W=W, total_ms=total_ms, launch_ms=launch_ms, clocks=clk, e2e_ms=e2e_ms,
+                h2d=x_host.numel() * 4, d2h=y_host.numel() * 4)
+
+
+def time_single_q8_0(dev, seed):
+    """Single Q8_0 GEMV 2048x2048: 64 distinct weight copies (285 MB, over 2x L2) rotated in a
+    captured CUDA graph; reports us per call and GB/s."""
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    import synth
+    copies = 64
+    Ws = [synth.q8_0_matrix(2048, 2048, seed, f"cfg1/copy{c}", device=dev) for c in range(copies)]
+    x = synth.normal_f32(seed, synth.stream_id("cfg1/x"), 2048).to(dev)
+    y = torch.empty(2048, device=dev)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for W in Ws:
+            bqg.qgemv(bqg.Q8_0, W, x, 2048, 2048, y)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for W in Ws:
+            bqg.qgemv(bqg.Q8_0, W, x, 2048, 2048, y)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    nbytes = 2048 * 64 * 34 + 4 * 2048 * 2
+    return {"workload": "q8_0 2048x2048 batch 1 (64 rotating weight copies, CUDA graph)",
+            "us_per_call": us, "GB/s": nbytes / us / 1e3, "bytes_per_call": nbytes}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    assert torch.cuda.is_available(), "bench.py --impl ours needs a CUDA device"
+    import block_quant_gemv_b200 as bqg
+    bqg.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peak, peak_kind = peaks()
+
+    r = time_decode_step(args, world, dev)
+    W = r["W"]
+    step_bytes = W.weight_bytes + W.activation_bytes
+    ms = r["total_ms"] / args.steps
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    achieved = step_bytes / (r["launch_ms"] * 1e-3) / 1e9
+    e2e_gbs = world * step_bytes / (r["e2e_ms"] * 1e-3) / 1e9
+
+    extras = {}
+    if not args.no_extras:
+        extras["q8_0_2048"] = time_single_q8_0(dev, args.seed)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b, t, n = oracle_sample(args.cpu_seconds, args.seed)
+        cpu = {"value": b / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"float64 oracle, single thread, the first {n} whole matrices of the decode step "
+                         f"({b / 1e6:.0f} MB in {t:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "q4_0/q8_0 weights x fp32 activations, fp32 accumulate",
+            "data": "synthetic", "config": workload_config(),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": committed_traffic(),
+                         "kernel": "k_qgemv (qgemv_batched, 155 matrices)",
+                         "algorithmic_bytes_per_launch": step_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_gbs, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                    "ms_per_step": r["e2e_ms"]},
+            "gpu_launches": args.steps,
+            "clocks": r["clocks"],
+            "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,265 @@
+"""Python binding of libbqg.so — block-quantized GEMV, MoE layer and prefill GEMM on B200.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  There is no CPU
+fallback: if the library is not built, every call raises.
+
+The functions mirror the C ABI in include/bqg.h (same names):
+    qgemv, qgemv_batched, qgemm_prefill, moe_router_logits, moe_router_topk,
+    moe_workspace_size, moe_forward, bqg_status_string, bqg_weight_bytes, bqg_device_errors
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "Q8_0", "Q4_0", "I4_ROW", "ACT_GELU_TANH", "ACT_SILU", "BQGError",
+    "lib", "library_path", "bqg_status_string", "bqg_weight_bytes", "bqg_device_errors",
+    "qgemv", "qgemv_batched", "GemvBatch", "qgemm_prefill", "moe_router_logits",
+    "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward",
+]
+
+Q8_0, Q4_0, I4_ROW = 1, 2, 3
+ACT_GELU_TANH, ACT_SILU = 1, 2
+MAX_COLS, MAX_BATCH, MAX_EXPERTS, MAX_TOPK = 15360, 256, 256, 8
+DEVERR_TIMEOUT, DEVERR_EXPERT_ID = 0x1, 0x2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libbqg.so")
+_lib: Optional[ctypes.CDLL] = None
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+
+class BQGError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {bqg_status_string(status)} ({status})" if what else bqg_status_string(status))
+
+
+class GemvDesc(ctypes.Structure):
+    _fields_ = [("fmt", _i), ("rows", _i), ("cols", _i), ("reserved", _i),
+                ("W", _vp), ("x", _vp), ("y", _vp)]
+
+
+class MoELayerC(ctypes.Structure):
+    _fields_ = [("n_experts", _i), ("top_k", _i), ("hidden", _i), ("inter", _i),
+                ("expert_fmt", _i), ("act", _i),
+                ("gate", _vp), ("up", _vp), ("down", _vp),
+                ("gate_stride", _sz), ("up_stride", _sz), ("down_stride", _sz),
+                ("shared_inter", _i), ("shared_fmt", _i),
+                ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp)]
+
+
+_SIGNATURES = {
+    "bqg_status_string": (ctypes.c_char_p, [_i]),
+    "bqg_version": (_i, []),
+    "bqg_weight_bytes": (_sz, [_i, _i, _i]),
+    "bqg_device_errors": (_i, [ctypes.POINTER(_i)]),
+    "qgemv": (_i, [_i, _vp, _vp, _vp, _i, _i, _vp]),
+    "qgemv_batched": (_i, [ctypes.POINTER(GemvDesc), _i, _vp]),
+    "qgemm_prefill": (_i, [_i, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "moe_router_logits": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "moe_router_topk": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_workspace_size": (_sz, [ctypes.POINTER(MoELayerC), _i]),
+    "moe_forward": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+}
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library.  Raises if it has not been built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is not built; run `python -m block_quant_gemv_b200.build` "
+                               "(the CUDA library is required; there is no CPU fallback)")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(L, name, None)
+            if f is None:
+                continue
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def bqg_status_string(status: int) -> str:
+    return lib().bqg_status_string(int(status)).decode()
+
+
+def bqg_weight_bytes(fmt: int, rows: int, cols: int) -> int:
+    return int(lib().bqg_weight_bytes(fmt, rows, cols))
+
+
+def bqg_device_errors() -> int:
+    """Reads and clears the device error bits (synchronises the device)."""
+    bits = _i(0)
+    _check(lib().bqg_device_errors(ctypes.byref(bits)), "bqg_device_errors")
+    return int(bits.value)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise BQGError(status, what)
+
+
+def _stream(t: torch.Tensor) -> _vp:
+    return _vp(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> _vp:
+    return _vp(0 if t is None else t.data_ptr())
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype: torch.dtype):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ---------------------------------------------------------------- GEMV
+def qgemv(fmt: int, W: torch.Tensor, x: torch.Tensor, rows: int, cols: int,
+          y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = W x for a quantized matrix W (uint8 bytes in the canonical layout of `fmt`)."""
+    _need_cuda("W", W, torch.uint8)
+    _need_cuda("x", x, torch.float32)
+    if y is None:
+        y = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _need_cuda("y", y, torch.float32)
+    if W.numel() < bqg_weight_bytes(fmt, rows, cols) or x.numel() < cols or y.numel() < rows:
+        raise ValueError("tensor smaller than the shape requires")
+    _check(lib().qgemv(fmt, _ptr(W), _ptr(x), _ptr(y), rows, cols, _stream(x)), "qgemv")
+    return y
+
+
+class GemvBatch:
+    """A prepared list of independent GEMVs (fmt, W, x, y, rows, cols) launched as one
+    qgemv_batched call.  Keeps the tensors alive and the descriptor array ready."""
+
+    def __init__(self, items: Sequence[tuple]):
+        if not 1 <= len(items) <= MAX_BATCH:
+            raise ValueError(f"1..{MAX_BATCH} descriptors")
+        self.items = list(items)
+        self.descs = (GemvDesc * len(items))()
+        for d, (fmt, W, x, y, rows, cols) in zip(self.descs, self.items):
+            _need_cuda("W", W, torch.uint8)
+            _need_cuda("x", x, torch.float32)
+            _need_cuda("y", y, torch.float32)
+            if W.numel() < bqg_weight_bytes(fmt, rows, cols) or x.numel() < cols or y.numel() < rows:
+                raise ValueError("tensor smaller than the shape requires")
+            d.fmt, d.rows, d.cols, d.reserved = fmt, rows, cols, 0
+            d.W, d.x, d.y = W.data_ptr(), x.data_ptr(), y.data_ptr()
+        self.device = self.items[0][2].device
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None):
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        _check(lib().qgemv_batched(self.descs, len(self.descs), _vp(s.cuda_stream)), "qgemv_batched")
+
+
+def qgemv_batched(items: Sequence[tuple]) -> None:
+    """Every (fmt, W, x, y, rows, cols) item's y = W x, in one launch."""
+    GemvBatch(items).run()
+
+
+# ---------------------------------------------------------------- prefill GEMM
+def qgemm_prefill(fmt: int, W: torch.Tensor, X: torch.Tensor, n: int, k: int,
+                  Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y[tokens, n] = X[tokens, k] W^T with fp16 X and Y (tensor cores, fp32 accumulation)."""
+    _need_cuda("W", W, torch.uint8)
+    _need_cuda("X", X, torch.float16)
+    tokens = X.shape[0]
+    if Y is None:
+        Y = torch.empty(tokens, n, dtype=torch.float16, device=X.device)
+    _need_cuda("Y", Y, torch.float16)
+    if X.numel() != tokens * k or Y.numel() < tokens * n or W.numel() < bqg_weight_bytes(fmt, n, k):
+        raise ValueError("tensor shapes do not match")
+    _check(lib().qgemm_prefill(fmt, _ptr(W), _ptr(X), _ptr(Y), tokens, n, k, _stream(X)), "qgemm_prefill")
+    return Y
+
+
+# ---------------------------------------------------------------- router
+def moe_router_logits(R: torch.Tensor, x: torch.Tensor, logits: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need_cuda("R", R, torch.float32)
+    _need_cuda("x", x, torch.float32)
+    n_experts, hidden = R.shape
+    tokens = x.numel() // hidden
+    if logits is None:
+        logits = torch.empty(tokens, n_experts, dtype=torch.float32, device=x.device)
+    _need_cuda("logits", logits, torch.float32)
+    _check(lib().moe_router_logits(_ptr(R), _ptr(x), _ptr(logits), tokens, n_experts, hidden, _stream(x)),
+           "moe_router_logits")
+    return logits
+
+
+def moe_router_topk(logits: torch.Tensor, k: int, idx: Optional[torch.Tensor] = None,
+                    weights: Optional[torch.Tensor] = None):
+    _need_cuda("logits", logits, torch.float32)
+    tokens, n_experts = logits.shape
+    if idx is None:
+        idx = torch.empty(tokens, k, dtype=torch.int32, device=logits.device)
+    if weights is None:
+        weights = torch.empty(tokens, k, dtype=torch.float32, device=logits.device)
+    _need_cuda("idx", idx, torch.int32)
+    _need_cuda("weights", weights, torch.float32)
+    _check(lib().moe_router_topk(_ptr(logits), tokens, n_experts, k, _ptr(idx), _ptr(weights), _stream(logits)),
+           "moe_router_topk")
+    return idx, weights
+
+
+# ---------------------------------------------------------------- MoE layer
+class MoELayer:
+    """Device tensors of one MoE layer plus its C description.
+
+    gate/up/down: uint8 tensors holding n_experts matrices each, expert e at byte offset
+    e * <name>_stride.  shared: optional (fmt, inter, gate, up, down) uint8 tensors."""
+
+    def __init__(self, n_experts: int, top_k: int, hidden: int, inter: int, expert_fmt: int, act: int,
+                 gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor,
+                 gate_stride: int, up_stride: int, down_stride: int, shared=None):
+        self.tensors = [gate, up, down]
+        c = MoELayerC()
+        c.n_experts, c.top_k, c.hidden, c.inter = n_experts, top_k, hidden, inter
+        c.expert_fmt, c.act = expert_fmt, act
+        c.gate, c.up, c.down = gate.data_ptr(), up.data_ptr(), down.data_ptr()
+        c.gate_stride, c.up_stride, c.down_stride = gate_stride, up_stride, down_stride
+        if shared is not None:
+            sfmt, sinter, sg, su, sd = shared
+            self.tensors += [sg, su, sd]
+            c.shared_inter, c.shared_fmt = sinter, sfmt
+            c.s_gate, c.s_up, c.s_down = sg.data_ptr(), su.data_ptr(), sd.data_ptr()
+        self.c = c
+        self.hidden, self.top_k, self.n_experts = hidden, top_k, n_experts
+
+
+def moe_workspace_size(layer: MoELayer, tokens: int) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(layer.c), tokens))
+
+
+def moe_forward(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor,
+                y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("idx", idx, torch.int32)
+    _need_cuda("w", w, torch.float32)
+    tokens = x.numel() // layer.hidden
+    if y is None:
+        y = torch.empty(tokens, layer.hidden, dtype=torch.float32, device=x.device)
+    _need_cuda("y", y, torch.float32)
+    need = moe_workspace_size(layer, tokens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _need_cuda("workspace", workspace, torch.uint8)
+    _check(lib().moe_forward(ctypes.byref(layer.c), _ptr(x), _ptr(idx), _ptr(w), _ptr(y), tokens,
+                             _ptr(workspace), workspace.numel(), _stream(x)), "moe_forward")
+    return y

@@ -1,0 +1,64 @@
+// Host-side helpers shared by the C-ABI entry points: device capability checks, cached
+// device attributes, argument checks.  Part of the single translation unit bqg.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "bqg.h"
+
+namespace bqg {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int cc_major = 0;
+  int cc_minor = 0;
+  bool ready = false;
+};
+
+inline DeviceInfo g_devices[kMaxDevices];
+
+// Attributes of the current device (queried once per device).  Returns BQG_OK,
+// BQG_ERR_CUDA or BQG_ERR_DEVICE (not compute capability 10.0).
+inline int current_device(int* dev_out, DeviceInfo** info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BQG_ERR_CUDA;
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BQG_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return BQG_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return BQG_ERR_CUDA;
+    d.ready = true;
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0) return BQG_ERR_DEVICE;
+  *dev_out = dev;
+  *info = &d;
+  return BQG_OK;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BQG_OK : BQG_ERR_CUDA;
+}
+
+// Per-device "dynamic shared memory attribute already set" flags for one kernel.
+struct SmemAttrOnce {
+  std::atomic<bool> done[kMaxDevices] = {};
+  template <typename K>
+  int ensure(int dev, K kernel, size_t bytes) {
+    if (done[dev].load(std::memory_order_acquire)) return BQG_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess)
+      return BQG_ERR_CUDA;
+    done[dev].store(true, std::memory_order_release);
+    return BQG_OK;
+  }
+};
+
+}  // namespace bqg

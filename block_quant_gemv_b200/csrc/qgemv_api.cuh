@@ -1,0 +1,104 @@
+// Host side of qgemv / qgemv_batched: argument checks, problem descriptors, launch.
+#pragma once
+
+#include "host_common.h"
+#include "qgemv.cuh"
+
+namespace bqg {
+
+inline size_t weight_bytes(int fmt, int rows, int cols) {
+  if (rows < 1 || cols < 32 || cols % 32 != 0) return 0;
+  const size_t nb = size_t(cols) / 32;
+  switch (fmt) {
+    case BQG_Q8_0: return size_t(rows) * nb * 34;
+    case BQG_Q4_0: return size_t(rows) * nb * 18;
+    case BQG_I4_ROW: {
+      const size_t packed = size_t(rows) * size_t(cols / 2);
+      return (packed + 15) / 16 * 16 + 4 * size_t(rows);
+    }
+    default: return 0;
+  }
+}
+
+// Fills a GemvProb from one (fmt, W, x, y, rows, cols) after checking it.
+inline int make_gemv_prob(int fmt, const void* W, const float* x, float* y, int rows, int cols, GemvProb* out) {
+  if (W == nullptr || x == nullptr || y == nullptr || rows < 1 || cols < 1) return BQG_ERR_ARG;
+  if (fmt != BQG_Q8_0 && fmt != BQG_Q4_0 && fmt != BQG_I4_ROW) return BQG_ERR_FMT;
+  if (cols % 32 != 0 || cols > BQG_MAX_COLS) return BQG_ERR_SHAPE;
+  if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 4)) return BQG_ERR_ALIGN;
+  GemvProb P{};
+  P.W = static_cast<const uint8_t*>(W);
+  P.x = x;
+  P.y = y;
+  P.rows = rows;
+  P.cols = cols;
+  const int nb = cols / 32;
+  if (fmt == BQG_Q8_0) {
+    P.kind = (nb % 2 == 0) ? kQ8Pair : kQ8One;
+    P.row_bytes = nb * 34;
+  } else if (fmt == BQG_Q4_0) {
+    P.kind = (nb % 2 == 0) ? kQ4Pair : kQ4One;
+    P.row_bytes = nb * 18;
+  } else {
+    P.kind = (cols % 64 == 0) ? kI4x64 : kI4x32;
+    P.row_bytes = cols / 2;
+    const long long packed = (long long)rows * P.row_bytes;
+    if ((packed + 15) / 16 * 16 > 0x7fffffffLL) return BQG_ERR_LIMIT;
+    P.scale_off = int((packed + 15) / 16 * 16);
+  }
+  P.units = P.row_bytes / unit_bytes(P.kind);
+  if (P.units > kGemvCompute) return BQG_ERR_SHAPE;
+  *out = P;
+  return BQG_OK;
+}
+
+inline SmemAttrOnce g_gemv_attr1, g_gemv_attrN;
+
+template <int MAXP>
+inline int launch_gemv(GemvParams<MAXP>& prm, long long total_rows, cudaStream_t stream) {
+  int dev;
+  DeviceInfo* info;
+  int st = current_device(&dev, &info);
+  if (st != BQG_OK) return st;
+  SmemAttrOnce& attr = (MAXP == 1) ? g_gemv_attr1 : g_gemv_attrN;
+  st = attr.ensure(dev, k_qgemv<MAXP>, kGemvSmemBytes);
+  if (st != BQG_OK) return st;
+  long long total = 0;
+  for (int i = 0; i < prm.n; ++i) {
+    prm.p[i].byte_start = total;
+    total += (long long)prm.p[i].rows * prm.p[i].row_bytes;
+  }
+  prm.total_bytes = total;
+  const int grid = int(total_rows < info->sm_count ? total_rows : info->sm_count);
+  k_qgemv<MAXP><<<grid, kGemvThreads, kGemvSmemBytes, stream>>>(prm);
+  return launch_status();
+}
+
+}  // namespace bqg
+
+extern "C" size_t bqg_weight_bytes(int fmt, int rows, int cols) { return bqg::weight_bytes(fmt, rows, cols); }
+
+extern "C" int qgemv(int fmt, const void* W, const float* x, float* y, int rows, int cols, void* stream) {
+  bqg::GemvParams<1> prm{};
+  int st = bqg::make_gemv_prob(fmt, W, x, y, rows, cols, &prm.p[0]);
+  if (st != BQG_OK) return st;
+  prm.n = 1;
+  return bqg::launch_gemv<1>(prm, rows, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream) {
+  if (descs == nullptr || n < 1) return BQG_ERR_ARG;
+  if (n > BQG_MAX_BATCH) return BQG_ERR_LIMIT;
+  static_assert(sizeof(bqg::GemvParams<BQG_MAX_BATCH>) < 32000, "kernel parameter block too large");
+  bqg::GemvParams<BQG_MAX_BATCH> prm{};
+  long long total_rows = 0;
+  for (int i = 0; i < n; ++i) {
+    const bqg_gemv_desc& d = descs[i];
+    if (d.reserved != 0) return BQG_ERR_ARG;
+    int st = bqg::make_gemv_prob(d.fmt, d.W, d.x, d.y, d.rows, d.cols, &prm.p[i]);
+    if (st != BQG_OK) return st;
+    total_rows += d.rows;
+  }
+  prm.n = n;
+  return bqg::launch_gemv<BQG_MAX_BATCH>(prm, total_rows, static_cast<cudaStream_t>(stream));
+}

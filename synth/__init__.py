@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import math
 import zlib
+from typing import Optional
 
 import torch
 
@@ -81,30 +82,34 @@ def _words_as_bytes(w: torch.Tensor) -> torch.Tensor:
     return w32.view(torch.uint8)
 
 
-def random_bytes(seed: int, stream: int, nbytes: int, device="cpu") -> torch.Tensor:
-    nw = (nbytes + 3) // 4
-    return _words_as_bytes(words(seed, stream, nw, device))[:nbytes]
+def random_bytes(seed: int, stream: int, nbytes: int, device="cpu", start: int = 0) -> torch.Tensor:
+    """Bytes start..start+nbytes-1 of the stream (byte b is byte b%4 of word b//4)."""
+    w0 = start // 4
+    nw = (start + nbytes + 3) // 4 - w0
+    b = _words_as_bytes(words(seed, stream, nw, device, start=w0))
+    return b[start - 4 * w0: start - 4 * w0 + nbytes]
 
 
-def uniform_f32(seed: int, stream: int, n: int, lo: float, hi: float, device="cpu") -> torch.Tensor:
+def uniform_f32(seed: int, stream: int, n: int, lo: float, hi: float, device="cpu", start: int = 0) -> torch.Tensor:
     """float32 values lo + (hi-lo)*u with u = k/2**24, k uniform in [0, 2**24).
 
     Every step is a single correctly rounded fp32 operation on fp32 tensors, so the
     result is bit-identical on CPU and GPU."""
-    u = (words(seed, stream, n, device) >> 8).to(torch.float32) * (2.0 ** -24)
+    u = (words(seed, stream, n, device, start=start) >> 8).to(torch.float32) * (2.0 ** -24)
     span = torch.tensor(hi - lo, dtype=torch.float32, device=device)
     base = torch.tensor(lo, dtype=torch.float32, device=device)
     return u * span + base
 
 
-def uniform_f16(seed: int, stream: int, n: int, lo: float, hi: float, device="cpu") -> torch.Tensor:
+def uniform_f16(seed: int, stream: int, n: int, lo: float, hi: float, device="cpu", start: int = 0) -> torch.Tensor:
     """fp16 scale values: the fp32 uniform value rounded to fp16 (round-to-nearest-even)."""
-    return uniform_f32(seed, stream, n, lo, hi, device).to(torch.float16)
+    return uniform_f32(seed, stream, n, lo, hi, device, start).to(torch.float16)
 
 
-def int8_uniform(seed: int, stream: int, n: int, lo: int = -127, hi: int = 127, device="cpu") -> torch.Tensor:
+def int8_uniform(seed: int, stream: int, n: int, lo: int = -127, hi: int = 127, device="cpu",
+                 start: int = 0) -> torch.Tensor:
     span = hi - lo + 1
-    return ((words(seed, stream, n, device) % span) + lo).to(torch.int8)
+    return ((words(seed, stream, n, device, start=start) % span) + lo).to(torch.int8)
 
 
 # ---------------------------------------------------------------- gaussians (host only)
@@ -149,47 +154,59 @@ def i4_row_scale_offset(rows: int, cols: int) -> int:
 
 
 def q8_0_matrix(rows: int, cols: int, seed: int, name: str, device="cpu",
-                d_range=(1e-3, 1e-2), q_range=(-127, 127)) -> torch.Tensor:
-    """Q8_0 matrix bytes: per block an fp16 scale d ~ U[d_range] and 32 int8 q ~ U{q_range}."""
+                d_range=(1e-3, 1e-2), q_range=(-127, 127), r0: int = 0, r1: Optional[int] = None) -> torch.Tensor:
+    """Q8_0 matrix bytes: per block an fp16 scale d ~ U[d_range] and 32 int8 q ~ U{q_range}.
+    With r0/r1, only rows r0..r1-1 of the same matrix (as a standalone matrix)."""
     assert cols % 32 == 0
-    nblk = rows * (cols // 32)
+    r1 = rows if r1 is None else r1
+    nb = cols // 32
+    b0, nblk = r0 * nb, (r1 - r0) * nb
     s = stream_id(name)
-    d = uniform_f16(seed, s ^ 0x1, nblk, *d_range, device=device).view(torch.uint8).view(nblk, 2)
-    q = int8_uniform(seed, s ^ 0x2, nblk * 32, *q_range, device=device).view(torch.uint8).view(nblk, 32)
+    d = uniform_f16(seed, s ^ 0x1, nblk, *d_range, device=device, start=b0).view(torch.uint8).view(nblk, 2)
+    q = int8_uniform(seed, s ^ 0x2, nblk * 32, *q_range, device=device, start=32 * b0)
+    q = q.view(torch.uint8).view(nblk, 32)
     return torch.cat([d, q], dim=1).reshape(-1)
 
 
 def q4_0_matrix(rows: int, cols: int, seed: int, name: str, device="cpu",
-                d_range=(1e-3, 1e-2)) -> torch.Tensor:
+                d_range=(1e-3, 1e-2), r0: int = 0, r1: Optional[int] = None) -> torch.Tensor:
     """Q4_0 matrix bytes: per block an fp16 scale d ~ U[d_range] and 16 uniformly random bytes
-    (each byte holds two independent nibbles uniform in 0..15)."""
+    (each byte holds two independent nibbles uniform in 0..15).
+    With r0/r1, only rows r0..r1-1 of the same matrix (as a standalone matrix)."""
     assert cols % 32 == 0
-    nblk = rows * (cols // 32)
+    r1 = rows if r1 is None else r1
+    nb = cols // 32
+    b0, nblk = r0 * nb, (r1 - r0) * nb
     s = stream_id(name)
-    d = uniform_f16(seed, s ^ 0x1, nblk, *d_range, device=device).view(torch.uint8).view(nblk, 2)
-    qs = random_bytes(seed, s ^ 0x2, nblk * 16, device=device).view(nblk, 16)
+    d = uniform_f16(seed, s ^ 0x1, nblk, *d_range, device=device, start=b0).view(torch.uint8).view(nblk, 2)
+    qs = random_bytes(seed, s ^ 0x2, nblk * 16, device=device, start=16 * b0).view(nblk, 16)
     return torch.cat([d, qs], dim=1).reshape(-1)
 
 
 def i4_row_matrix(rows: int, cols: int, seed: int, name: str, device="cpu",
-                  s_range=(1e-3, 1e-2)) -> torch.Tensor:
+                  s_range=(1e-3, 1e-2), r0: int = 0, r1: Optional[int] = None) -> torch.Tensor:
     """i4_row matrix bytes: uniformly random packed nibbles (two's-complement values -8..7),
-    zero padding to 16 B, then fp32 row scales ~ U[s_range]."""
+    zero padding to 16 B, then fp32 row scales ~ U[s_range].
+    With r0/r1, only rows r0..r1-1 of the same matrix (as a standalone matrix)."""
     assert cols % 2 == 0
+    r1 = rows if r1 is None else r1
+    n = r1 - r0
     s = stream_id(name)
-    packed = rows * (cols // 2)
-    off = i4_row_scale_offset(rows, cols)
-    out = torch.zeros(off + 4 * rows, dtype=torch.uint8, device=device)
-    out[:packed] = random_bytes(seed, s ^ 0x2, packed, device=device)
-    out[off:] = uniform_f32(seed, s ^ 0x1, rows, *s_range, device=device).view(torch.uint8)
+    rb = cols // 2
+    packed = n * rb
+    off = i4_row_scale_offset(n, cols)
+    out = torch.zeros(off + 4 * n, dtype=torch.uint8, device=device)
+    out[:packed] = random_bytes(seed, s ^ 0x2, packed, device=device, start=r0 * rb)
+    out[off:] = uniform_f32(seed, s ^ 0x1, n, *s_range, device=device, start=r0).view(torch.uint8)
     return out
 
 
-def matrix(fmt: int, rows: int, cols: int, seed: int, name: str, device="cpu") -> torch.Tensor:
+def matrix(fmt: int, rows: int, cols: int, seed: int, name: str, device="cpu",
+           r0: int = 0, r1: Optional[int] = None) -> torch.Tensor:
     if fmt == FMT_Q8_0:
-        return q8_0_matrix(rows, cols, seed, name, device)
+        return q8_0_matrix(rows, cols, seed, name, device, r0=r0, r1=r1)
     if fmt == FMT_Q4_0:
-        return q4_0_matrix(rows, cols, seed, name, device)
+        return q4_0_matrix(rows, cols, seed, name, device, r0=r0, r1=r1)
     if fmt == FMT_I4_ROW:
-        return i4_row_matrix(rows, cols, seed, name, device)
+        return i4_row_matrix(rows, cols, seed, name, device, r0=r0, r1=r1)
     raise ValueError(f"unknown format {fmt}")

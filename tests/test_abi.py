@@ -1,0 +1,96 @@
+"""The C-ABI library on the host: it builds, loads, exports every symbol include/bqg.h
+declares, and rejects invalid arguments with typed errors before touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import synth
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bqg.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_quant_gemv_b200 import build
+    build.build()
+    import block_quant_gemv_b200 as bqg
+    return bqg
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for want in ["qgemv", "qgemv_batched", "bqg_status_string", "bqg_weight_bytes",
+                 "bqg_device_errors", "bqg_version"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    so = ctypes.CDLL(L.library_path())
+    for name in declared_functions():
+        assert hasattr(so, name), f"{name} declared in bqg.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", L.library_path()], capture_output=True, text=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if " T " in line)
+    for name in declared_functions():
+        assert name in exported
+
+
+def test_status_strings(L):
+    for s in range(0, -9, -1):
+        assert L.bqg_status_string(s).startswith("BQG")
+    assert L.lib().bqg_version() >= 100
+
+
+def test_weight_bytes_agrees_with_generator(L):
+    for fmt in (1, 2, 3):
+        for rows, cols in [(1, 32), (7, 96), (2048, 2048), (6144, 2048), (3, 704)]:
+            assert L.bqg_weight_bytes(fmt, rows, cols) == synth.weight_bytes(fmt, rows, cols)
+    assert L.bqg_weight_bytes(9, 4, 32) == 0
+    assert L.bqg_weight_bytes(1, 4, 33) == 0
+    assert L.bqg_weight_bytes(1, 0, 32) == 0
+
+
+def test_qgemv_argument_errors_before_any_launch(L):
+    f = L.lib().qgemv
+    A = 0x10000  # a 16-byte aligned fake address; nothing is dereferenced on these paths
+    assert f(9, A, A, A, 4, 32, None) == -2                # unknown format
+    assert f(1, None, A, A, 4, 32, None) == -1             # null W
+    assert f(1, A, A, A, 0, 32, None) == -1                # rows < 1
+    assert f(1, A, A, A, 4, 33, None) == -3                # cols % 32
+    assert f(2, A, A, A, 4, 15360 + 32, None) == -3        # cols above the maximum
+    assert f(2, A + 2, A, A, 4, 32, None) == -4            # W not 16-byte aligned
+    assert f(2, A, A + 4, A, 4, 32, None) == -4            # x not 16-byte aligned
+    assert f(2, A, A, A + 2, 4, 32, None) == -4            # y not 4-byte aligned
+
+
+def test_qgemv_batched_argument_errors(L):
+    f = L.lib().qgemv_batched
+    D = (L.GemvDesc * 300)()
+    for d in D:
+        d.fmt, d.rows, d.cols, d.W, d.x, d.y = 2, 4, 32, 0x10000, 0x10000, 0x10000
+    assert f(None, 1, None) == -1
+    assert f(D, 0, None) == -1
+    assert f(D, 300, None) == -8
+    D[3].cols = 48
+    assert f(D, 5, None) == -3
+    D[3].cols = 32
+    D[1].reserved = 1
+    assert f(D, 5, None) == -1
+
+
+def test_valid_call_without_gpu_fails_loudly(L):
+    """With no usable device, a valid call returns an error: there is no CPU fallback."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.lib().qgemv(2, 0x10000, 0x10000, 0x10000, 4, 32, None) in (-6, -7)

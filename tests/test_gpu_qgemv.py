@@ -1,0 +1,125 @@
+"""GPU parity of qgemv / qgemv_batched against the float64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import block_quant_gemv_b200 as bqg
+import synth
+from synth import workloads as wl
+from oracle import qgemv as oq
+from tests.util import assert_close, need_gpu
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [bqg.Q8_0, bqg.Q4_0, bqg.I4_ROW]
+# (rows, cols): single block, odd block counts (unpaired units), ragged rows, several
+# stages per CTA, rows not 16-byte aligned (cols 704 / 2112), the largest cols.
+SHAPES = [(1, 32), (3, 64), (37, 96), (5, 160), (130, 704), (300, 2112), (77, 5632),
+          (1000, 2048), (2048, 2048), (4099, 256), (64, 15360), (513, 2816)]
+
+
+def _run(fmt, rows, cols, seed=0):
+    need_gpu()
+    name = f"t/{fmt}/{rows}x{cols}"
+    W_host = synth.matrix(fmt, rows, cols, seed, name)
+    x_host = synth.normal_f32(seed, synth.stream_id(name + "/x"), cols)
+    y = bqg.qgemv(fmt, W_host.cuda(), x_host.cuda(), rows, cols)
+    torch.cuda.synchronize()
+    ref = oq.qgemv(fmt, W_host.numpy(), x_host.numpy().astype(np.float64), rows, cols)
+    return y, ref
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("rows,cols", SHAPES)
+def test_qgemv_matches_oracle(fmt, rows, cols):
+    y, ref = _run(fmt, rows, cols)
+    assert_close(y, ref, what=f"fmt {fmt} {rows}x{cols}")
+    # fp32 accumulation of exact dequantized products: far inside the tolerance
+    assert_close(y, ref, tol=1e-5, what=f"fmt {fmt} {rows}x{cols} (fp32 accuracy)")
+
+
+def test_q8_0_2048_config_seed0():
+    """The single Q8_0 GEMV configuration: W 2048x2048, seed 0."""
+    y, ref = _run(bqg.Q8_0, 2048, 2048, seed=0)
+    assert_close(y, ref, what="q8_0 2048x2048")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_qgemv_deterministic(fmt):
+    need_gpu()
+    W = synth.matrix(fmt, 999, 2048, 1, "det").cuda()
+    x = synth.normal_f32(1, 2, 2048).cuda()
+    a = bqg.qgemv(fmt, W, x, 999, 2048)
+    b = bqg.qgemv(fmt, W, x, 999, 2048)
+    assert torch.equal(a, b)
+
+
+def test_qgemv_special_inputs():
+    """x = 0 gives exactly 0; all-zero scales give 0; a unit vector reads one column."""
+    need_gpu()
+    rows, cols = 64, 256
+    for fmt in FMTS:
+        W = synth.matrix(fmt, rows, cols, 2, "sp")
+        y0 = bqg.qgemv(fmt, W.cuda(), torch.zeros(cols, device="cuda"), rows, cols)
+        assert torch.count_nonzero(y0) == 0
+        e = torch.zeros(cols)
+        e[37] = 1.0
+        y1 = bqg.qgemv(fmt, W.cuda(), e.cuda(), rows, cols).cpu().numpy()
+        ref = oq.dequantize(fmt, W.numpy(), rows, cols)[:, 37]
+        np.testing.assert_allclose(y1, ref, rtol=1e-6, atol=1e-9)
+    # zero scales in Q8_0 / Q4_0
+    for fmt, blk in ((bqg.Q8_0, 34), (bqg.Q4_0, 18)):
+        W = synth.matrix(fmt, rows, cols, 3, "zs").view(-1, blk).clone()
+        W[:, 0:2] = 0
+        y = bqg.qgemv(fmt, W.reshape(-1).cuda(), synth.normal_f32(3, 4, cols).cuda(), rows, cols)
+        assert torch.count_nonzero(y) == 0
+
+
+def test_qgemv_batched_mixed_matches_oracle():
+    need_gpu()
+    shapes = [(bqg.Q4_0, 2048, 2048), (bqg.Q4_0, 256, 2048), (bqg.Q8_0, 300, 2112), (bqg.I4_ROW, 129, 6144),
+              (bqg.Q4_0, 2816, 704), (bqg.Q8_0, 7, 96), (bqg.Q4_0, 33, 5632), (bqg.I4_ROW, 5, 32)]
+    host, items = [], []
+    for i, (fmt, rows, cols) in enumerate(shapes):
+        W = synth.matrix(fmt, rows, cols, 5, f"b{i}")
+        x = synth.normal_f32(5, 100 + i, cols)
+        y = torch.full((rows,), float("nan"), device="cuda")
+        host.append((fmt, W, x, rows, cols))
+        items.append((fmt, W.cuda(), x.cuda(), y, rows, cols))
+    bqg.qgemv_batched(items)
+    torch.cuda.synchronize()
+    for (fmt, W, x, rows, cols), it in zip(host, items):
+        ref = oq.qgemv(fmt, W.numpy(), x.numpy().astype(np.float64), rows, cols)
+        assert_close(it[3], ref, what=f"batched fmt {fmt} {rows}x{cols}")
+
+
+def test_generator_same_bytes_on_gpu_and_cpu():
+    need_gpu()
+    for fmt in FMTS:
+        a = synth.matrix(fmt, 300, 2112 if fmt != bqg.I4_ROW else 2048, 9, "xdev")
+        b = synth.matrix(fmt, 300, 2112 if fmt != bqg.I4_ROW else 2048, 9, "xdev", device="cuda")
+        assert torch.equal(a, b.cpu())
+
+
+def test_tinyllama_decode_step_full_size_sampled():
+    """The decode-step workload at full size in the benchmark's launch configuration (one
+    qgemv_batched call over all 155 matrices): sampled rows of every matrix against the
+    oracle on rows regenerated on the host."""
+    need_gpu()
+    specs = wl.decode_step_specs()
+    W = wl.build_gemv_workload(specs, seed=0, device="cuda")
+    batch = bqg.GemvBatch(W.items())
+    batch.run()
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    xs = {}
+    for i, s in enumerate(specs):
+        if s.x_name not in xs:
+            xs[s.x_name] = wl.x_host(specs, s.x_name, 0).numpy().astype(np.float64)
+        sel = sorted(set([0, s.rows - 1] + rng.integers(0, s.rows, 6).tolist()))
+        y = W.y(i).cpu().numpy()[sel]
+        ref = np.array([oq.qgemv(s.fmt, synth.matrix(s.fmt, s.rows, s.cols, 0, s.name, r0=r, r1=r + 1).numpy(),
+                                 xs[s.x_name], 1, s.cols)[0] for r in sel])
+        assert_close(y, ref, what=s.name)
+        assert_close(y, ref, tol=1e-5, what=s.name + " (fp32 accuracy)")
+    assert W.weight_bytes == 614_629_376
