@@ -11,6 +11,8 @@
 #include "common.cuh"
 #include "host_common.h"
 #include "qgemv_api.cuh"
+#include "router.cuh"
+#include "moe_api.cuh"
 
 extern "C" const char* bqg_status_string(int status) {
   switch (status) {

@@ -7,19 +7,22 @@
 //
 // Design (B200):
 //  * The problem list is one byte stream.  Each CTA (one per SM) owns a contiguous,
-//    byte-balanced range of rows, cut into stages of whole rows (<= 24 KB).
-//  * A producer warp streams the stages with 1-D bulk copies (TMA) into a 4-deep shared
-//    memory ring, completing on mbarriers; rows keep their canonical byte layout (18/34-byte
-//    blocks), unaligned starts are handled by copying from the 16-byte boundary below.
-//  * 16 consumer warps: thread t owns "unit" p = t % P of every row (a pair of blocks, one
-//    block, or 32/64 int4 weights) and row group g = t / P.  Its 64 x values stay in
-//    registers for the whole matrix, so each weight byte is read once from shared memory and
-//    x costs no shared-memory traffic.
+//    byte-balanced range of rows (computed on the host), cut into stages of whole rows.
+//  * A producer warp streams the stages with 1-D bulk copies (TMA) into two 72 KB shared-memory
+//    slots (double buffering), completing on mbarriers.  Rows keep their canonical byte
+//    layout (18/34-byte blocks); an unaligned start is copied from the 16-byte boundary below.
+//  * 15 consumer warps.  A row is split into "units" (a pair of blocks, one block, or 32/64
+//    int4 weights); a row group of W = ceil(units/32) warps owns whole rows, lane l of its
+//    warp j handling unit 32j+l.  Each thread keeps its unit's 64 x values (fp32) in registers
+//    for the whole matrix: each weight byte is read once from shared memory and x costs no
+//    shared-memory traffic in the loop.  x itself is bulk-copied into shared memory by the
+//    producer one matrix ahead.  Two rows are processed together for more independent FMAs.
 //  * Dequantization uses byte permutes into the fp32 mantissa: a nibble q becomes the float
-//    128+q exactly (bits 0x43qq0000), an int8 becomes 2^23+128+q; sums are fp32 FMAs and the
-//    constant offset is removed with a per-unit sum of x.
-//  * Per-(row, unit) partials go to shared memory; one stage later each consumer warp sums a
-//    few rows in a fixed order (warp butterfly) and writes y.  Results are deterministic.
+//    128+q exactly (bits 0x43qq0000), an int8 becomes 2^23+128+q (then minus 2^23+128); sums
+//    are fp32 FMAs and the constant offset of the nibble formats is removed with a per-block
+//    sum of x.  All products are exact; only the fp32 sums round.
+//  * Each row is reduced with a warp butterfly (plus a fixed-order sum over the W warps of a
+//    group through shared memory), so results are deterministic.
 #pragma once
 
 #include "common.cuh"
@@ -29,14 +32,21 @@ namespace bqg {
 constexpr int kGemvConsumerWarps = 15;  // + 1 producer = 16 warps: 4 per SM sub-partition, 128 registers each
 constexpr int kGemvCompute = kGemvConsumerWarps * 32;       // consumer threads
 constexpr int kGemvThreads = kGemvCompute + 32;             // + one producer warp
-constexpr int kGemvStages = 4;
-constexpr int kGemvStageBytes = 24576;                      // payload of one stage (whole rows)
+#ifndef BQG_GEMV_STAGES
+#define BQG_GEMV_STAGES 2
+#endif
+#ifndef BQG_GEMV_STAGE_BYTES
+#define BQG_GEMV_STAGE_BYTES 73728
+#endif
+constexpr int kGemvStages = BQG_GEMV_STAGES;
+constexpr int kGemvStageBytes = BQG_GEMV_STAGE_BYTES;       // payload of one stage (whole rows)
 constexpr int kGemvStageAlloc = kGemvStageBytes + 48;       // + slack for unaligned head / tail
-constexpr int kGemvPartSlots = kGemvStages + 2;             // partial buffers (see reduce lag)
-constexpr int kGemvPartFloats = kGemvStageBytes / 16;       // units per stage <= bytes / 16
-constexpr size_t kGemvSmemBytes = size_t(kGemvStages) * kGemvStageAlloc +
-                                  size_t(kGemvPartSlots) * kGemvPartFloats * sizeof(float) +
-                                  2 * kGemvStages * sizeof(uint64_t);
+constexpr int kGemvMaxCols = BQG_MAX_COLS;
+constexpr int kGemvRedRows = 40;                            // rows per group per stage when W > 1
+constexpr size_t kGemvSmemBytes = size_t(kGemvStages) * kGemvStageAlloc +            // weight ring
+                                  size_t(kGemvMaxCols) * sizeof(float) +              // x staging
+                                  size_t(2 * kGemvConsumerWarps * kGemvRedRows) * sizeof(float) +
+                                  (2 * kGemvStages + 2) * sizeof(uint64_t);
 
 // Unit kinds: how many weights a consumer thread handles per row, and their byte size.
 enum UnitKind : int {
@@ -61,12 +71,21 @@ struct GemvProb {
   int scale_off;  // I4: byte offset of the fp32 row scales, else 0
 };
 
+constexpr int kGemvMaxGrid = 160;  // >= SM count of a B200 (148)
+
+// Rows owned by one CTA: from row r0 of problem p0 up to (not including) row r1 of problem
+// p1, in problem order.  Computed on the host so that the kernel does no 64-bit divisions.
+struct CtaRange {
+  int p0, r0, p1, r1;
+};
+
 template <int MAXP>
 struct GemvParams {
   int n;
   int pad;
   long long total_bytes;
   GemvProb p[MAXP];
+  CtaRange cta[kGemvMaxGrid];
 };
 
 __host__ __device__ constexpr int unit_bytes(int kind) {
@@ -75,29 +94,43 @@ __host__ __device__ constexpr int unit_bytes(int kind) {
 __host__ __device__ constexpr int unit_weights(int kind) {
   return (kind == kQ8Pair || kind == kQ4Pair || kind == kI4x64) ? 64 : 32;
 }
+__host__ __device__ constexpr bool is_i4(int kind) { return kind == kI4x64 || kind == kI4x32; }
+__host__ __device__ constexpr bool is_q8(int kind) { return kind == kQ8Pair || kind == kQ8One; }
+
+// Geometry shared by host and device: warps per row group, groups, rows per stage.
+__host__ __device__ constexpr int gemv_group_warps(int units) { return (units + 31) / 32; }
+__host__ __device__ constexpr int gemv_groups(int units) { return kGemvConsumerWarps / gemv_group_warps(units); }
+// The most whole rows that fit a stage, rounded down to a multiple of the number of groups so
+// that every group owns the same number of rows of each stage.  (groups * row_bytes <= 15 *
+// 32 * largest unit <= the stage size, so one row per group always fits.)
+__host__ __device__ constexpr int gemv_stage_rows(int units, int row_bytes) {
+  return (kGemvStageBytes / row_bytes) / gemv_groups(units) * gemv_groups(units);
+}
+static_assert(kGemvStageBytes >= kGemvCompute * 68, "a stage must hold one row per row group");
 
 // ---------------------------------------------------------------- dequant + dot helpers
 // Nibbles: bytes of `lo` hold elements 0,2,4,6 and bytes of `hi` elements 1,3,5,7 (each 0..15).
 // __byte_perm(v, 0x43, 0x4k55) = 0x43 << 24 | byte_k(v) << 16, the float 128 + byte_k(v).
-__device__ __forceinline__ void dot8_nib(uint32_t lo, uint32_t hi, const float* x, float& a0, float& a1) {
+__device__ __forceinline__ void dot8_nib(uint32_t lo, uint32_t hi, const float* x, float& a0, float& a1, float& a2,
+                                         float& a3) {
   a0 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4055u)), x[0], a0);
   a1 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4055u)), x[1], a1);
-  a0 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4155u)), x[2], a0);
-  a1 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4155u)), x[3], a1);
+  a2 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4155u)), x[2], a2);
+  a3 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4155u)), x[3], a3);
   a0 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4255u)), x[4], a0);
   a1 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4255u)), x[5], a1);
-  a0 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4355u)), x[6], a0);
-  a1 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4355u)), x[7], a1);
+  a2 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4355u)), x[6], a2);
+  a3 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4355u)), x[7], a3);
 }
 
 // Q4_0 word (8 unsigned nibbles, element 2m low / 2m+1 high nibble of byte m): adds (128+q)*x.
-__device__ __forceinline__ void dot8_q4(uint32_t w, const float* x, float& a0, float& a1) {
-  dot8_nib(w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu, x, a0, a1);
+__device__ __forceinline__ void dot8_q4(uint32_t w, const float* x, float& a0, float& a1, float& a2, float& a3) {
+  dot8_nib(w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu, x, a0, a1, a2, a3);
 }
 
 // int4 word (two's-complement nibbles): xor 8 maps q to q+8 in 0..15; adds (136+q)*x.
-__device__ __forceinline__ void dot8_i4(uint32_t w, const float* x, float& a0, float& a1) {
-  dot8_nib((w ^ 0x08080808u) & 0x0F0F0F0Fu, ((w >> 4) ^ 0x08080808u) & 0x0F0F0F0Fu, x, a0, a1);
+__device__ __forceinline__ void dot8_i4(uint32_t w, const float* x, float& a0, float& a1, float& a2, float& a3) {
+  dot8_nib((w ^ 0x08080808u) & 0x0F0F0F0Fu, ((w >> 4) ^ 0x08080808u) & 0x0F0F0F0Fu, x, a0, a1, a2, a3);
 }
 
 // Q8_0 word (4 int8): xor 0x80 gives q+128 in 0..255; __byte_perm(u, 0x4B, 0x455k) is the
@@ -111,148 +144,261 @@ __device__ __forceinline__ void dot4_q8(uint32_t w, const float* x, float& a0, f
   a1 = fmaf(__uint_as_float(__byte_perm(u, 0x4Bu, 0x4553u)) - off, x[3], a1);
 }
 
-// Partial dot product of one unit (bytes at `u` in shared memory) with the thread's x.
-// c0/c1: 136 * (sum of x over block 0 / block 1 of the unit) for the nibble formats.
-template <int KIND>
-__device__ __forceinline__ float unit_dot(const uint8_t* u, const float (&x)[64], float c0, float c1) {
+// Loads one unit's x values from xs into registers and the per-block offset constants of the
+// nibble formats: c[b] = 136 * sum of x over block b (sum_i (128+u_i) x_i - c = sum (u_i-8) x_i).
+__device__ __forceinline__ void build_x(int kind, const float* xs, float (&x)[64], float& c0, float& c1) {
+  const int uw = unit_weights(kind);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < uw / 4) v = reinterpret_cast<const float4*>(xs)[i];
+    x[4 * i] = v.x;
+    x[4 * i + 1] = v.y;
+    x[4 * i + 2] = v.z;
+    x[4 * i + 3] = v.w;
+  }
+  c0 = c1 = 0.f;
+  if (!is_q8(kind)) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s0 += x[i];
+#pragma unroll
+    for (int i = 32; i < 64; ++i) s1 += x[i];
+    c0 = 136.f * s0;
+    c1 = 136.f * s1;
+  }
+}
+
+// Partial dot products of the same unit of NR rows (shared-memory byte addresses u[n]) with
+// the thread's x registers.  Two rows at once give twice the independent FMA chains per thread.
+template <int KIND, int NR>
+__device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const float (&x)[64], float c0, float c1,
+                                          float (&out)[NR]) {
   if constexpr (KIND == kQ4Pair) {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(u);  // 4-byte aligned
-    uint32_t v[9];
+    uint32_t v[NR][9];
 #pragma unroll
-    for (int i = 0; i < 9; ++i) v[i] = w[i];
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+    for (int n = 0; n < NR; ++n)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      dot8_q4(__funnelshift_r(v[k], v[k + 1], 16), &x[8 * k], a0, a1);  // block A: bytes 2..17
-      dot8_q4(v[5 + k], &x[32 + 8 * k], b0, b1);                          // block B: bytes 20..35
-    }
-    const float dA = half_bits_to_float(v[0]);
-    const float dB = half_bits_to_float(v[4] >> 16);
-    return dA * ((a0 + a1) - c0) + dB * ((b0 + b1) - c1);
+      for (int i = 0; i < 9; ++i) v[n][i] = lds32(u[n] + 4 * i);  // 4-byte aligned
+    float a[NR][4], b[NR][4];
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[n][i] = b[n][i] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int n = 0; n < NR; ++n) {
+        dot8_q4(__funnelshift_r(v[n][m], v[n][m + 1], 16), &x[8 * m], a[n][0], a[n][1], a[n][2], a[n][3]);  // block A
+        dot8_q4(v[n][5 + m], &x[32 + 8 * m], b[n][0], b[n][1], b[n][2], b[n][3]);                          // block B
+      }
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+      out[n] = half_bits_to_float(v[n][0]) * (((a[n][0] + a[n][1]) + (a[n][2] + a[n][3])) - c0) +
+               half_bits_to_float(v[n][4] >> 16) * (((b[n][0] + b[n][1]) + (b[n][2] + b[n][3])) - c1);
   } else if constexpr (KIND == kQ4One) {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(u);
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~uintptr_t(3));
-    const uint32_t sh = uint32_t(a & 2) * 8;  // 0 or 16
-    uint32_t v[5];
+    uint32_t v[NR][5], sh[NR];
 #pragma unroll
-    for (int i = 0; i < 5; ++i) v[i] = w[i];
-    float a0 = 0.f, a1 = 0.f;
+    for (int n = 0; n < NR; ++n) {
+      const uint32_t w = u[n] & ~3u;
+      sh[n] = (u[n] & 2u) * 8;  // 0 or 16
 #pragma unroll
-    for (int k = 0; k < 4; ++k) dot8_q4(__funnelshift_rc(v[k], v[k + 1], 16 + sh), &x[8 * k], a0, a1);
-    const float d = half_bits_to_float(__funnelshift_r(v[0], v[1], sh));
-    return d * ((a0 + a1) - c0);
-  } else if constexpr (KIND == kQ8Pair) {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(u);
-    uint32_t v[17];
-#pragma unroll
-    for (int i = 0; i < 17; ++i) v[i] = w[i];
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      dot4_q8(__funnelshift_r(v[k], v[k + 1], 16), &x[4 * k], a0, a1);  // block A: bytes 2..33
-      dot4_q8(v[9 + k], &x[32 + 4 * k], b0, b1);                          // block B: bytes 36..67
+      for (int i = 0; i < 5; ++i) v[n][i] = lds32(w + 4 * i);
     }
-    const float dA = half_bits_to_float(v[0]);
-    const float dB = half_bits_to_float(v[8] >> 16);
-    return dA * (a0 + a1) + dB * (b0 + b1);
+    float a[NR][4];
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[n][i] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int n = 0; n < NR; ++n)
+        dot8_q4(__funnelshift_rc(v[n][m], v[n][m + 1], 16 + sh[n]), &x[8 * m], a[n][0], a[n][1], a[n][2], a[n][3]);
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+      out[n] = half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) *
+               (((a[n][0] + a[n][1]) + (a[n][2] + a[n][3])) - c0);
+  } else if constexpr (KIND == kQ8Pair) {
+    uint32_t v[NR][17];
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+#pragma unroll
+      for (int i = 0; i < 17; ++i) v[n][i] = lds32(u[n] + 4 * i);
+    float a[NR][2], b[NR][2];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) a[n][0] = a[n][1] = b[n][0] = b[n][1] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int n = 0; n < NR; ++n) {
+        dot4_q8(__funnelshift_r(v[n][m], v[n][m + 1], 16), &x[4 * m], a[n][0], a[n][1]);  // block A: bytes 2..33
+        dot4_q8(v[n][9 + m], &x[32 + 4 * m], b[n][0], b[n][1]);                          // block B: bytes 36..67
+      }
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+      out[n] = half_bits_to_float(v[n][0]) * (a[n][0] + a[n][1]) + half_bits_to_float(v[n][8] >> 16) * (b[n][0] + b[n][1]);
   } else if constexpr (KIND == kQ8One) {
-    const uintptr_t a = reinterpret_cast<uintptr_t>(u);
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(a & ~uintptr_t(3));
-    const uint32_t sh = uint32_t(a & 2) * 8;
-    uint32_t v[9];
+    uint32_t v[NR][9], sh[NR];
 #pragma unroll
-    for (int i = 0; i < 9; ++i) v[i] = w[i];
-    float a0 = 0.f, a1 = 0.f;
+    for (int n = 0; n < NR; ++n) {
+      const uint32_t w = u[n] & ~3u;
+      sh[n] = (u[n] & 2u) * 8;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) dot4_q8(__funnelshift_rc(v[k], v[k + 1], 16 + sh), &x[4 * k], a0, a1);
-    const float d = half_bits_to_float(__funnelshift_r(v[0], v[1], sh));
-    return d * (a0 + a1);
-  } else if constexpr (KIND == kI4x64) {
-    const uint4* w = reinterpret_cast<const uint4*>(u);  // 16-byte aligned
-    const uint4 p0 = w[0], p1 = w[1];
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-    dot8_i4(p0.x, &x[0], a0, a1);
-    dot8_i4(p0.y, &x[8], b0, b1);
-    dot8_i4(p0.z, &x[16], a0, a1);
-    dot8_i4(p0.w, &x[24], b0, b1);
-    dot8_i4(p1.x, &x[32], a0, a1);
-    dot8_i4(p1.y, &x[40], b0, b1);
-    dot8_i4(p1.z, &x[48], a0, a1);
-    dot8_i4(p1.w, &x[56], b0, b1);
-    return ((a0 + a1) + (b0 + b1)) - (c0 + c1);
-  } else {  // kI4x32
-    const uint4 p0 = *reinterpret_cast<const uint4*>(u);
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-    dot8_i4(p0.x, &x[0], a0, a1);
-    dot8_i4(p0.y, &x[8], b0, b1);
-    dot8_i4(p0.z, &x[16], a0, a1);
-    dot8_i4(p0.w, &x[24], b0, b1);
-    return ((a0 + a1) + (b0 + b1)) - c0;
+      for (int i = 0; i < 9; ++i) v[n][i] = lds32(w + 4 * i);
+    }
+    float a[NR][2];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) a[n][0] = a[n][1] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int n = 0; n < NR; ++n) dot4_q8(__funnelshift_rc(v[n][m], v[n][m + 1], 16 + sh[n]), &x[4 * m], a[n][0], a[n][1]);
+#pragma unroll
+    for (int n = 0; n < NR; ++n) out[n] = half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) * (a[n][0] + a[n][1]);
+  } else {  // int4 with per-row scale (applied by the caller): kI4x64 (8 words) or kI4x32 (4 words)
+    constexpr int NW = (KIND == kI4x64) ? 8 : 4;
+    uint32_t q[NR][8];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      const uint4 p0 = lds128(u[n]);  // 16-byte aligned
+      q[n][0] = p0.x; q[n][1] = p0.y; q[n][2] = p0.z; q[n][3] = p0.w;
+      if constexpr (NW == 8) {
+        const uint4 p1 = lds128(u[n] + 16);
+        q[n][4] = p1.x; q[n][5] = p1.y; q[n][6] = p1.z; q[n][7] = p1.w;
+      }
+    }
+    float a[NR][4], b[NR][4];
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[n][i] = b[n][i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < NW; k += 2)
+#pragma unroll
+      for (int n = 0; n < NR; ++n) {
+        dot8_i4(q[n][k], &x[8 * k], a[n][0], a[n][1], a[n][2], a[n][3]);
+        dot8_i4(q[n][k + 1], &x[8 * k + 8], b[n][0], b[n][1], b[n][2], b[n][3]);
+      }
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+      out[n] = (((a[n][0] + a[n][1]) + (a[n][2] + a[n][3])) + ((b[n][0] + b[n][1]) + (b[n][2] + b[n][3]))) - (c0 + c1);
   }
 }
 
 // ---------------------------------------------------------------- CTA work range
-// Rows of problem p owned by this CTA: those whose first byte lies in [lo, hi).
-__device__ __forceinline__ void owned_rows(const GemvProb& P, long long lo, long long hi, int& r0, int& r1) {
-  const long long rb = P.row_bytes;
-  long long a = lo - P.byte_start, b = hi - P.byte_start;
-  a = a <= 0 ? 0 : (a + rb - 1) / rb;
-  b = b <= 0 ? 0 : (b + rb - 1) / rb;
-  r0 = int(a < P.rows ? a : P.rows);
-  r1 = int(b < P.rows ? b : P.rows);
+// Rows [ra, rb) of problem pi owned by this CTA (empty when ra >= rb).
+__device__ __forceinline__ void cta_rows(const CtaRange& c, const GemvProb& P, int pi, int& ra, int& rb) {
+  ra = pi == c.p0 ? c.r0 : 0;
+  rb = pi < c.p1 ? P.rows : (pi == c.p1 ? c.r1 : 0);
+  if (pi < c.p0) rb = 0;
 }
 
-__device__ __forceinline__ int stage_rows(const GemvProb& P) {
-  const int sr = kGemvStageBytes / P.row_bytes;
-  return sr < 1 ? 1 : sr;
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// ---------------------------------------------------------------- consumer helpers
-struct StageRef {
-  int prob;  // -1: none
-  int r0, r1;
-  int slot_part;
-};
+// One matrix's rows [ra, rbnd) on the consumer side, specialised for its unit kind.
+// Returns false if a bounded wait gave up.
+template <int KIND, int MAXP>
+__device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi, int ra, int rbnd, uint8_t* ring,
+                                            float* xs, float* red, uint64_t* full, uint64_t* xfull, uint64_t* xfree,
+                                            uint64_t* empty, int& s, int& xs_n, float (&X)[64]) {
+  const GemvProb& P = prm.p[pi];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = P.units, row_bytes = P.row_bytes;
+  const int gw = gemv_group_warps(units);
+  const int groups = gemv_groups(units);
+  const int g = warp / gw, j = warp - g * gw;  // row group, warp within the group
+  const int p = 32 * j + lane;                 // this thread's unit
+  const bool in_group = g < groups;
+  const bool active = in_group && p < units;
+  constexpr int UB = unit_bytes(KIND), UW = unit_weights(KIND);
 
-template <int MAXP>
-__device__ __forceinline__ void reduce_stage(const GemvParams<MAXP>& prm, const StageRef& st, const float* parts,
-                                             int warp, int lane) {
-  if (st.prob < 0) return;
-  const GemvProb& P = prm.p[st.prob];
-  const float* part = parts + size_t(st.slot_part) * kGemvPartFloats;
-  const int nrows = st.r1 - st.r0;
-  for (int i = warp; i < nrows; i += kGemvConsumerWarps) {
-    float v = 0.f;
-    for (int q = lane; q < P.units; q += 32) v += part[i * P.units + q];
-    v = warp_sum(v);
-    if (lane == 0) {
-      const int row = st.r0 + i;
-      if (P.kind == kI4x64 || P.kind == kI4x32)
-        v *= __ldg(reinterpret_cast<const float*>(P.W + P.scale_off) + row);
-      P.y[row] = v;
+  // x was bulk-copied into xs by the producer; load this thread's x values into registers
+  if (!mbar_wait(xfull, uint32_t(xs_n) & 1u)) return false;
+  float c0 = 0.f, c1 = 0.f;
+  if (active) build_x(KIND, xs + size_t(p) * UW, X, c0, c1);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(xfree);
+  ++xs_n;
+
+  const uint32_t ring_s = smem_u32(ring);
+  const int sr = gemv_stage_rows(units, row_bytes);
+  for (int r0 = ra; r0 < rbnd; r0 += sr, ++s) {
+    const int r1 = min(r0 + sr, rbnd);
+    const int slot = s % kGemvStages;
+    if (!mbar_wait(&full[slot], uint32_t(s / kGemvStages) & 1u)) return false;
+    const uint32_t src_lo = uint32_t(reinterpret_cast<uintptr_t>(P.W) + size_t(r0) * row_bytes) & 15u;
+    const uint32_t base = ring_s + uint32_t(slot) * kGemvStageAlloc + src_lo + uint32_t(p) * UB;
+    const int nrows = r1 - r0;
+    const int par = s & 1;  // group reduction buffer of this stage (same in every warp)
+    int nmine = 0;
+    if (in_group) {
+      // group g owns rows g, g + groups, ... of the stage; two of them are done together
+      const float* scales = reinterpret_cast<const float*>(P.W + P.scale_off) + r0;
+      for (int i = g; i < nrows; i += 2 * groups) {
+        const bool two = i + groups < nrows;
+        float v[2] = {0.f, 0.f};
+        if (active) {
+          if (two) {
+            const uint32_t u2[2] = {base + uint32_t(i) * row_bytes, base + uint32_t(i + groups) * row_bytes};
+            units_dot<KIND, 2>(u2, X, c0, c1, v);
+          } else {
+            const uint32_t u1[1] = {base + uint32_t(i) * row_bytes};
+            float o1[1];
+            units_dot<KIND, 1>(u1, X, c0, c1, o1);
+            v[0] = o1[0];
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {  // two interleaved butterflies
+          v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+          v[1] += __shfl_xor_sync(0xffffffffu, v[1], o);
+        }
+        if (lane == 0) {
+          if (gw == 1) {
+            if (is_i4(KIND)) v[0] *= __ldg(scales + i);
+            P.y[r0 + i] = v[0];
+            if (two) {
+              if (is_i4(KIND)) v[1] *= __ldg(scales + i + groups);
+              P.y[r0 + i + groups] = v[1];
+            }
+          } else {
+            red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine] = v[0];
+            if (two) red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine + 1] = v[1];
+          }
+        }
+        nmine += two ? 2 : 1;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (gw > 1 && in_group) {
+      // fixed-order sum over the group's warps, by the group's first warp
+      named_bar_sync(2 + g, 32 * gw);
+      if (j == 0 && lane < nmine) {
+        float v = 0.f;
+        for (int jj = 0; jj < gw; ++jj) v += red[(par * kGemvConsumerWarps + g * gw + jj) * kGemvRedRows + lane];
+        const int row = r0 + g + lane * groups;
+        if (is_i4(KIND)) v *= __ldg(reinterpret_cast<const float*>(P.W + P.scale_off) + row);
+        P.y[row] = v;
+      }
     }
   }
-}
-
-// One unit's partial dot product, the format chosen at run time (uniform across the CTA).
-__device__ __forceinline__ float unit_dot_any(int kind, const uint8_t* u, const float (&x)[64], float c0, float c1) {
-  switch (kind) {
-    case kQ4Pair: return unit_dot<kQ4Pair>(u, x, c0, c1);
-    case kQ8Pair: return unit_dot<kQ8Pair>(u, x, c0, c1);
-    case kI4x64: return unit_dot<kI4x64>(u, x, c0, c1);
-    case kQ4One: return unit_dot<kQ4One>(u, x, c0, c1);
-    case kQ8One: return unit_dot<kQ8One>(u, x, c0, c1);
-    default: return unit_dot<kI4x32>(u, x, c0, c1);
-  }
+  return true;
 }
 
 template <int MAXP>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant__ GemvParams<MAXP> prm) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
-  float* parts = reinterpret_cast<float*>(smem + size_t(kGemvStages) * kGemvStageAlloc);
-  uint64_t* full = reinterpret_cast<uint64_t*>(parts + size_t(kGemvPartSlots) * kGemvPartFloats);
+  float* xs = reinterpret_cast<float*>(smem + size_t(kGemvStages) * kGemvStageAlloc);
+  float* red = xs + kGemvMaxCols;  // [2][kGemvConsumerWarps][kGemvRedRows]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kGemvConsumerWarps * kGemvRedRows);
   uint64_t* empty = full + kGemvStages;
+  uint64_t* xfull = empty + kGemvStages;  // x of the current problem landed in xs
+  uint64_t* xfree = xfull + 1;            // every consumer warp has read xs
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -261,24 +407,37 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kGemvConsumerWarps);
     }
+    mbar_init(xfull, 1);
+    mbar_init(xfree, kGemvConsumerWarps);
     fence_barrier_init();
   }
   __syncthreads();
 
-  const long long lo = prm.total_bytes * blockIdx.x / gridDim.x;
-  const long long hi = prm.total_bytes * (blockIdx.x + 1) / gridDim.x;
+  const CtaRange cr = prm.cta[blockIdx.x];
+  const int p_last = min(cr.p1, prm.n - 1);
 
   if (warp == kGemvConsumerWarps) {
     // ------------------------------------------------ producer warp (one elected lane)
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
+    const uint64_t pol_x = policy_evict_last();
     int s = 0;
+    int xs_n = 0;  // problems whose x has been staged
     bool ok = true;
-    for (int pi = 0; pi < prm.n && ok; ++pi) {
+    for (int pi = cr.p0; pi <= p_last && ok; ++pi) {
       const GemvProb& P = prm.p[pi];
       int ra, rbnd;
-      owned_rows(P, lo, hi, ra, rbnd);
-      const int sr = stage_rows(P);
+      cta_rows(cr, P, pi, ra, rbnd);
+      if (ra >= rbnd) continue;
+      // stage this problem's x once the consumers have read the previous one
+      if (xs_n > 0 && !mbar_wait(xfree, uint32_t(xs_n - 1) & 1u)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(xfull, uint32_t(P.cols) * 4u);
+      bulk_g2s(xs, P.x, uint32_t(P.cols) * 4u, xfull, pol_x);
+      ++xs_n;
+      const int sr = gemv_stage_rows(P.units, P.row_bytes);
       const uintptr_t wbeg = reinterpret_cast<uintptr_t>(P.W);
       const uintptr_t wend = wbeg + size_t(P.rows) * P.row_bytes;
       for (int r0 = ra; r0 < rbnd; r0 += sr, ++s) {
@@ -312,88 +471,33 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
       // wait (bounded) for the copies already issued so none lands after the CTA exits
       for (int q = (s > kGemvStages ? s - kGemvStages : 0); q < s; ++q)
         mbar_wait(&full[q % kGemvStages], uint32_t(q / kGemvStages) & 1u);
+      if (xs_n > 0) mbar_wait(xfull, uint32_t(xs_n - 1) & 1u);
     }
     return;
   }
 
   // ------------------------------------------------ consumer warps
-  const int t = warp * 32 + lane;
-  int s = 0;
-  StageRef prev{-1, 0, 0, 0};
-  float x[64];
-  for (int pi = 0; pi < prm.n; ++pi) {
+  int s = 0;     // stage counter (same sequence as the producer's, and in every consumer warp)
+  int xs_n = 0;  // problems whose x has been read
+  float X[64];
+  for (int pi = cr.p0; pi <= p_last; ++pi) {
     const GemvProb& P = prm.p[pi];
     int ra, rbnd;
-    owned_rows(P, lo, hi, ra, rbnd);
+    cta_rows(cr, P, pi, ra, rbnd);
     if (ra >= rbnd) continue;
-    const int kind = P.kind;
-    const int units = P.units;
-    const int groups = kGemvCompute / units;
-    const int g = t / units;
-    const int p = t - g * units;
-    const bool active = g < groups;
-    const int uw = unit_weights(kind);
-    const int ub = unit_bytes(kind);
-
-    // this thread's x values stay in registers for the whole matrix
-    float c0 = 0.f, c1 = 0.f;
-    if (active) {
-      const float4* xs = reinterpret_cast<const float4*>(P.x + size_t(p) * uw);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < uw / 4) v = __ldg(xs + i);
-        x[4 * i] = v.x;
-        x[4 * i + 1] = v.y;
-        x[4 * i + 2] = v.z;
-        x[4 * i + 3] = v.w;
-      }
-      if (kind != kQ8Pair && kind != kQ8One) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s0 += x[i];
-#pragma unroll
-        for (int i = 32; i < 64; ++i) s1 += x[i];
-        c0 = 136.f * s0;
-        c1 = 136.f * s1;
-      }
+    // Every consumer warp has finished the previous matrix (including the group reductions
+    // that read `red`): row groups may be composed differently from one matrix to the next.
+    named_bar_sync(1, kGemvCompute);
+    bool ok;
+    switch (P.kind) {
+      case kQ4Pair: ok = gemv_matrix<kQ4Pair, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
+      case kQ8Pair: ok = gemv_matrix<kQ8Pair, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
+      case kI4x64: ok = gemv_matrix<kI4x64, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
+      case kQ4One: ok = gemv_matrix<kQ4One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
+      case kQ8One: ok = gemv_matrix<kQ8One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
+      default: ok = gemv_matrix<kI4x32, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
     }
-
-    const int sr = stage_rows(P);
-    for (int r0 = ra; r0 < rbnd; r0 += sr, ++s) {
-      const int r1 = min(r0 + sr, rbnd);
-      const int slot = s % kGemvStages;
-      if (!mbar_wait(&full[slot], uint32_t(s / kGemvStages) & 1u)) return;
-      const uintptr_t src = reinterpret_cast<uintptr_t>(P.W) + size_t(r0) * P.row_bytes;
-      const uint8_t* base = ring + size_t(slot) * kGemvStageAlloc + (src & 15);
-      const int pslot = s % kGemvPartSlots;
-      float* part = parts + size_t(pslot) * kGemvPartFloats;
-      if (active) {
-        // rows of this stage owned by group g: (r - ra) % groups == g
-        int r = r0 + ((g - (r0 - ra) % groups) % groups + groups) % groups;
-        for (; r < r1; r += groups) {
-          const int i = r - r0;
-          part[i * units + p] = unit_dot_any(kind, base + size_t(i) * P.row_bytes + size_t(p) * ub, x, c0, c1);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
-      // reduce the previous stage once every consumer warp has released it
-      if (prev.prob >= 0) {
-        const int ps = s - 1;
-        if (!mbar_wait(&empty[ps % kGemvStages], uint32_t(ps / kGemvStages) & 1u)) return;
-        reduce_stage(prm, prev, parts, warp, lane);
-      }
-      prev.prob = pi;
-      prev.r0 = r0;
-      prev.r1 = r1;
-      prev.slot_part = pslot;
-    }
-  }
-  if (prev.prob >= 0) {
-    const int ps = s - 1;
-    if (!mbar_wait(&empty[ps % kGemvStages], uint32_t(ps / kGemvStages) & 1u)) return;
-    reduce_stage(prm, prev, parts, warp, lane);
+    if (!ok) return;
   }
 }
 

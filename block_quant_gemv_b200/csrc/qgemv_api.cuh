@@ -69,7 +69,41 @@ inline int launch_gemv(GemvParams<MAXP>& prm, long long total_rows, cudaStream_t
     total += (long long)prm.p[i].rows * prm.p[i].row_bytes;
   }
   prm.total_bytes = total;
-  const int grid = int(total_rows < info->sm_count ? total_rows : info->sm_count);
+  long long g = total_rows < info->sm_count ? total_rows : info->sm_count;
+  if (g > kGemvMaxGrid) g = kGemvMaxGrid;
+  const int grid = int(g);
+  // Byte-balanced split: CTA c owns the rows whose first byte lies in [c*T/G, (c+1)*T/G).
+  // first_row(b) = the first (problem, row) whose start byte is >= b; b grows with c, so one
+  // forward sweep over the problems serves all CTAs.
+  int sweep = 0;
+  auto first_row = [&](long long b, int& p, int& r) {
+    for (p = sweep; p < prm.n; ++p) {
+      const GemvProb& P = prm.p[p];
+      const long long end = P.byte_start + (long long)P.rows * P.row_bytes;
+      if (b < end) {
+        const long long off = b - P.byte_start;
+        r = off <= 0 ? 0 : int((off + P.row_bytes - 1) / P.row_bytes);
+        if (r < P.rows) {
+          sweep = p;
+          return;
+        }
+      }
+    }
+    sweep = p = prm.n;  // past the end
+    r = 0;
+  };
+  CtaRange prev{};
+  for (int c = 0; c <= grid; ++c) {
+    CtaRange cur{};
+    first_row(total * c / grid, cur.p0, cur.r0);
+    if (c > 0) {
+      prm.cta[c - 1].p0 = prev.p0;
+      prm.cta[c - 1].r0 = prev.r0;
+      prm.cta[c - 1].p1 = cur.p0;
+      prm.cta[c - 1].r1 = cur.r0;
+    }
+    prev = cur;
+  }
   k_qgemv<MAXP><<<grid, kGemvThreads, kGemvSmemBytes, stream>>>(prm);
   return launch_status();
 }

@@ -40,6 +40,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* Only the functions below are exported; everything else in the library has hidden visibility. */
+#if defined(__GNUC__)
+#define BQG_API __attribute__((visibility("default")))
+#else
+#define BQG_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -64,24 +71,25 @@ enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 #define BQG_MAX_BATCH 256        /* largest descriptor count of one qgemv_batched call     */
 #define BQG_MAX_EXPERTS 256      /* largest n_experts of the router / MoE calls            */
 #define BQG_MAX_TOPK 8           /* largest k of the router / MoE calls                    */
+#define BQG_MAX_MOE_COLS 8192    /* largest hidden / inter / shared_inter of moe_forward   */
 
 /* Device-side error bits, reported by bqg_device_errors(). */
 #define BQG_DEVERR_TIMEOUT 0x1   /* a bounded in-kernel wait gave up (the kernel returned early) */
 #define BQG_DEVERR_EXPERT_ID 0x2 /* moe_forward met an expert id outside [0, n_experts); skipped */
 
 /* Human-readable name of a bqg_status value (static string, never NULL). */
-const char* bqg_status_string(int status);
+BQG_API const char* bqg_status_string(int status);
 
 /* Library version as 10000*major + 100*minor + patch. */
-int bqg_version(void);
+BQG_API int bqg_version(void);
 
 /* Byte size of a rows x cols matrix in the canonical layout of `fmt` (see above), or 0 when
  * the format is unknown or the shape is invalid (rows < 1, cols < 32 or cols % 32 != 0). */
-size_t bqg_weight_bytes(int fmt, int rows, int cols);
+BQG_API size_t bqg_weight_bytes(int fmt, int rows, int cols);
 
 /* Reads and clears the device-side error bits (BQG_DEVERR_*) of the current device.
  * Synchronises the device.  Returns BQG_OK or BQG_ERR_CUDA; *bits receives the bits. */
-int bqg_device_errors(int* bits);
+BQG_API int bqg_device_errors(int* bits);
 
 /* ---------------------------------------------------------------- a1, a2, a3: one GEMV
  * qgemv: y = W x for one quantized matrix.
@@ -92,7 +100,7 @@ int bqg_device_errors(int* bits);
  *   x     device fp32 [cols], 16-byte aligned.   y  device fp32 [rows], 4-byte aligned.
  *   rows  >= 1.   cols  multiple of 32, 32 <= cols <= BQG_MAX_COLS.
  *   y must not overlap W or x.  Results are deterministic (fixed summation order). */
-int qgemv(int fmt, const void* W, const float* x, float* y, int rows, int cols, void* stream);
+BQG_API int qgemv(int fmt, const void* W, const float* x, float* y, int rows, int cols, void* stream);
 
 /* ---------------------------------------------------------------- a4: a decode step's GEMVs
  * qgemv_batched: every descriptor's y = W x, in ONE persistent launch that streams all the
@@ -112,10 +120,80 @@ typedef struct {
   float* y;
 } bqg_gemv_desc;
 
-int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream);
+BQG_API int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream);
+
+/* ---------------------------------------------------------------- a5: router logits
+ * moe_router_logits: logits[t, e] = sum_h R[e, h] x[t, h] in fp32.
+ *   Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (router choosing experts per token).
+ *   R       device fp32 [n_experts x hidden], 16-byte aligned.
+ *   x       device fp32 [tokens x hidden], 16-byte aligned.   logits  device fp32 [tokens x n_experts].
+ *   tokens >= 1, 1 <= n_experts <= BQG_MAX_EXPERTS, hidden multiple of 4, 4 <= hidden <= BQG_MAX_COLS. */
+BQG_API int moe_router_logits(const float* R, const float* x, float* logits, int tokens, int n_experts,
+                      int hidden, void* stream);
+
+/* ---------------------------------------------------------------- a6: softmax, top-k, renormalise
+ * moe_router_topk: per token, idx[t, 0..k-1] = the k experts with the largest logits in
+ * descending order, an exact tie going to the lower expert index; weights[t, j] =
+ * p[idx[t, j]] / sum_j' p[idx[t, j']] with p = softmax(logits[t, :]) over all n_experts.
+ *   Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (top-8 of 128); colibri wiki summary,
+ *   "핵심 아이디어" (256 routed experts); Camelid README, "Windows bring-up, perf & GPU"
+ *   (an exact expert-probability tie goes to the lower index).
+ *   logits  device fp32 [tokens x n_experts] (finite values).
+ *   idx     device int32 [tokens x k].   weights  device fp32 [tokens x k].
+ *   tokens >= 1, 1 <= k <= BQG_MAX_TOPK, k <= n_experts <= BQG_MAX_EXPERTS. */
+BQG_API int moe_router_topk(const float* logits, int tokens, int n_experts, int k, int32_t* idx,
+                    float* weights, void* stream);
+
+/* ---------------------------------------------------------------- a7-a10: the MoE layer
+ * One routed-expert layer.  Expert e's gate matrix starts at gate + e * gate_stride bytes
+ * (likewise up and down).  gate and up are [inter x hidden]; down is [hidden x inter]; all
+ * three in expert_fmt.  The optional shared expert (s_gate == NULL means none) has
+ * s_gate, s_up [shared_inter x hidden] and s_down [hidden x shared_inter] in shared_fmt.
+ * act selects the gated activation for both: GeGLU with the tanh form of GELU, or SwiGLU. */
+typedef struct {
+  int n_experts;     /* 1..BQG_MAX_EXPERTS                          */
+  int top_k;         /* 1..BQG_MAX_TOPK, <= n_experts               */
+  int hidden;        /* multiple of 32, <= BQG_MAX_MOE_COLS         */
+  int inter;         /* multiple of 32, <= BQG_MAX_MOE_COLS         */
+  int expert_fmt;    /* BQG_Q8_0, BQG_Q4_0 or BQG_I4_ROW            */
+  int act;           /* BQG_ACT_GELU_TANH or BQG_ACT_SILU           */
+  const void* gate;  /* device, 16-byte aligned                      */
+  const void* up;
+  const void* down;
+  size_t gate_stride; /* bytes between consecutive experts, multiple of 16 */
+  size_t up_stride;
+  size_t down_stride;
+  int shared_inter;  /* multiple of 32, <= BQG_MAX_MOE_COLS (ignored without a shared expert) */
+  int shared_fmt;
+  const void* s_gate; /* NULL: no shared expert */
+  const void* s_up;
+  const void* s_down;
+} bqg_moe_layer;
+
+/* Bytes of device workspace moe_forward needs for `tokens` tokens (0 on invalid arguments). */
+BQG_API size_t moe_workspace_size(const bqg_moe_layer* L, int tokens);
+
+/* moe_forward: y[t] = sum_{j<k} w[t, j] * FFN_{idx[t, j]}(x[t]) (+ shared FFN(x[t])), where
+ * FFN(v) = down (act(gate v) * (up v)).  Tokens are grouped by expert on the device so that
+ * each touched expert's weights are streamed once per call and applied to all its tokens.
+ * The per-(token, slot) outputs are summed in slot order j = 0..k-1, then the shared output
+ * is added, so results are deterministic.
+ *   Source: Camelid README, "Gemma 4" (dense shared-expert + sparse top-8 branch); TurboFieldfare
+ *   wiki, "메모리·전문가 스트리밍" (routed experts split from the shared branch, each expert read
+ *   reused by every row routed to it).
+ *   L          HOST pointer to the layer description.
+ *   x          device fp32 [tokens x hidden], 16-byte aligned.
+ *   idx, w     device int32 / fp32 [tokens x top_k] (as written by moe_router_topk).
+ *   y          device fp32 [tokens x hidden], must not overlap x.
+ *   workspace  device, >= moe_workspace_size(L, tokens) bytes, 256-byte aligned; contents
+ *              are scratch, overwritten by the call.
+ *   An expert id outside [0, n_experts) is skipped and sets BQG_DEVERR_EXPERT_ID. */
+BQG_API int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
+                float* y, int tokens, void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }
 #endif
 
 #endif /* BQG_H */
+

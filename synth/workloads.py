@@ -14,7 +14,7 @@ Nothing here computes any part of the method; it only draws inputs (see synth).
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from typing import List
+from typing import List, Optional
 
 import torch
 
@@ -107,3 +107,97 @@ def x_host(specs: List[GemvSpec], name: str, seed: int) -> torch.Tensor:
     """The host copy of one named input vector (identical to the workload's device copy)."""
     cols = next(s.cols for s in specs if s.x_name == name)
     return normal_f32(seed, stream_id(name), cols)
+
+
+# ---------------------------------------------------------------- MoE layers
+@dataclass
+class MoESpec:
+    """Shape of one routed-expert layer (see the MoE configurations)."""
+    name: str
+    n_experts: int
+    top_k: int
+    hidden: int
+    inter: int
+    expert_fmt: int
+    act: int                      # 1 GeGLU (tanh GELU), 2 SwiGLU
+    shared_inter: int = 0
+    shared_fmt: int = 0
+    router: bool = True           # fp32 router matrix R ~ N(0, 0.02); else logits are given
+
+    def mat_bytes(self, which: str) -> int:
+        if which == "down":
+            return weight_bytes(self.expert_fmt, self.hidden, self.inter)
+        return weight_bytes(self.expert_fmt, self.inter, self.hidden)
+
+    def shared_bytes(self, which: str) -> int:
+        if which == "down":
+            return weight_bytes(self.shared_fmt, self.hidden, self.shared_inter)
+        return weight_bytes(self.shared_fmt, self.shared_inter, self.hidden)
+
+
+# Gemma-4-26B-A4B-like layer: hidden 2816, 128 experts, top-8, GeGLU experts of 704 in Q4_0,
+# shared dense GeGLU expert of 2112 in Q8_0, fp32 router 128 x 2816.
+GEMMA_MOE = MoESpec("gemma_moe", 128, 8, 2816, 704, FMT_Q4_0, 1, 2112, FMT_Q8_0, True)
+# GLM-style layer: hidden 6144, 256 experts, top-8, SwiGLU experts of 2048 in packed int4 with
+# fp32 row scales, no shared expert, logits given (N(0,1)); 8 such layers are stacked.
+GLM_MOE = MoESpec("glm_moe", 256, 8, 6144, 2048, FMT_I4_ROW, 2, 0, 0, False)
+GLM_LAYERS = 8
+
+
+def _align16(n: int) -> int:
+    return (n + 15) // 16 * 16
+
+
+def expert_matrix(spec: MoESpec, seed: int, layer: int, e: int, which: str, device="cpu") -> torch.Tensor:
+    rows, cols = (spec.hidden, spec.inter) if which == "down" else (spec.inter, spec.hidden)
+    return matrix(spec.expert_fmt, rows, cols, seed, f"{spec.name}/L{layer}/E{e}/{which}", device=device)
+
+
+def shared_matrix(spec: MoESpec, seed: int, layer: int, which: str, device="cpu") -> torch.Tensor:
+    rows, cols = (spec.hidden, spec.shared_inter) if which == "down" else (spec.shared_inter, spec.hidden)
+    return matrix(spec.shared_fmt, rows, cols, seed, f"{spec.name}/L{layer}/shared/{which}", device=device)
+
+
+@dataclass
+class MoETensors:
+    spec: MoESpec
+    gate: torch.Tensor            # [E * stride] bytes, expert e at e * stride
+    up: torch.Tensor
+    down: torch.Tensor
+    gate_stride: int
+    up_stride: int
+    down_stride: int
+    shared: Optional[tuple] = None  # (s_gate, s_up, s_down)
+    R: Optional[torch.Tensor] = None
+
+
+def build_moe_layer(spec: MoESpec, seed: int, layer: int = 0, device="cuda") -> MoETensors:
+    """All experts of one layer stacked per family (each expert padded to 16 bytes)."""
+    strides = {w: _align16(spec.mat_bytes(w)) for w in ("gate", "up", "down")}
+    fam = {}
+    for w in ("gate", "up", "down"):
+        t = torch.zeros(spec.n_experts * strides[w], dtype=torch.uint8, device=device)
+        n = spec.mat_bytes(w)
+        for e in range(spec.n_experts):
+            t[e * strides[w]: e * strides[w] + n] = expert_matrix(spec, seed, layer, e, w, device=device)
+        fam[w] = t
+    shared = None
+    if spec.shared_inter:
+        shared = tuple(shared_matrix(spec, seed, layer, w, device=device) for w in ("gate", "up", "down"))
+    R = None
+    if spec.router:
+        R = normal_f32(seed, stream_id(f"{spec.name}/L{layer}/router"), spec.n_experts * spec.hidden,
+                       std=0.02).view(spec.n_experts, spec.hidden).to(device)
+    return MoETensors(spec, fam["gate"], fam["up"], fam["down"], strides["gate"], strides["up"], strides["down"],
+                      shared, R)
+
+
+def moe_tokens(spec: MoESpec, seed: int, tokens: int) -> torch.Tensor:
+    """Host fp32 activations x ~ N(0, 1), [tokens, hidden]."""
+    return normal_f32(seed, stream_id(f"{spec.name}/x/T{tokens}"), tokens * spec.hidden).view(tokens, spec.hidden)
+
+
+def moe_logits(spec: MoESpec, seed: int, layer: int, tokens: int) -> torch.Tensor:
+    """Host fp32 router logits ~ N(0, 1), [tokens, n_experts] (for layers whose logits are given)."""
+    return normal_f32(seed, stream_id(f"{spec.name}/L{layer}/logits/T{tokens}"),
+                      tokens * spec.n_experts).view(tokens, spec.n_experts)

@@ -24,13 +24,13 @@ def L():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+    names = re.findall(r"^\s*(?:BQG_API\s+)?(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
 def test_header_declares_the_api():
     names = declared_functions()
-    for want in ["qgemv", "qgemv_batched", "bqg_status_string", "bqg_weight_bytes",
+    for want in ["qgemv", "qgemv_batched", "moe_router_logits", "moe_router_topk", "bqg_status_string", "bqg_weight_bytes",
                  "bqg_device_errors", "bqg_version"]:
         assert want in names
 
@@ -94,3 +94,24 @@ def test_valid_call_without_gpu_fails_loudly(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.lib().qgemv(2, 0x10000, 0x10000, 0x10000, 4, 32, None) in (-6, -7)
+
+
+def test_router_argument_errors(L):
+    lg, tk = L.lib().moe_router_logits, L.lib().moe_router_topk
+    A = 0x10000
+    assert lg(None, A, A, 1, 128, 2816, None) == -1
+    assert lg(A, A, A, 1, 300, 2816, None) == -8          # more than 256 experts
+    assert lg(A, A, A, 1, 128, 2818, None) == -3          # hidden % 4
+    assert lg(A + 4, A, A, 1, 128, 2816, None) == -4
+    assert tk(A, 1, 128, 9, A, A, None) == -8              # k above 8
+    assert tk(A, 1, 4, 8, A, A, None) == -3                # k > n_experts
+    assert tk(A, 0, 128, 8, A, A, None) == -1
+    assert tk(A + 2, 1, 128, 8, A, A, None) == -4
+
+
+def test_only_the_c_abi_is_exported(L):
+    """Internal symbols (kernels, per-device caches) are hidden, so two copies of the library
+    loaded in one process cannot share internal state."""
+    out = subprocess.run(["nm", "-D", "--defined-only", L.library_path()], capture_output=True, text=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.split()[1:2] and line.split()[1] in "TBDVWu")
+    assert exported <= set(declared_functions()) | {"_init", "_fini"}, exported - set(declared_functions())
