@@ -89,6 +89,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// Orders this thread's (and, through the preceding barrier, the CTA's) generic-proxy shared
+// memory accesses before later async-proxy (bulk copy) writes to the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- bulk copies (TMA, 1-D)
 // Global -> shared copy of `bytes` bytes (multiple of 16; both addresses 16-byte aligned),
 // completing as transaction bytes on `bar`.  The L2 policy marks the streamed weights

@@ -66,12 +66,13 @@ inline int check_layer(const bqg_moe_layer* L) {
 }
 
 // Matrix family description for the grouped kernel.
-inline MoeMat moe_mat(int fmt, const void* base, size_t stride, int rows, int cols) {
+inline int moe_mat(int fmt, const void* base, size_t stride, int rows, int cols, MoeMat* out) {
   MoeMat M{};
   GemvProb P{};
   // reuse the GEMV unit selection (kind, row bytes, units, scale offset)
-  make_gemv_prob(fmt, base, reinterpret_cast<const float*>(base), reinterpret_cast<float*>(const_cast<void*>(base)),
-                 rows, cols, &P);
+  const int st = make_gemv_prob(fmt, base, reinterpret_cast<const float*>(base),
+                                reinterpret_cast<float*>(const_cast<void*>(base)), rows, cols, &P);
+  if (st != BQG_OK) return st;
   M.base = static_cast<const uint8_t*>(base);
   M.stride = (long long)stride;
   M.rows = rows;
@@ -80,7 +81,8 @@ inline MoeMat moe_mat(int fmt, const void* base, size_t stride, int rows, int co
   M.row_bytes = P.row_bytes;
   M.units = P.units;
   M.scale_off = P.scale_off;
-  return M;
+  *out = M;
+  return BQG_OK;
 }
 
 // Lanes per row, rows per tile and tokens per token tile for one matrix family.
@@ -154,15 +156,15 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
     P.act = L->act;
     P.gateup = phase == 0;
     if (phase == 0) {
-      P.m0 = bqg::moe_mat(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden);
-      P.m1 = bqg::moe_mat(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden);
+      if ((st = bqg::moe_mat(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden, &P.m0)) != BQG_OK) return st;
+      if ((st = bqg::moe_mat(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden, &P.m1)) != BQG_OK) return st;
       P.nmat = 2;
       P.xin = x;
       P.xin_stride = L->hidden;
       P.out = h;
       P.out_stride = L->inter;
     } else {
-      P.m0 = bqg::moe_mat(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter);
+      if ((st = bqg::moe_mat(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, &P.m0)) != BQG_OK) return st;
       P.m1 = P.m0;
       P.nmat = 1;
       P.xin = h;
@@ -175,12 +177,14 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
     if (has_shared) {
       P.s_present = 1;
       if (phase == 0) {
-        P.s0 = bqg::moe_mat(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden);
-        P.s1 = bqg::moe_mat(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden);
+        if ((st = bqg::moe_mat(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden, &P.s0)) != BQG_OK) return st;
+        if ((st = bqg::moe_mat(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden, &P.s1)) != BQG_OK) return st;
+        P.s_xin = x;
+        P.s_xin_stride = L->hidden;
         P.s_out = hs;
         P.s_out_stride = L->shared_inter;
       } else {
-        P.s0 = bqg::moe_mat(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter);
+        if ((st = bqg::moe_mat(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, &P.s0)) != BQG_OK) return st;
         P.s1 = P.s0;
         P.s_xin = hs;
         P.s_xin_stride = L->shared_inter;

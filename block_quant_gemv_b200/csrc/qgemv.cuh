@@ -319,8 +319,7 @@ __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi,
   if (!mbar_wait(xfull, uint32_t(xs_n) & 1u)) return false;
   float c0 = 0.f, c1 = 0.f;
   if (active) build_x(KIND, xs + size_t(p) * UW, X, c0, c1);
-  __syncwarp();
-  if (lane == 0) mbar_arrive(xfree);
+  mbar_arrive(xfree);
   ++xs_n;
 
   const uint32_t ring_s = smem_u32(ring);
@@ -408,7 +407,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
       mbar_init(&empty[i], kGemvConsumerWarps);
     }
     mbar_init(xfull, 1);
-    mbar_init(xfree, kGemvConsumerWarps);
+    mbar_init(xfree, kGemvCompute);  // every consumer thread releases its own reads of xs
     fence_barrier_init();
   }
   __syncthreads();
@@ -434,6 +433,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
         ok = false;
         break;
       }
+      fence_proxy_async_smem();
       mbar_arrive_expect_tx(xfull, uint32_t(P.cols) * 4u);
       bulk_g2s(xs, P.x, uint32_t(P.cols) * 4u, xfull, pol_x);
       ++xs_n;
@@ -447,6 +447,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
           ok = false;
           break;
         }
+        fence_proxy_async_smem();
         const uintptr_t src = wbeg + size_t(r0) * P.row_bytes;
         const uintptr_t end = src + size_t(r1 - r0) * P.row_bytes;
         const uintptr_t a0 = src & ~uintptr_t(15);
