@@ -20,7 +20,7 @@ __all__ = [
     "Q8_0", "Q4_0", "I4_ROW", "ACT_GELU_TANH", "ACT_SILU", "BQGError",
     "lib", "library_path", "bqg_status_string", "bqg_weight_bytes", "bqg_device_errors",
     "qgemv", "qgemv_batched", "GemvBatch", "qgemm_prefill", "moe_router_logits",
-    "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward",
+    "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward", "moe_forward_noalloc",
 ]
 
 Q8_0, Q4_0, I4_ROW = 1, 2, 3
@@ -67,6 +67,7 @@ _SIGNATURES = {
     "moe_router_topk": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_workspace_size": (_sz, [ctypes.POINTER(MoELayerC), _i]),
     "moe_forward": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+    "moe_forward_noalloc": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp]),
 }
 
 
@@ -262,4 +263,22 @@ def moe_forward(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Te
     _need_cuda("workspace", workspace, torch.uint8)
     _check(lib().moe_forward(ctypes.byref(layer.c), _ptr(x), _ptr(idx), _ptr(w), _ptr(y), tokens,
                              _ptr(workspace), workspace.numel(), _stream(x)), "moe_forward")
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 24 << 20
+
+
+def moe_forward_noalloc(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor,
+                        y: torch.Tensor) -> torch.Tensor:
+    """moe_forward with the library's fixed scratch array instead of a caller workspace: for
+    callers that cannot allocate device memory around the call.  y must be preallocated; calls
+    that could overlap on the GPU share the scratch and must not be issued."""
+    _need_cuda("x", x, torch.float32)
+    _need_cuda("idx", idx, torch.int32)
+    _need_cuda("w", w, torch.float32)
+    _need_cuda("y", y, torch.float32)
+    tokens = x.numel() // layer.hidden
+    _check(lib().moe_forward_noalloc(ctypes.byref(layer.c), _ptr(x), _ptr(idx), _ptr(w), _ptr(y), tokens, _stream(x)),
+           "moe_forward_noalloc")
     return y

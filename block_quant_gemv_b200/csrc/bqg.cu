@@ -41,3 +41,41 @@ extern "C" int bqg_device_errors(int* bits) {
   *bits = v;
   return BQG_OK;
 }
+
+// ---------------------------------------------------------------- moe_forward without allocation
+// Some callers cannot allocate device memory around a call: code running inside a CUDA graph
+// being captured by someone else, real-time or embedded runtimes that forbid cudaMalloc after
+// start-up, and plugins handed only input and output buffers by a host framework that owns
+// all allocations.  For them moe_forward_noalloc runs the same MoE kernels with their scratch
+// (routing tables and per-pair intermediate rows) in the fixed array below, which is part of
+// the library image: every GPU that loads the library holds these bytes until the process
+// exits, and no call allocates or frees anything.
+static __device__ __align__(256) uint8_t g_moe_noalloc_scratch[BQG_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_moe_noalloc_scratch per device.  In host code the array's name is only a
+// host-side stand-in, so the address must be asked from the runtime (once per device).
+std::atomic<void*> g_noalloc_scratch_ptr[bqg::kMaxDevices];
+}  // namespace
+
+extern "C" int moe_forward_noalloc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
+                                   float* y, int tokens, void* stream) {
+  const size_t need = moe_workspace_size(L, tokens);
+  if (need == 0) {
+    const int st = bqg::check_layer(L);
+    return st != BQG_OK ? st : BQG_ERR_ARG;
+  }
+  if (need > size_t(BQG_NOALLOC_SCRATCH_BYTES)) return BQG_ERR_LIMIT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= bqg::kMaxDevices) return BQG_ERR_CUDA;
+  void* scratch = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (scratch == nullptr) {
+    // first call on this device: look the array up with this device current
+    if (cudaGetSymbolAddress(&scratch, g_moe_noalloc_scratch) != cudaSuccess || scratch == nullptr)
+      return BQG_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev].store(scratch, std::memory_order_release);
+  }
+  // Every region of the scratch is written by the kernels before it is read, so nothing has to
+  // be cleared between calls.
+  return moe_forward(L, x, idx, w, y, tokens, scratch, size_t(BQG_NOALLOC_SCRATCH_BYTES), stream);
+}

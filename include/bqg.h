@@ -191,6 +191,25 @@ BQG_API size_t moe_workspace_size(const bqg_moe_layer* L, int tokens);
 BQG_API int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
                 float* y, int tokens, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- moe_forward without allocation
+ * moe_forward_noalloc: the same computation as moe_forward, for callers that cannot allocate
+ * device memory around the call (a CUDA graph captured by another component, a runtime that
+ * forbids cudaMalloc after start-up, a plugin that only receives input and output buffers).
+ * The pages describe no such call; it has no counterpart there.
+ * Its scratch lives in a fixed array of BQG_NOALLOC_SCRATCH_BYTES inside the library image,
+ * held by every GPU that loads the library until the process exits; the call allocates and
+ * frees nothing.  Arguments are those of moe_forward without the workspace.
+ *   - Returns BQG_ERR_LIMIT when moe_workspace_size(L, tokens) exceeds BQG_NOALLOC_SCRATCH_BYTES.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress);
+ *     make that first call before any stream capture that includes it.
+ *   - All calls on a device share the one array: calls that may overlap on the GPU (different
+ *     streams without ordering between them) race and must not be issued.  Calls ordered on one
+ *     stream are fine; the array keeps the last call's contents, and every region the kernels read
+ *     is written first by the same call, so nothing needs clearing. */
+#define BQG_NOALLOC_SCRATCH_BYTES (24u << 20)
+BQG_API int moe_forward_noalloc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
+                                float* y, int tokens, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
