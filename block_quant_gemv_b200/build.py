@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     cmd = [nvcc_path(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "bqg.cu"), "-o", LIB + ".tmp", "-lcuda"]
+           os.path.join(CSRC, "bqg.cu"), "-o", LIB + ".tmp"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     log = res.stdout + res.stderr
     with open(os.path.join(PKG, "build.log"), "w") as f:

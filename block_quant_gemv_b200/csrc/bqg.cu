@@ -13,6 +13,7 @@
 #include "qgemv_api.cuh"
 #include "router.cuh"
 #include "moe_api.cuh"
+#include "prefill.cuh"
 
 extern "C" const char* bqg_status_string(int status) {
   switch (status) {

@@ -1,0 +1,477 @@
+// Prefill-chunk GEMM with Q4_0 weights on the 5th-generation tensor cores (tcgen05):
+//   Y[t, n] = sum_k X[t, k] * W[n, k],   X fp16 [tokens x k] (tokens <= 128), W Q4_0 [n x k],
+//   fp32 accumulation in tensor memory, Y fp16 (round to nearest even).
+//
+// Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (prefill in chunks of at most 128 tokens,
+// so that each weight read is reused by every prompt row of the chunk); Camelid README,
+// "Engine status" (GPU-resident single-shot prefill).
+//
+// One CTA computes a 128 (tokens, padded) x 128 (output features) tile over a range of k.
+//   warp 0     TMA: X tiles (128 rows x 64 k, fp16, 128-byte swizzle) and raw Q4_0 row chunks
+//              (128 rows x 144 bytes = 256 k) into shared-memory rings.
+//   warp 1     allocates the 128-column fp32 accumulator in tensor memory and issues the
+//              tcgen05.mma instructions (M=128, N=128, K=16 each, both operands K-major in
+//              shared memory); tcgen05.commit frees each stage when its MMAs have read it.
+//   warps 2-5  dequantize: each thread owns one weight row, turns 64 Q4_0 weights into fp16
+//              (q - 8) * d (exact nibble, one rounding of the product) and writes them into the
+//              B stage in the swizzled K-major layout the MMA reads; after the last stage they
+//              read the accumulator rows (one warp per 32 tensor-memory lanes), round to fp16
+//              and store Y.
+// With several k-splits per tile (small n), the CTAs of one tile form a thread-block cluster
+// and the partial tiles are summed through distributed shared memory in a fixed order.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "host_common.h"
+
+namespace bqg {
+
+constexpr int kPfThreads = 192;           // 6 warps
+constexpr int kPfTileN = 128;             // output features per CTA
+constexpr int kPfTileM = 128;             // tokens per CTA (MMA M)
+constexpr int kPfStageK = 64;             // k per stage (one 128-byte swizzle row of fp16)
+constexpr int kPfStages = 4;              // A/B stage ring depth
+constexpr int kPfRawK = 256;              // k per raw Q4_0 chunk (8 blocks = 144 bytes per row)
+constexpr int kPfRawBytesRow = kPfRawK / 32 * 18;  // 144
+constexpr int kPfRawStages = 3;
+constexpr int kPfABytes = kPfTileM * kPfStageK * 2;  // 16 KB
+constexpr int kPfBBytes = kPfTileN * kPfStageK * 2;  // 16 KB
+constexpr int kPfRawBytes = kPfTileN * kPfRawBytesRow;  // 18 KB
+constexpr int kPfMaxSplit = 8;            // k-splits per tile (cluster size)
+// smem: [A ring | B ring] (1024-aligned), raw ring, barriers, tmem address; + 1 KB alignment slack
+constexpr size_t kPfSmemBytes = 1024 + size_t(kPfStages) * (kPfABytes + kPfBBytes) +
+                                size_t(kPfRawStages) * kPfRawBytes + 256;
+
+struct PfParams {
+  void* Y;           // fp16 [tokens x n]
+  int tokens, n, k;
+  int ksplit;        // CTAs (cluster size) sharing one output tile
+  int kchunks;       // k / kPfRawK; split s owns chunks [s*kchunks/ksplit, (s+1)*kchunks/ksplit)
+};
+
+// ---------------------------------------------------------------- tcgen05 / TMA helpers
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  // K-major operand, 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFF);       // start address
+  d |= uint64_t(1) << 16;                     // leading byte offset (unused for swizzled K-major)
+  d |= uint64_t(1024 >> 4) << 32;             // stride byte offset: 8 rows x 128 bytes
+  d |= uint64_t(1) << 46;                     // descriptor version (sm_100)
+  d |= uint64_t(2) << 61;                     // swizzle: 128 bytes
+  return d;
+}
+
+// kind::f16 instruction descriptor: D fp32, A and B fp16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int m, int n) {
+  return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// Eight Q4_0 weights of one qs word (element 2m = low nibble of byte m) as fp16 (q-8)*d,
+// returned as 4 half2 in element order (e0,e1) (e2,e3) (e4,e5) (e6,e7).
+__device__ __forceinline__ void q4_word_to_f16(uint32_t w, __half2 d2, uint32_t (&o)[4]) {
+  const __half2 bias = __half2half2(__ushort_as_half(0x6408));  // 1032
+  // 1024 + q as fp16: (e0,e4) (e1,e5) (e2,e6) (e3,e7)
+  uint32_t p04 = (w & 0x000F000Fu) | 0x64006400u;
+  uint32_t p15 = ((w >> 4) & 0x000F000Fu) | 0x64006400u;
+  uint32_t p26 = ((w >> 8) & 0x000F000Fu) | 0x64006400u;
+  uint32_t p37 = ((w >> 12) & 0x000F000Fu) | 0x64006400u;
+  // (1024 + q) - 1032 = q - 8 exactly; times d rounds once
+  p04 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p04), bias), d2));
+  p15 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p15), bias), d2));
+  p26 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p26), bias), d2));
+  p37 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p37), bias), d2));
+  o[0] = __byte_perm(p04, p15, 0x5410);  // (e0, e1)
+  o[1] = __byte_perm(p26, p37, 0x5410);  // (e2, e3)
+  o[2] = __byte_perm(p04, p15, 0x7632);  // (e4, e5)
+  o[3] = __byte_perm(p26, p37, 0x7632);  // (e6, e7)
+}
+
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// ---------------------------------------------------------------- the kernel
+__global__ void __launch_bounds__(kPfThreads, 1)
+    k_prefill_q4(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                 const __grid_constant__ PfParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled operand tiles
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_s & 1023)) & 1023);
+  uint8_t* a_ring = smem;                                        // kPfStages x 16 KB
+  uint8_t* b_ring = a_ring + size_t(kPfStages) * kPfABytes;     // kPfStages x 16 KB
+  uint8_t* w_ring = b_ring + size_t(kPfStages) * kPfBBytes;     // kPfRawStages x 18 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(w_ring + size_t(kPfRawStages) * kPfRawBytes);
+  uint64_t* a_full = bars;                        // [kPfStages] TMA bytes of X
+  uint64_t* b_full = a_full + kPfStages;          // [kPfStages] 128 dequant threads
+  uint64_t* st_empty = b_full + kPfStages;        // [kPfStages] MMA commit
+  uint64_t* w_full = st_empty + kPfStages;        // [kPfRawStages] TMA bytes of raw W
+  uint64_t* w_empty = w_full + kPfRawStages;      // [kPfRawStages] 128 dequant threads
+  uint64_t* done = w_empty + kPfRawStages;        // final MMA commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / prm.ksplit;
+  const int split = blockIdx.x - tile * prm.ksplit;
+  const int n0 = tile * kPfTileN;
+  const int c0 = split * prm.kchunks / prm.ksplit;
+  const int nraw = (split + 1) * prm.kchunks / prm.ksplit - c0;  // >= 1 (kchunks >= ksplit)
+  const int k_begin = c0 * kPfRawK;
+  const int nst = nraw * (kPfRawK / kPfStageK);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPfStages; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&b_full[i], 128);
+      mbar_init(&st_empty[i], 1);
+    }
+    for (int i = 0; i < kPfRawStages; ++i) {
+      mbar_init(&w_full[i], 1);
+      mbar_init(&w_empty[i], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    // 128 fp32 columns of tensor memory for the 128 x 128 accumulator
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kPfTileN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0, r = 0;
+      for (; r < nraw && !*abort_flag; ++r) {
+        const int rs = r % kPfRawStages;
+        if (r >= kPfRawStages && !mbar_wait(&w_empty[rs], uint32_t(r / kPfRawStages - 1) & 1u)) {
+          *abort_flag = 1;
+          break;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&w_full[rs], uint32_t(kPfRawBytes));
+        tma_load_2d(w_ring + size_t(rs) * kPfRawBytes, &tmap_w, (k_begin / kPfRawK + r) * kPfRawBytesRow, n0,
+                    &w_full[rs]);
+        for (int q = 0; q < kPfRawK / kPfStageK; ++q, ++s) {
+          const int st = s % kPfStages;
+          if (s >= kPfStages && !mbar_wait(&st_empty[st], uint32_t(s / kPfStages - 1) & 1u)) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&a_full[st], uint32_t(kPfABytes));
+          tma_load_2d(a_ring + size_t(st) * kPfABytes, &tmap_x, k_begin + s * kPfStageK, 0, &a_full[st]);
+        }
+      }
+      if (*abort_flag) {
+        // bounded wait for the copies already issued, so none lands after the CTA exits
+        for (int q = (s > kPfStages ? s - kPfStages : 0); q < s; ++q)
+          mbar_wait(&a_full[q % kPfStages], uint32_t(q / kPfStages) & 1u);
+        for (int q = (r > kPfRawStages ? r - kPfRawStages : 0); q < r; ++q)
+          mbar_wait(&w_full[q % kPfRawStages], uint32_t(q / kPfRawStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(kPfTileM, kPfTileN);
+      for (int s = 0; s < nst; ++s) {
+        const int st = s % kPfStages;
+        const uint32_t par = uint32_t(s / kPfStages) & 1u;
+        if (!mbar_wait(&a_full[st], par) || !mbar_wait(&b_full[st], par)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_s = smem_u32(a_ring + size_t(st) * kPfABytes);
+        const uint32_t b_s = smem_u32(b_ring + size_t(st) * kPfBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kPfStageK / 16; ++kk)  // 16 fp16 = 32 bytes per MMA along k
+          umma_f16(tmem, umma_desc_sw128(a_s + 32 * kk), umma_desc_sw128(b_s + 32 * kk), idesc,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&st_empty[st]);  // frees the stage once these MMAs have read it
+      }
+      umma_commit(done);  // all MMAs issued by this thread have completed
+    }
+  } else {
+    // ------------------------------------------------ dequantize W into the B stages
+    const int t = threadIdx.x - 64;  // 0..127: weight row n0 + t of the tile
+    const uint32_t b_row_base = uint32_t(t >> 3) * 1024 + uint32_t(t & 7) * 128;
+    const int sw = t & 7;            // swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+    int s = 0;
+    bool ok = true;
+    for (int r = 0; r < nraw && ok; ++r) {
+      const int rs = r % kPfRawStages;
+      if (!mbar_wait(&w_full[rs], uint32_t(r / kPfRawStages) & 1u)) {
+        ok = false;
+        break;
+      }
+      const uint32_t raw_row = smem_u32(w_ring + size_t(rs) * kPfRawBytes) + uint32_t(t) * kPfRawBytesRow;
+      for (int q = 0; q < kPfRawK / kPfStageK; ++q, ++s) {
+        const int st = s % kPfStages;
+        if (s >= kPfStages && !mbar_wait(&st_empty[st], uint32_t(s / kPfStages - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        // two Q4_0 blocks (36 bytes) of this row: block A at bytes 0..17, block B at 18..35
+        uint32_t v[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) v[i] = lds32(raw_row + 36 * q + 4 * i);
+        const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
+        const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[4] >> 16)));
+        const uint32_t b_s = smem_u32(b_ring + size_t(st) * kPfBBytes) + b_row_base;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {  // block A: k = 8m .. 8m+7
+          uint32_t o[4];
+          q4_word_to_f16(__funnelshift_r(v[m], v[m + 1], 16), dA, o);
+          sts128(b_s + uint32_t((m ^ sw) * 16), o[0], o[1], o[2], o[3]);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {  // block B: k = 32 + 8m .. 32 + 8m + 7
+          uint32_t o[4];
+          q4_word_to_f16(v[5 + m], dB, o);
+          sts128(b_s + uint32_t(((4 + m) ^ sw) * 16), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();  // make the fp16 tile visible to the tensor core
+        mbar_arrive(&b_full[st]);
+      }
+      mbar_arrive(&w_empty[rs]);
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  // ------------------------------------------------ epilogue: accumulator -> fp16 Y
+  // Warps 2-5 own the accumulator rows (tensor-memory lanes 32*(warp%4) .. +31 = tokens).  With a
+  // k-split cluster every CTA parks its partial tile in its (now idle) A ring and rank 0 sums the
+  // ranks in order through distributed shared memory; every thread of every CTA takes part in the
+  // two cluster barriers.
+  const bool epi_warp = warp >= 2;
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;  // token
+  bool have = false;
+  if (epi_warp) {
+    have = !*abort_flag && mbar_wait(done, 0);
+    tc_fence_after();
+  }
+  float* park = reinterpret_cast<float*>(a_ring);  // [kPfTileN][kPfTileM] fp32 = 64 KB
+  const uint32_t tm_row = tmem + (uint32_t(quarter * 32) << 16);
+  if (prm.ksplit > 1) {
+    if (epi_warp) {
+#pragma unroll 1
+      for (int c = 0; c < kPfTileN; c += 16) {
+        uint32_t r16[16];
+        if (have) tmem_ld16(tm_row + uint32_t(c), r16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) park[(c + i) * kPfTileM + row] = have ? __uint_as_float(r16[i]) : 0.f;
+      }
+    }
+    __syncwarp();
+    cluster_sync();
+    if (epi_warp && cluster_ctarank() == 0 && row < prm.tokens) {
+      __half* y = static_cast<__half*>(prm.Y) + size_t(row) * prm.n + n0;
+      const int ncols = min(kPfTileN, prm.n - n0);
+#pragma unroll 1
+      for (int c = 0; c < ncols; c += 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = park[(c + i) * kPfTileM + row];
+        for (int rk = 1; rk < prm.ksplit; ++rk)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] += ld_dsmem_f32(smem_u32(&park[(c + i) * kPfTileM + row]), uint32_t(rk));
+        uint4 pk;
+        pk.x = h2_bits(__floats2half2_rn(v[0], v[1]));
+        pk.y = h2_bits(__floats2half2_rn(v[2], v[3]));
+        pk.z = h2_bits(__floats2half2_rn(v[4], v[5]));
+        pk.w = h2_bits(__floats2half2_rn(v[6], v[7]));
+        *reinterpret_cast<uint4*>(y + c) = pk;
+      }
+    }
+    __syncwarp();
+    cluster_sync();  // peers keep their shared memory until rank 0 has read it
+  } else if (epi_warp && have) {
+    // tcgen05.ld is warp-collective: every lane loads, only rows < tokens store
+    __half* y = static_cast<__half*>(prm.Y) + size_t(row) * prm.n + n0;
+    const int ncols = row < prm.tokens ? min(kPfTileN, prm.n - n0) : 0;
+#pragma unroll 1
+    for (int c = 0; c < kPfTileN; c += 16) {
+      uint32_t r16[16];
+      tmem_ld16(tm_row + uint32_t(c), r16);
+      if (c < ncols) {
+        uint4 pk;
+        pk.x = h2_bits(__floats2half2_rn(__uint_as_float(r16[0]), __uint_as_float(r16[1])));
+        pk.y = h2_bits(__floats2half2_rn(__uint_as_float(r16[2]), __uint_as_float(r16[3])));
+        pk.z = h2_bits(__floats2half2_rn(__uint_as_float(r16[4]), __uint_as_float(r16[5])));
+        pk.w = h2_bits(__floats2half2_rn(__uint_as_float(r16[6]), __uint_as_float(r16[7])));
+        *reinterpret_cast<uint4*>(y + c) = pk;
+      }
+      if (c + 8 < ncols) {
+        uint4 pk;
+        pk.x = h2_bits(__floats2half2_rn(__uint_as_float(r16[8]), __uint_as_float(r16[9])));
+        pk.y = h2_bits(__floats2half2_rn(__uint_as_float(r16[10]), __uint_as_float(r16[11])));
+        pk.z = h2_bits(__floats2half2_rn(__uint_as_float(r16[12]), __uint_as_float(r16[13])));
+        pk.w = h2_bits(__floats2half2_rn(__uint_as_float(r16[14]), __uint_as_float(r16[15])));
+        *reinterpret_cast<uint4*>(y + c + 8) = pk;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPfTileN));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return nullptr;
+    f = reinterpret_cast<EncodeTiledFn>(p);
+    fn.store(f, std::memory_order_release);
+  }
+  return f;
+}
+
+inline SmemAttrOnce g_prefill_attr;
+
+}  // namespace bqg
+
+extern "C" int qgemm_prefill(int fmt, const void* W, const void* X, void* Y, int tokens, int n, int k, void* stream) {
+  using namespace bqg;
+  if (W == nullptr || X == nullptr || Y == nullptr || tokens < 1 || n < 1 || k < 1) return BQG_ERR_ARG;
+  if (fmt != BQG_Q4_0) return BQG_ERR_FMT;
+  if (tokens > kPfTileM || n % 16 != 0 || k % kPfRawK != 0 || k > BQG_MAX_COLS) return BQG_ERR_SHAPE;
+  if (!aligned(W, 16) || !aligned(X, 16) || !aligned(Y, 16)) return BQG_ERR_ALIGN;
+  int dev;
+  DeviceInfo* info;
+  int st = current_device(&dev, &info);
+  if (st != BQG_OK) return st;
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (encode == nullptr) return BQG_ERR_CUDA;
+  st = g_prefill_attr.ensure(dev, k_prefill_q4, kPfSmemBytes);
+  if (st != BQG_OK) return st;
+
+  // X: fp16 [tokens x k], tiles of 64 k x 128 rows, 128-byte swizzle; rows >= tokens read as 0
+  CUtensorMap tx, tw;
+  {
+    const cuuint64_t dims[2] = {cuuint64_t(k), cuuint64_t(tokens)};
+    const cuuint64_t strides[1] = {cuuint64_t(k) * 2};
+    const cuuint32_t box[2] = {cuuint32_t(kPfStageK), cuuint32_t(kPfTileM)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return BQG_ERR_CUDA;
+  }
+  // W: the Q4_0 bytes as a [n x row_bytes] byte matrix, tiles of 144 bytes (256 k) x 128 rows;
+  // rows >= n read as 0 (scale 0: weights 0)
+  {
+    const cuuint64_t rb = cuuint64_t(k / 32) * 18;
+    const cuuint64_t dims[2] = {rb, cuuint64_t(n)};
+    const cuuint64_t strides[1] = {rb};
+    const cuuint32_t box[2] = {cuuint32_t(kPfRawBytesRow), cuuint32_t(kPfTileN)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(W), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return BQG_ERR_CUDA;
+  }
+
+  // Split k across a cluster of CTAs when the output tiles alone would leave SMs idle.
+  const int ntiles = (n + kPfTileN - 1) / kPfTileN;
+  const int kchunks = k / kPfRawK;
+  int ksplit = 1;
+  while (ksplit * 2 <= kPfMaxSplit && ntiles * ksplit * 2 <= info->sm_count && kchunks >= ksplit * 2) ksplit *= 2;
+  PfParams prm{};
+  prm.Y = Y;
+  prm.tokens = tokens;
+  prm.n = n;
+  prm.k = k;
+  prm.ksplit = ksplit;
+  prm.kchunks = kchunks;
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(ntiles * ksplit), 1, 1);
+  cfg.blockDim = dim3(kPfThreads, 1, 1);
+  cfg.dynamicSmemBytes = kPfSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(ksplit);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_prefill_q4, tx, tw, prm) != cudaSuccess) return BQG_ERR_CUDA;
+  return launch_status();
+}

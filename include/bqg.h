@@ -122,6 +122,21 @@ typedef struct {
 
 BQG_API int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream);
 
+/* ---------------------------------------------------------------- a11: prefill-chunk GEMM
+ * qgemm_prefill: Y = X W^T with fp16 activations and Q4_0 weights on the tcgen05 tensor
+ * cores (fp16 operands, fp32 accumulation in tensor memory, fp16 output, round to nearest).
+ *   Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (prefill in chunks of at most 128
+ *   tokens, each weight read reused by every prompt row of the chunk).
+ *   fmt     BQG_Q4_0.
+ *   W       device, bqg_weight_bytes(BQG_Q4_0, n, k) bytes, 16-byte aligned.
+ *   X       device fp16 [tokens x k] row-major, 16-byte aligned.
+ *   Y       device fp16 [tokens x n] row-major, 16-byte aligned.
+ *   tokens  1..128.   n  >= 16, multiple of 16.   k  multiple of 256, 256 <= k <= BQG_MAX_COLS.
+ *   Small n is split along k over a thread-block cluster (up to 8 CTAs) whose partial tiles are
+ *   summed in a fixed order, so results are deterministic. */
+BQG_API int qgemm_prefill(int fmt, const void* W, const void* X, void* Y, int tokens, int n, int k,
+                  void* stream);
+
 /* ---------------------------------------------------------------- a5: router logits
  * moe_router_logits: logits[t, e] = sum_h R[e, h] x[t, h] in fp32.
  *   Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (router choosing experts per token).

@@ -30,7 +30,8 @@ def declared_functions():
 
 def test_header_declares_the_api():
     names = declared_functions()
-    for want in ["qgemv", "qgemv_batched", "moe_router_logits", "moe_router_topk", "bqg_status_string", "bqg_weight_bytes",
+    for want in ["qgemv", "qgemv_batched", "qgemm_prefill", "moe_router_logits", "moe_router_topk",
+                 "moe_workspace_size", "moe_forward", "moe_forward_noalloc", "bqg_status_string", "bqg_weight_bytes",
                  "bqg_device_errors", "bqg_version"]:
         assert want in names
 
@@ -115,3 +116,34 @@ def test_only_the_c_abi_is_exported(L):
     out = subprocess.run(["nm", "-D", "--defined-only", L.library_path()], capture_output=True, text=True).stdout
     exported = set(line.split()[-1] for line in out.splitlines() if line.split()[1:2] and line.split()[1] in "TBDVWu")
     assert exported <= set(declared_functions()) | {"_init", "_fini"}, exported - set(declared_functions())
+
+
+def test_prefill_argument_errors(L):
+    f = L.lib().qgemm_prefill
+    A = 0x10000
+    assert f(1, A, A, A, 128, 1024, 4096, None) == -2        # only Q4_0
+    assert f(2, A, A, A, 129, 1024, 4096, None) == -3        # more than 128 tokens
+    assert f(2, A, A, A, 128, 1000, 4096, None) == -3        # n % 16
+    assert f(2, A, A, A, 128, 1024, 4000, None) == -3        # k % 256
+    assert f(2, A + 8, A, A, 128, 1024, 4096, None) == -4
+    assert f(2, None, A, A, 128, 1024, 4096, None) == -1
+
+
+def test_moe_argument_errors(L):
+    import block_quant_gemv_b200 as bqg
+    c = bqg.MoELayerC()
+    c.n_experts, c.top_k, c.hidden, c.inter, c.expert_fmt, c.act = 128, 8, 2816, 704, 2, 1
+    c.gate = c.up = c.down = 0x10000
+    c.gate_stride = c.up_stride = c.down_stride = synth.weight_bytes(2, 704, 2816) + 16 - synth.weight_bytes(2, 704, 2816) % 16
+    size = L.lib().moe_workspace_size(ctypes.byref(c), 16)
+    assert size > 0
+    A = 0x10000
+    fwd = L.lib().moe_forward
+    assert fwd(ctypes.byref(c), A, A, A, A, 16, A, size - 1, None) == -5   # workspace too small
+    assert fwd(ctypes.byref(c), A, A, A, A, 16, A + 16, size, None) == -4  # workspace alignment
+    c.top_k = 9
+    assert fwd(ctypes.byref(c), A, A, A, A, 16, A, size, None) == -8
+    c.top_k, c.act = 8, 7
+    assert fwd(ctypes.byref(c), A, A, A, A, 16, A, size, None) == -1
+    c.act, c.hidden = 1, 2820
+    assert L.lib().moe_workspace_size(ctypes.byref(c), 16) == 0
