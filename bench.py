@@ -31,6 +31,7 @@ if ROOT not in sys.path:
 METRIC = "quantized GEMV/MoE weight-stream GB/s (% of HBM peak); us per MoE layer"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["common.cuh", "qgemv.cuh"]
 
 
@@ -43,6 +44,7 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-glm", action="store_true", help="skip the 39 GB GLM-like MoE stack")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     return ap.parse_args()
 
@@ -55,6 +57,18 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense fp16 tensor peak in TFLOP/s: the measured bf16 burst figure (fp16 and bf16 run at the
+    same nominal rate on the tensor cores), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"])
+    return FALLBACK_BF16_TFLOPS
 
 
 def kernel_source_hash() -> str:
@@ -276,12 +290,14 @@ def time_decode_step(args, world, dev):
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.2)
+    torch.cuda.nvtx.range_push("timed")  # lets a profiler select exactly the timed launches
     t_begin.record(stream)
     for i in range(args.steps):
         starts[i].record(stream)
         batch.run()
         ends[i].record(stream)
     t_end.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier(world)
@@ -351,6 +367,143 @@ def time_single_q8_0(dev, seed):
             "us_per_call": us, "GB/s": nbytes / us / 1e3, "bytes_per_call": nbytes}
 
 
+def graph_us(fn, reps: int = 20) -> float:
+    """Device time of fn (a sequence of library calls) captured once in a CUDA graph: warm-up
+    replays, then CUDA events around `reps` replays on the capture stream."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    # replay() launches on the current stream: the events go there too
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def time_prefill(dev, seed, tensor_peak):
+    """Q4_0 prefill-chunk GEMM, 128 tokens x K=4096, N in (14336, 4096, 1024): enough distinct
+    weight copies rotated in one graph that a rotation touches >= 256 MB (2x L2)."""
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    import synth
+    out = {}
+    t, k = 128, 4096
+    X = synth.normal_f16(seed, synth.stream_id("prefill/X"), t * k).view(t, k).to(dev)
+    for n in (14336, 4096, 1024):
+        wb = synth.weight_bytes(bqg.Q4_0, n, k)
+        copies = max(1, -(-(256 << 20) // wb))
+        Ws = [synth.q4_0_matrix(n, k, seed, f"prefill/N{n}/copy{c}", device=dev) for c in range(copies)]
+        Y = torch.empty(t, n, dtype=torch.float16, device=dev)
+
+        def fn():
+            for W in Ws:
+                bqg.qgemm_prefill(bqg.Q4_0, W, X, n, k, Y)
+        us = graph_us(fn, reps=10) / copies
+        flops = 2.0 * t * n * k
+        nbytes = wb + 2 * t * k + 2 * t * n
+        out[f"N{n}"] = {"us_per_call": us, "TFLOP/s": flops / us / 1e6, "tensor_frac": flops / us / 1e6 / tensor_peak,
+                        "GB/s": nbytes / us / 1e3, "rotating_copies": copies}
+        del Ws
+    out["workload"] = "prefill chunk 128 tokens x K=4096 fp16, Q4_0 W N x 4096, fp16 out"
+    out["tensor_peak_TFLOP/s"] = tensor_peak
+    return out
+
+
+def moe_device_layer(T):
+    import block_quant_gemv_b200 as bqg
+    s = T.spec
+    shared = None if T.shared is None else (s.shared_fmt, s.shared_inter) + tuple(T.shared)
+    return bqg.MoELayer(s.n_experts, s.top_k, s.hidden, s.inter, s.expert_fmt, s.act, T.gate, T.up, T.down,
+                        T.gate_stride, T.up_stride, T.down_stride, shared)
+
+
+def time_moe_gemma(dev, seed, peak, copies=8):
+    """Gemma-like MoE layer (router, top-8 of 128, grouped GeGLU experts, shared expert) at
+    T = 1, 16, 128: `copies` independent layers rotated in one graph (>= 2x L2 of touched bytes
+    at T = 1); us per layer includes the router."""
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    spec = wl.GEMMA_MOE
+    Ts = [wl.build_moe_layer(spec, seed, layer=l, device=dev) for l in range(copies)]
+    Ls = [moe_device_layer(T) for T in Ts]
+    shared_bytes = sum(spec.shared_bytes(w) for w in ("gate", "up", "down"))
+    expert_bytes = sum(spec.mat_bytes(w) for w in ("gate", "up", "down"))
+    router_bytes = 4 * spec.n_experts * spec.hidden
+    out = {"workload": "gemma_moe: hidden 2816, 128 experts Q4_0 GeGLU 704, top-8, shared Q8_0 GeGLU 2112, "
+                       f"fp32 router; {copies} layers rotated"}
+    for T in (1, 16, 128):
+        x = wl.moe_tokens(spec, seed, T).to(dev)
+        logits = [torch.empty(T, spec.n_experts, device=dev) for _ in Ls]
+        idx = [torch.empty(T, spec.top_k, dtype=torch.int32, device=dev) for _ in Ls]
+        w = [torch.empty(T, spec.top_k, device=dev) for _ in Ls]
+        y = torch.empty(T, spec.hidden, device=dev)
+        ws = torch.empty(bqg.moe_workspace_size(Ls[0], T), dtype=torch.uint8, device=dev)
+
+        def fn():
+            for l in range(copies):
+                bqg.moe_router_logits(Ts[l].R, x, logits[l])
+                bqg.moe_router_topk(logits[l], spec.top_k, idx[l], w[l])
+                bqg.moe_forward(Ls[l], x, idx[l], w[l], y, ws)
+        us = graph_us(fn) / copies
+        distinct = sum(int(torch.unique(i).numel()) for i in idx) / copies
+        nbytes = router_bytes + shared_bytes + distinct * expert_bytes + 8 * T * spec.hidden
+        out[f"T{T}"] = {"us_per_layer": us, "distinct_experts": distinct, "bytes_per_layer": nbytes,
+                        "GB/s": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak}
+    del Ts, Ls
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_moe_glm(dev, seed, peak):
+    """GLM-like stack: 8 resident layers of 256 int4-row SwiGLU experts (38.7 GB), given N(0,1)
+    logits, top-8, layers chained (x of layer l+1 = y of layer l); T = 1, 8, 64."""
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    spec = wl.GLM_MOE
+    Ts = [wl.build_moe_layer(spec, seed, layer=l, device=dev) for l in range(wl.GLM_LAYERS)]
+    Ls = [moe_device_layer(T) for T in Ts]
+    expert_bytes = sum(spec.mat_bytes(w) for w in ("gate", "up", "down"))
+    resident = sum(T.gate.numel() + T.up.numel() + T.down.numel() for T in Ts)
+    out = {"workload": f"glm_moe: {wl.GLM_LAYERS} layers x 256 int4-row experts (hidden 6144, SwiGLU 2048), "
+                       f"top-8 of given N(0,1) logits, chained; {resident / 1e9:.1f} GB resident"}
+    for T in (1, 8, 64):
+        logits = [wl.moe_logits(spec, seed, l, T).to(dev) for l in range(len(Ls))]
+        idx = [torch.empty(T, spec.top_k, dtype=torch.int32, device=dev) for _ in Ls]
+        w = [torch.empty(T, spec.top_k, device=dev) for _ in Ls]
+        xs = [wl.moe_tokens(spec, seed, T).to(dev)] + [torch.empty(T, spec.hidden, device=dev) for _ in Ls]
+        ws = torch.empty(bqg.moe_workspace_size(Ls[0], T), dtype=torch.uint8, device=dev)
+
+        def fn():
+            for l in range(len(Ls)):
+                bqg.moe_router_topk(logits[l], spec.top_k, idx[l], w[l])
+                bqg.moe_forward(Ls[l], xs[l], idx[l], w[l], xs[l + 1], ws)
+        us = graph_us(fn, reps=5) / len(Ls)
+        distinct = sum(int(torch.unique(i).numel()) for i in idx) / len(Ls)
+        nbytes = distinct * expert_bytes + 8 * T * spec.hidden + 4 * T * spec.n_experts
+        out[f"T{T}"] = {"us_per_layer": us, "distinct_experts": distinct, "bytes_per_layer": nbytes,
+                        "GB/s": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak}
+    del Ts, Ls
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
     assert torch.cuda.is_available(), "bench.py --impl ours needs a CUDA device"
@@ -370,6 +523,10 @@ def run_ours(args, world, rank, local):
     extras = {}
     if not args.no_extras:
         extras["q8_0_2048"] = time_single_q8_0(dev, args.seed)
+        extras["prefill"] = time_prefill(dev, args.seed, tensor_peak())
+        extras["moe_gemma"] = time_moe_gemma(dev, args.seed, peak)
+        if not args.no_glm:
+            extras["moe_glm"] = time_moe_glm(dev, args.seed, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -126,3 +126,33 @@ def test_tinyllama_decode_step_full_size_sampled():
         assert_close(y, ref, what=s.name)
         assert_close(y, ref, tol=1e-4, what=s.name + " (fp32 accuracy)")
     assert W.weight_bytes == 614_629_376
+
+
+def test_repeated_launches_and_graph_replays():
+    """Thousands of back-to-back launches, and replays of a captured graph of launches, all
+    give the same rows (no state is carried from one launch to the next)."""
+    need_gpu()
+    rows, cols = 3000, 2048
+    W = synth.q4_0_matrix(rows, cols, 0, "sched/W").cuda()
+    x = synth.normal_f32(0, 11, cols).cuda()
+    ref = bqg.qgemv(bqg.Q4_0, W, x, rows, cols).clone()
+    ys = [torch.empty(rows, device="cuda") for _ in range(4)]
+    for i in range(4200):
+        bqg.qgemv(bqg.Q4_0, W, x, rows, cols, ys[i % 4])
+        if i % 700 == 0 or i >= 4196:
+            torch.cuda.synchronize()
+            assert torch.equal(ys[i % 4], ref), f"launch {i}"
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for y in ys:
+            bqg.qgemv(bqg.Q4_0, W, x, rows, cols, y)
+    for rep in range(5):
+        for y in ys:
+            y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for y in ys:
+            assert torch.equal(y, ref), f"replay {rep}"
+    assert bqg.bqg_device_errors() == 0
