@@ -13,14 +13,15 @@
 //    layout (18/34-byte blocks); an unaligned start is copied from the 16-byte boundary below.
 //  * 15 consumer warps.  A row is split into "units" (a pair of blocks, one block, or 32/64
 //    int4 weights); a row group of W = ceil(units/32) warps owns whole rows, lane l of its
-//    warp j handling unit 32j+l.  Each thread keeps its unit's 64 x values (fp32) in registers
-//    for the whole matrix: each weight byte is read once from shared memory and x costs no
-//    shared-memory traffic in the loop.  x itself is bulk-copied into shared memory by the
-//    producer one matrix ahead.  Two rows are processed together for more independent FMAs.
-//  * Dequantization uses byte permutes into the fp32 mantissa: a nibble q becomes the float
-//    128+q exactly (bits 0x43qq0000), an int8 becomes 2^23+128+q (then minus 2^23+128); sums
-//    are fp32 FMAs and the constant offset of the nibble formats is removed with a per-block
-//    sum of x.  All products are exact; only the fp32 sums round.
+//    warp j handling unit 32j+l.  Each thread keeps its unit's x (in the integer form below) in
+//    registers for the whole matrix: each weight byte is read once from shared memory and x
+//    costs no shared-memory traffic in the loop.  x itself is bulk-copied into shared memory by the
+//    producer one matrix ahead.  Two rows are processed together for more independent chains.
+//  * Integer dot products: each thread converts its unit of x once per matrix to 16-bit fixed
+//    point (per-unit scale), split into high and low bytes; a 4-byte weight word then costs two
+//    dp4a (Q8_0), or two masks and four dp4a (nibble formats), with exact int32 sums per block.  The block
+//    scale and the sum over blocks are fp32.  (dp4a has about 2.4x the throughput per weight of
+//    an fp32 decode by byte permutes plus FMAs on B200, which keeps the kernel memory-bound.)
 //  * Each row is reduced with a warp butterfly (plus a fixed-order sum over the W warps of a
 //    group through shared memory), so results are deterministic.
 #pragma once
@@ -109,93 +110,137 @@ __host__ __device__ constexpr int gemv_stage_rows(int units, int row_bytes) {
 static_assert(kGemvStageBytes >= kGemvCompute * 68, "a stage must hold one row per row group");
 
 // ---------------------------------------------------------------- dequant + dot helpers
-// Nibbles: bytes of `lo` hold elements 0,2,4,6 and bytes of `hi` elements 1,3,5,7 (each 0..15).
-// __byte_perm(v, 0x43, 0x4k55) = 0x43 << 24 | byte_k(v) << 16, the float 128 + byte_k(v).
-__device__ __forceinline__ void dot8_nib(uint32_t lo, uint32_t hi, const float* x, float& a0, float& a1, float& a2,
-                                         float& a3) {
-  a0 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4055u)), x[0], a0);
-  a1 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4055u)), x[1], a1);
-  a2 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4155u)), x[2], a2);
-  a3 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4155u)), x[3], a3);
-  a0 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4255u)), x[4], a0);
-  a1 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4255u)), x[5], a1);
-  a2 = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4355u)), x[6], a2);
-  a3 = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4355u)), x[7], a3);
+// x of one unit (32 or 64 values) in 16-bit fixed point: x_i ~= s * X_i with X_i =
+// round(x_i * 32767 / max|x|) (per unit, so |X_i| <= 32767), split into a signed high byte and
+// an unsigned low byte, X_i = 256 * H_i + L_i, packed four per word in the order in which the
+// weight bytes hold their elements.  The integer dot products sum_i q_i X_i are then exact
+// (dp4a, int32) for every block, and only the per-block scaling and the sum over blocks use
+// fp32.  The quantization of x is the only approximation: |x_i - s X_i| <= max|x| / 65534,
+// about 3e-5 of a typical |y| for Gaussian x.
+//   nibble formats: word 2m holds elements 8m, 8m+2, 8m+4, 8m+6 (low nibbles of bytes 4m..4m+3),
+//                   word 2m+1 holds 8m+1, 8m+3, 8m+5, 8m+7 (high nibbles);
+//   Q8_0:           word m holds elements 4m..4m+3.
+struct XUnit {
+  uint32_t h[16];  // high bytes (signed)
+  uint32_t l[16];  // low bytes (unsigned)
+  int c0, c1;      // nibble formats: -8 * sum of X over block 0 / block 1 (the q - 8 offset)
+  float s;         // x_i ~= s * X_i
+};
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {  // a unsigned bytes, b signed
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {  // a signed bytes, b unsigned
+  int d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-// Q4_0 word (8 unsigned nibbles, element 2m low / 2m+1 high nibble of byte m): adds (128+q)*x.
-__device__ __forceinline__ void dot8_q4(uint32_t w, const float* x, float& a0, float& a1, float& a2, float& a3) {
-  dot8_nib(w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu, x, a0, a1, a2, a3);
+// Bytes k of four integers as one word (k = 0: low bytes, k = 1: second bytes).
+__device__ __forceinline__ uint32_t pack_byte(int a, int b, int c, int d, int k) {
+  const uint32_t sel = k == 0 ? 0x0040u : 0x0051u;
+  return __byte_perm(__byte_perm(uint32_t(a), uint32_t(b), sel), __byte_perm(uint32_t(c), uint32_t(d), sel), 0x5410u);
 }
 
-// int4 word (two's-complement nibbles): xor 8 maps q to q+8 in 0..15; adds (136+q)*x.
-__device__ __forceinline__ void dot8_i4(uint32_t w, const float* x, float& a0, float& a1, float& a2, float& a3) {
-  dot8_nib((w ^ 0x08080808u) & 0x0F0F0F0Fu, ((w >> 4) ^ 0x08080808u) & 0x0F0F0F0Fu, x, a0, a1, a2, a3);
-}
-
-// Q8_0 word (4 int8): xor 0x80 gives q+128 in 0..255; __byte_perm(u, 0x4B, 0x455k) is the
-// float 2^23 + q + 128, so subtracting 2^23 + 128 recovers q exactly.
-__device__ __forceinline__ void dot4_q8(uint32_t w, const float* x, float& a0, float& a1) {
-  const uint32_t u = w ^ 0x80808080u;
-  const float off = 8388736.0f;  // 2^23 + 128
-  a0 = fmaf(__uint_as_float(__byte_perm(u, 0x4Bu, 0x4550u)) - off, x[0], a0);
-  a1 = fmaf(__uint_as_float(__byte_perm(u, 0x4Bu, 0x4551u)) - off, x[1], a1);
-  a0 = fmaf(__uint_as_float(__byte_perm(u, 0x4Bu, 0x4552u)) - off, x[2], a0);
-  a1 = fmaf(__uint_as_float(__byte_perm(u, 0x4Bu, 0x4553u)) - off, x[3], a1);
-}
-
-// Loads one unit's x values from xs into registers and the per-block offset constants of the
-// nibble formats: c[b] = 136 * sum of x over block b (sum_i (128+u_i) x_i - c = sum (u_i-8) x_i).
-__device__ __forceinline__ void build_x(int kind, const float* xs, float (&x)[64], float& c0, float& c1) {
-  const int uw = unit_weights(kind);
+// Loads one unit's x from xs and converts it (see XUnit).
+template <int KIND>
+__device__ __forceinline__ void build_x(const float* xs, XUnit& X) {
+  constexpr int UW = unit_weights(KIND);
+  float xv[UW];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < uw / 4) v = reinterpret_cast<const float4*>(xs)[i];
-    x[4 * i] = v.x;
-    x[4 * i + 1] = v.y;
-    x[4 * i + 2] = v.z;
-    x[4 * i + 3] = v.w;
+  for (int i = 0; i < UW / 4; ++i) {
+    const float4 v = reinterpret_cast<const float4*>(xs)[i];
+    xv[4 * i] = v.x;
+    xv[4 * i + 1] = v.y;
+    xv[4 * i + 2] = v.z;
+    xv[4 * i + 3] = v.w;
   }
-  c0 = c1 = 0.f;
-  if (!is_q8(kind)) {
-    float s0 = 0.f, s1 = 0.f;
+  float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) s0 += x[i];
+  for (int i = 0; i < UW; ++i) amax = fmaxf(amax, fabsf(xv[i]));
+  const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+  X.s = amax * (1.f / 32767.f);
+  int xi[UW];
 #pragma unroll
-    for (int i = 32; i < 64; ++i) s1 += x[i];
-    c0 = 136.f * s0;
-    c1 = 136.f * s1;
+  for (int i = 0; i < UW; ++i) xi[i] = __float2int_rn(xv[i] * inv);
+  if constexpr (is_q8(KIND)) {
+#pragma unroll
+    for (int m = 0; m < UW / 4; ++m) {
+      X.h[m] = pack_byte(xi[4 * m], xi[4 * m + 1], xi[4 * m + 2], xi[4 * m + 3], 1);
+      X.l[m] = pack_byte(xi[4 * m], xi[4 * m + 1], xi[4 * m + 2], xi[4 * m + 3], 0);
+    }
+    X.c0 = X.c1 = 0;
+  } else {
+#pragma unroll
+    for (int m = 0; m < UW / 8; ++m) {
+      X.h[2 * m] = pack_byte(xi[8 * m], xi[8 * m + 2], xi[8 * m + 4], xi[8 * m + 6], 1);
+      X.l[2 * m] = pack_byte(xi[8 * m], xi[8 * m + 2], xi[8 * m + 4], xi[8 * m + 6], 0);
+      X.h[2 * m + 1] = pack_byte(xi[8 * m + 1], xi[8 * m + 3], xi[8 * m + 5], xi[8 * m + 7], 1);
+      X.l[2 * m + 1] = pack_byte(xi[8 * m + 1], xi[8 * m + 3], xi[8 * m + 5], xi[8 * m + 7], 0);
+    }
+    int s0 = 0, s1 = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s0 += xi[i];
+#pragma unroll
+    for (int i = 32; i < UW; ++i) s1 += xi[i];
+    X.c0 = -8 * s0;
+    X.c1 = -8 * s1;
   }
+}
+
+// sum over the 8 elements of one nibble word of u * X (u the unsigned nibble), into (h, l).
+__device__ __forceinline__ void dot8_nib(uint32_t lo, uint32_t hi, uint32_t xh0, uint32_t xh1, uint32_t xl0,
+                                         uint32_t xl1, int& h, int& l) {
+  h = dp4a_us(lo, xh0, h);
+  h = dp4a_us(hi, xh1, h);
+  l = dp4a_uu(lo, xl0, l);
+  l = dp4a_uu(hi, xl1, l);
 }
 
 // Partial dot products of the same unit of NR rows (shared-memory byte addresses u[n]) with
-// the thread's x registers.  Two rows at once give twice the independent FMA chains per thread.
+// the thread's x.  Two rows at once give twice the independent chains per thread.
 template <int KIND, int NR>
-__device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const float (&x)[64], float c0, float c1,
-                                          float (&out)[NR]) {
+__device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const XUnit& X, float (&out)[NR]) {
   if constexpr (KIND == kQ4Pair) {
     uint32_t v[NR][9];
 #pragma unroll
     for (int n = 0; n < NR; ++n)
 #pragma unroll
       for (int i = 0; i < 9; ++i) v[n][i] = lds32(u[n] + 4 * i);  // 4-byte aligned
-    float a[NR][4], b[NR][4];
+    int ha[NR], la[NR], hb[NR], lb[NR];
 #pragma unroll
-    for (int n = 0; n < NR; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[n][i] = b[n][i] = 0.f;
+    for (int n = 0; n < NR; ++n) {
+      ha[n] = hb[n] = 0;
+      la[n] = X.c0;
+      lb[n] = X.c1;
+    }
 #pragma unroll
     for (int m = 0; m < 4; ++m)
 #pragma unroll
       for (int n = 0; n < NR; ++n) {
-        dot8_q4(__funnelshift_r(v[n][m], v[n][m + 1], 16), &x[8 * m], a[n][0], a[n][1], a[n][2], a[n][3]);  // block A
-        dot8_q4(v[n][5 + m], &x[32 + 8 * m], b[n][0], b[n][1], b[n][2], b[n][3]);                          // block B
+        const uint32_t wa = __funnelshift_r(v[n][m], v[n][m + 1], 16);  // block A: qs bytes 2..17
+        dot8_nib(wa & 0x0F0F0F0Fu, (wa >> 4) & 0x0F0F0F0Fu, X.h[2 * m], X.h[2 * m + 1], X.l[2 * m], X.l[2 * m + 1],
+                 ha[n], la[n]);
+        const uint32_t wb = v[n][5 + m];  // block B: qs bytes 20..35
+        dot8_nib(wb & 0x0F0F0F0Fu, (wb >> 4) & 0x0F0F0F0Fu, X.h[8 + 2 * m], X.h[9 + 2 * m], X.l[8 + 2 * m],
+                 X.l[9 + 2 * m], hb[n], lb[n]);
       }
 #pragma unroll
     for (int n = 0; n < NR; ++n)
-      out[n] = half_bits_to_float(v[n][0]) * (((a[n][0] + a[n][1]) + (a[n][2] + a[n][3])) - c0) +
-               half_bits_to_float(v[n][4] >> 16) * (((b[n][0] + b[n][1]) + (b[n][2] + b[n][3])) - c1);
+      out[n] = X.s * fmaf(half_bits_to_float(v[n][0]), float(ha[n] * 256 + la[n]),
+                          half_bits_to_float(v[n][4] >> 16) * float(hb[n] * 256 + lb[n]));
   } else if constexpr (KIND == kQ4One) {
     uint32_t v[NR][5], sh[NR];
 #pragma unroll
@@ -205,39 +250,47 @@ __device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const float (
 #pragma unroll
       for (int i = 0; i < 5; ++i) v[n][i] = lds32(w + 4 * i);
     }
-    float a[NR][4];
+    int h[NR], l[NR];
 #pragma unroll
-    for (int n = 0; n < NR; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[n][i] = 0.f;
+    for (int n = 0; n < NR; ++n) {
+      h[n] = 0;
+      l[n] = X.c0;
+    }
 #pragma unroll
     for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int n = 0; n < NR; ++n)
-        dot8_q4(__funnelshift_rc(v[n][m], v[n][m + 1], 16 + sh[n]), &x[8 * m], a[n][0], a[n][1], a[n][2], a[n][3]);
+      for (int n = 0; n < NR; ++n) {
+        const uint32_t w = __funnelshift_rc(v[n][m], v[n][m + 1], 16 + sh[n]);
+        dot8_nib(w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu, X.h[2 * m], X.h[2 * m + 1], X.l[2 * m], X.l[2 * m + 1], h[n],
+                 l[n]);
+      }
 #pragma unroll
     for (int n = 0; n < NR; ++n)
-      out[n] = half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) *
-               (((a[n][0] + a[n][1]) + (a[n][2] + a[n][3])) - c0);
+      out[n] = X.s * half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) * float(h[n] * 256 + l[n]);
   } else if constexpr (KIND == kQ8Pair) {
     uint32_t v[NR][17];
 #pragma unroll
     for (int n = 0; n < NR; ++n)
 #pragma unroll
       for (int i = 0; i < 17; ++i) v[n][i] = lds32(u[n] + 4 * i);
-    float a[NR][2], b[NR][2];
+    int ha[NR], la[NR], hb[NR], lb[NR];
 #pragma unroll
-    for (int n = 0; n < NR; ++n) a[n][0] = a[n][1] = b[n][0] = b[n][1] = 0.f;
+    for (int n = 0; n < NR; ++n) ha[n] = la[n] = hb[n] = lb[n] = 0;
 #pragma unroll
     for (int m = 0; m < 8; ++m)
 #pragma unroll
       for (int n = 0; n < NR; ++n) {
-        dot4_q8(__funnelshift_r(v[n][m], v[n][m + 1], 16), &x[4 * m], a[n][0], a[n][1]);  // block A: bytes 2..33
-        dot4_q8(v[n][9 + m], &x[32 + 4 * m], b[n][0], b[n][1]);                          // block B: bytes 36..67
+        const uint32_t wa = __funnelshift_r(v[n][m], v[n][m + 1], 16);  // block A: q bytes 2..33
+        ha[n] = dp4a_ss(wa, X.h[m], ha[n]);
+        la[n] = dp4a_su(wa, X.l[m], la[n]);
+        const uint32_t wb = v[n][9 + m];  // block B: q bytes 36..67
+        hb[n] = dp4a_ss(wb, X.h[8 + m], hb[n]);
+        lb[n] = dp4a_su(wb, X.l[8 + m], lb[n]);
       }
 #pragma unroll
     for (int n = 0; n < NR; ++n)
-      out[n] = half_bits_to_float(v[n][0]) * (a[n][0] + a[n][1]) + half_bits_to_float(v[n][8] >> 16) * (b[n][0] + b[n][1]);
+      out[n] = X.s * fmaf(half_bits_to_float(v[n][0]), float(ha[n] * 256 + la[n]),
+                          half_bits_to_float(v[n][8] >> 16) * float(hb[n] * 256 + lb[n]));
   } else if constexpr (KIND == kQ8One) {
     uint32_t v[NR][9], sh[NR];
 #pragma unroll
@@ -247,15 +300,20 @@ __device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const float (
 #pragma unroll
       for (int i = 0; i < 9; ++i) v[n][i] = lds32(w + 4 * i);
     }
-    float a[NR][2];
+    int h[NR], l[NR];
 #pragma unroll
-    for (int n = 0; n < NR; ++n) a[n][0] = a[n][1] = 0.f;
+    for (int n = 0; n < NR; ++n) h[n] = l[n] = 0;
 #pragma unroll
     for (int m = 0; m < 8; ++m)
 #pragma unroll
-      for (int n = 0; n < NR; ++n) dot4_q8(__funnelshift_rc(v[n][m], v[n][m + 1], 16 + sh[n]), &x[4 * m], a[n][0], a[n][1]);
+      for (int n = 0; n < NR; ++n) {
+        const uint32_t w = __funnelshift_rc(v[n][m], v[n][m + 1], 16 + sh[n]);
+        h[n] = dp4a_ss(w, X.h[m], h[n]);
+        l[n] = dp4a_su(w, X.l[m], l[n]);
+      }
 #pragma unroll
-    for (int n = 0; n < NR; ++n) out[n] = half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) * (a[n][0] + a[n][1]);
+    for (int n = 0; n < NR; ++n)
+      out[n] = X.s * half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) * float(h[n] * 256 + l[n]);
   } else {  // int4 with per-row scale (applied by the caller): kI4x64 (8 words) or kI4x32 (4 words)
     constexpr int NW = (KIND == kI4x64) ? 8 : 4;
     uint32_t q[NR][8];
@@ -268,21 +326,21 @@ __device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const float (
         q[n][4] = p1.x; q[n][5] = p1.y; q[n][6] = p1.z; q[n][7] = p1.w;
       }
     }
-    float a[NR][4], b[NR][4];
+    int h[NR], l[NR];
 #pragma unroll
-    for (int n = 0; n < NR; ++n)
+    for (int n = 0; n < NR; ++n) {
+      h[n] = 0;
+      l[n] = X.c0 + X.c1;
+    }
+    // two's-complement nibble t: t ^ 8 = t + 8 in 0..15, so the q - 8 offset applies as for Q4_0
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[n][i] = b[n][i] = 0.f;
+    for (int k = 0; k < NW; ++k)
 #pragma unroll
-    for (int k = 0; k < NW; k += 2)
+      for (int n = 0; n < NR; ++n)
+        dot8_nib((q[n][k] ^ 0x08080808u) & 0x0F0F0F0Fu, ((q[n][k] >> 4) ^ 0x08080808u) & 0x0F0F0F0Fu, X.h[2 * k],
+                 X.h[2 * k + 1], X.l[2 * k], X.l[2 * k + 1], h[n], l[n]);
 #pragma unroll
-      for (int n = 0; n < NR; ++n) {
-        dot8_i4(q[n][k], &x[8 * k], a[n][0], a[n][1], a[n][2], a[n][3]);
-        dot8_i4(q[n][k + 1], &x[8 * k + 8], b[n][0], b[n][1], b[n][2], b[n][3]);
-      }
-#pragma unroll
-    for (int n = 0; n < NR; ++n)
-      out[n] = (((a[n][0] + a[n][1]) + (a[n][2] + a[n][3])) + ((b[n][0] + b[n][1]) + (b[n][2] + b[n][3]))) - (c0 + c1);
+    for (int n = 0; n < NR; ++n) out[n] = X.s * float(h[n] * 256 + l[n]);
   }
 }
 
@@ -303,7 +361,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 template <int KIND, int MAXP>
 __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi, int ra, int rbnd, uint8_t* ring,
                                             float* xs, float* red, uint64_t* full, uint64_t* xfull, uint64_t* xfree,
-                                            uint64_t* empty, int& s, int& xs_n, float (&X)[64]) {
+                                            uint64_t* empty, int& s, int& xs_n, XUnit& X) {
   const GemvProb& P = prm.p[pi];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = P.units, row_bytes = P.row_bytes;
@@ -317,8 +375,7 @@ __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi,
 
   // x was bulk-copied into xs by the producer; load this thread's x values into registers
   if (!mbar_wait(xfull, uint32_t(xs_n) & 1u)) return false;
-  float c0 = 0.f, c1 = 0.f;
-  if (active) build_x(KIND, xs + size_t(p) * UW, X, c0, c1);
+  if (active) build_x<KIND>(xs + size_t(p) * UW, X);
   mbar_arrive(xfree);
   ++xs_n;
 
@@ -342,11 +399,11 @@ __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi,
         if (active) {
           if (two) {
             const uint32_t u2[2] = {base + uint32_t(i) * row_bytes, base + uint32_t(i + groups) * row_bytes};
-            units_dot<KIND, 2>(u2, X, c0, c1, v);
+            units_dot<KIND, 2>(u2, X, v);
           } else {
             const uint32_t u1[1] = {base + uint32_t(i) * row_bytes};
             float o1[1];
-            units_dot<KIND, 1>(u1, X, c0, c1, o1);
+            units_dot<KIND, 1>(u1, X, o1);
             v[0] = o1[0];
           }
         }
@@ -480,7 +537,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
   // ------------------------------------------------ consumer warps
   int s = 0;     // stage counter (same sequence as the producer's, and in every consumer warp)
   int xs_n = 0;  // problems whose x has been read
-  float X[64];
+  XUnit X;
   for (int pi = cr.p0; pi <= p_last; ++pi) {
     const GemvProb& P = prm.p[pi];
     int ra, rbnd;

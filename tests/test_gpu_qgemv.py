@@ -34,11 +34,11 @@ def _run(fmt, rows, cols, seed=0):
 def test_qgemv_matches_oracle(fmt, rows, cols):
     y, ref = _run(fmt, rows, cols)
     assert_close(y, ref, what=f"fmt {fmt} {rows}x{cols}")
-    # Exact dequantized products with fp32 sums: far inside the tolerance on outputs of many
-    # rows (the 128+q float encoding of nibbles costs a few bits on one-block rows, so tiny
-    # outputs are held to the specified bound only); 1e-4 still catches any misread weight.
+    # Exact integer block sums; the only approximation is x in 16-bit fixed point per unit of
+    # 32/64 values (|x_i - s X_i| <= max|x| / 65534, about 3e-5 of a typical |y|), so outputs
+    # of many rows stay far inside the tolerance; 2e-4 still catches any misread weight.
     if rows >= 64:
-        assert_close(y, ref, tol=1e-4, what=f"fmt {fmt} {rows}x{cols} (fp32 accuracy)")
+        assert_close(y, ref, tol=2e-4, what=f"fmt {fmt} {rows}x{cols} (x fixed-point accuracy)")
 
 
 def test_q8_0_2048_config_seed0():
@@ -124,7 +124,7 @@ def test_tinyllama_decode_step_full_size_sampled():
         ref = np.array([oq.qgemv(s.fmt, synth.matrix(s.fmt, s.rows, s.cols, 0, s.name, r0=r, r1=r + 1).numpy(),
                                  xs[s.x_name], 1, s.cols)[0] for r in sel])
         assert_close(y, ref, what=s.name)
-        assert_close(y, ref, tol=1e-4, what=s.name + " (fp32 accuracy)")
+        assert_close(y, ref, tol=2e-4, what=s.name + " (x fixed-point accuracy)")
     assert W.weight_bytes == 614_629_376
 
 
