@@ -7,16 +7,20 @@
 // summary, "핵심 아이디어" and "구현 범위" (256 routed int4 experts with per-row scales).
 //
 // Steps (all on the caller's stream):
-//   1. k_moe_route    one CTA: per-expert counts, offsets, the list of touched experts and a
+//   1. k_moe_prep     block 0: per-expert counts, offsets, the list of touched experts and a
 //                     stable permutation of the (token, slot) pairs grouped by expert, in token
-//                     order.  Expert ids outside [0, E) are skipped and flagged.
-//   2. k_moe_grouped  (phase gate/up) every touched expert's gate and up rows are streamed once
-//                     (bulk copies into shared memory, next tile prefetched) and applied to all
-//                     of its tokens; h = act(g) * u is written per pair.  The shared expert is
-//                     one more work list over all tokens.
-//   3. k_moe_grouped  (phase down) the same over the down matrices, x = h of each pair; writes
-//                     one output row per pair (and the shared output).
-//   4. k_moe_combine  y_t = sum_j w_tj * out_(t,j) in slot order, plus the shared output.
+//                     order (expert ids outside [0, E) are skipped and flagged); it also zeroes
+//                     the work counters.  Other blocks: x of every token in the integer form
+//                     the GEMV kernel uses (16-bit fixed point per unit, see XUnit).
+//   2. k_moe_gemv     (gate/up) a persistent grouped GEMV over work items = stages of up to
+//                     72 KB of rows of one matrix of one touched expert (or of the shared
+//                     expert).  Each stage is bulk-copied into shared memory ONCE and applied
+//                     to every token routed to that expert, so each touched expert's bytes
+//                     are read from HBM once per call.  Items are claimed from a counter, the
+//                     shared expert's (all tokens) first.  Outputs g and u per pair.
+//   3. k_moe_quant    h = act(g) * u per pair (and for the shared expert), in the integer form.
+//   4. k_moe_gemv     (down) the same over the down matrices; one output row per pair.
+//   5. k_moe_combine  y_t = sum_j w_tj * out_(t,j) in slot order, plus the shared output.
 // Every sum has a fixed order, so results are deterministic.
 #pragma once
 
@@ -26,23 +30,138 @@
 
 namespace bqg {
 
-// ---------------------------------------------------------------- 1. route grouping
-constexpr int kRouteThreads = 1024;
+// ---------------------------------------------------------------- activations in integer form
+// Records of XUnit in global memory: words [0, UW/4) high bytes, [UW/4, UW/2) low bytes, then
+// c0, c1, s; padded to whole 16-byte chunks (9 chunks for 64-value units, 5 for 32).
+__host__ __device__ constexpr int xrec_chunks(int kind) { return unit_weights(kind) == 64 ? 9 : 5; }
 
-struct RouteWs {
-  int32_t* counts;   // [E]
-  int32_t* offsets;  // [E + 1]
-  int32_t* active;   // [E] touched experts in increasing id order
-  int32_t* n_active; // [1]
-  int32_t* perm;     // [T * k] pair ids (t * k + j) grouped by expert, token order inside
+template <int KIND>
+__device__ __forceinline__ void store_xunit(const XUnit& X, uint4* rec) {
+  constexpr int UW = unit_weights(KIND), NW = UW / 4;
+  uint32_t w[4 * xrec_chunks(KIND)];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    w[i] = X.h[i];
+    w[NW + i] = X.l[i];
+  }
+  w[2 * NW] = uint32_t(X.c0);
+  w[2 * NW + 1] = uint32_t(X.c1);
+  w[2 * NW + 2] = __float_as_uint(X.s);
+#pragma unroll
+  for (int i = 2 * NW + 3; i < 4 * xrec_chunks(KIND); ++i) w[i] = 0u;
+#pragma unroll
+  for (int c = 0; c < xrec_chunks(KIND); ++c) rec[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+
+template <int KIND>
+__device__ __forceinline__ void load_xunit(const uint4* rec, XUnit& X) {
+  constexpr int NW = unit_weights(KIND) / 4;
+#pragma unroll
+  for (int c = 0; c < xrec_chunks(KIND); ++c) {
+    const uint4 v = __ldg(rec + c);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 4 * c + k;  // compile-time after unrolling
+      if (i < NW) X.h[i] = w4[k];
+      else if (i < 2 * NW) X.l[i - NW] = w4[k];
+      else if (i == 2 * NW) X.c0 = int(w4[k]);
+      else if (i == 2 * NW + 1) X.c1 = int(w4[k]);
+      else if (i == 2 * NW + 2) X.s = __uint_as_float(w4[k]);
+    }
+  }
+}
+
+__device__ __forceinline__ float act_fn(int act, float g) {
+  if (act == BQG_ACT_SILU) return g / (1.f + expf(-g));
+  const float c = 0.7978845608028654f;  // sqrt(2/pi)
+  return 0.5f * g * (1.f + tanhf(c * (g + 0.044715f * g * g * g)));
+}
+
+// One conversion job: rows x cols values (row stride cols) -> records [rows][cols / UW].
+// With b != nullptr the values are act(a) * b (the gated FFN's hidden activation).
+struct QuantJob {
+  const float* a;
+  const float* b;
+  uint4* dst;
+  int rows, cols, kind, act;
+};
+struct QuantJobs {
+  QuantJob j[2];
+  int n;
 };
 
-__global__ void __launch_bounds__(kRouteThreads) k_moe_route(const int32_t* __restrict__ idx, int pairs,
-                                                             int n_experts, RouteWs ws) {
+template <int KIND>
+__device__ __forceinline__ void quant_one(const QuantJob& J, int row, int u) {
+  constexpr int UW = unit_weights(KIND);
+  const size_t off = size_t(row) * J.cols + size_t(u) * UW;
+  float xv[UW];
+#pragma unroll
+  for (int i = 0; i < UW / 4; ++i) {
+    const float4 v = *reinterpret_cast<const float4*>(J.a + off + 4 * i);
+    xv[4 * i] = v.x;
+    xv[4 * i + 1] = v.y;
+    xv[4 * i + 2] = v.z;
+    xv[4 * i + 3] = v.w;
+  }
+  if (J.b != nullptr) {
+#pragma unroll
+    for (int i = 0; i < UW / 4; ++i) {
+      const float4 v = *reinterpret_cast<const float4*>(J.b + off + 4 * i);
+      xv[4 * i] = act_fn(J.act, xv[4 * i]) * v.x;
+      xv[4 * i + 1] = act_fn(J.act, xv[4 * i + 1]) * v.y;
+      xv[4 * i + 2] = act_fn(J.act, xv[4 * i + 2]) * v.z;
+      xv[4 * i + 3] = act_fn(J.act, xv[4 * i + 3]) * v.w;
+    }
+  }
+  XUnit X;
+  quantize_unit<KIND>(xv, X);
+  store_xunit<KIND>(X, J.dst + (size_t(row) * (J.cols / UW) + u) * xrec_chunks(KIND));
+}
+
+// Converts every unit of the jobs; thread i of nthreads takes units i, i + nthreads, ...
+__device__ __forceinline__ void quant_jobs(const QuantJobs& Q, long long i0, long long nthreads) {
+  for (int jn = 0; jn < Q.n; ++jn) {
+    const QuantJob& J = Q.j[jn];
+    const int units = J.cols / unit_weights(J.kind);
+    const long long total = (long long)J.rows * units;
+    for (long long i = i0; i < total; i += nthreads) {
+      const int row = int(i / units), u = int(i - (long long)row * units);
+      switch (J.kind) {
+        case kQ4Pair: quant_one<kQ4Pair>(J, row, u); break;
+        case kQ4One: quant_one<kQ4One>(J, row, u); break;
+        case kQ8Pair: quant_one<kQ8Pair>(J, row, u); break;
+        case kQ8One: quant_one<kQ8One>(J, row, u); break;
+        case kI4x64: quant_one<kI4x64>(J, row, u); break;
+        default: quant_one<kI4x32>(J, row, u); break;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) k_moe_quant(const __grid_constant__ QuantJobs Q) {
+  quant_jobs(Q, (long long)blockIdx.x * blockDim.x + threadIdx.x, (long long)gridDim.x * blockDim.x);
+}
+
+// ---------------------------------------------------------------- 1. route grouping
+constexpr int kRouteThreads = 512;
+
+struct RouteWs {
+  int32_t* counts;    // [E]
+  int32_t* offsets;   // [E + 1]
+  int32_t* active;    // [E] touched experts in increasing id order
+  int32_t* n_active;  // [1]
+  int32_t* perm;      // [T * k] pair ids (t * k + j) grouped by expert, token order inside
+  uint32_t* ctr;      // [2] work item counters of the two grouped GEMV launches
+};
+
+__device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int pairs, int n_experts,
+                                          const RouteWs& ws) {
   __shared__ int cnt[BQG_MAX_EXPERTS];
   __shared__ int base[BQG_MAX_EXPERTS];
   __shared__ int wcnt[kRouteThreads / 32][BQG_MAX_EXPERTS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid < 2) ws.ctr[tid] = 0u;
   for (int e = tid; e < n_experts; e += kRouteThreads) cnt[e] = 0;
   __syncthreads();
   bool bad = false;
@@ -97,405 +216,247 @@ __global__ void __launch_bounds__(kRouteThreads) k_moe_route(const int32_t* __re
   }
 }
 
-// ---------------------------------------------------------------- 2/3. grouped expert GEMM
-constexpr int kMoeThreads = 256;                 // 8 warps
-constexpr int kMoeSlotBytes = 72 * 1024;         // weight tile buffer (x2: current + prefetch)
-constexpr int kMoeXBytes = 64 * 1024;            // token tile of activations
-constexpr int kMoeMaxTok = 8;                    // tokens per token tile
-constexpr int kMoeMaxVRows = 32;                 // rows per tile (both matrices together)
-constexpr size_t kMoeSmemBytes = 2 * size_t(kMoeSlotBytes + 64) + kMoeXBytes +
-                                 size_t(2 * kMoeMaxTok * kMoeMaxVRows) * sizeof(float) + 64;
-
-struct MoeMat {          // one family of stacked matrices (gate, up or down of all experts)
-  const uint8_t* base;   // expert e's matrix at base + e * stride
-  long long stride;
-  int rows, cols;        // of one expert's matrix
-  int kind, row_bytes, units, scale_off;
-};
-
-struct MoePhase {
-  // routed experts
-  MoeMat m0, m1;         // gate/up phase: m0 = gate, m1 = up; down phase: m0 = down
-  int nmat;              // 2 (gate/up) or 1 (down)
-  int lpr;               // lanes per row: 8, 16 or 32
-  int tile_rows;         // rows of one matrix per tile
-  int tiles;             // tiles per expert
-  int tb;                // tokens per token tile
-  // shared expert (optional)
-  MoeMat s0, s1;
-  int s_present;
-  int s_lpr, s_tile_rows, s_tiles, s_tb;
-  // activations
-  const float* xin;      // gate/up: x [T x hidden]; down: h [pairs x inter]
-  const float* s_xin;    // down: shared h [T x shared_inter]
-  float* out;            // gate/up: h [pairs x inter]; down: per-pair output [pairs x hidden]
-  float* s_out;          // gate/up: shared h; down: shared output [T x hidden]
-  int xin_stride, s_xin_stride, out_stride, s_out_stride;
-  int gateup;            // 1: gate/up phase (epilogue act(g) * u), 0: down phase
-  int act;
-  int tokens, top_k;
-  RouteWs route;
-};
-
-__device__ __forceinline__ float act_fn(int act, float g) {
-  if (act == BQG_ACT_SILU) return g / (1.f + expf(-g));
-  const float c = 0.7978845608028654f;  // sqrt(2/pi)
-  return 0.5f * g * (1.f + tanhf(c * (g + 0.044715f * g * g * g)));
-}
-
-// Decodes one unit into exact fp32 weight values (without the I4 row scale).
-template <int KIND>
-__device__ __forceinline__ void unit_decode(const uint8_t* u, float (&w)[64]) {
-  if constexpr (KIND == kQ4Pair || KIND == kQ4One) {
-    uint32_t v[9];
-    uint32_t q[8];
-    float dA, dB = 0.f;
-    if constexpr (KIND == kQ4Pair) {
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(u);
-#pragma unroll
-      for (int i = 0; i < 9; ++i) v[i] = p[i];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) q[k] = __funnelshift_r(v[k], v[k + 1], 16);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) q[4 + k] = v[5 + k];
-      dA = half_bits_to_float(v[0]);
-      dB = half_bits_to_float(v[4] >> 16);
-    } else {
-      const uintptr_t a = reinterpret_cast<uintptr_t>(u);
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(a & ~uintptr_t(3));
-      const uint32_t sh = uint32_t(a & 2) * 8;
-#pragma unroll
-      for (int i = 0; i < 5; ++i) v[i] = p[i];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) q[k] = __funnelshift_rc(v[k], v[k + 1], 16 + sh);
-      dA = half_bits_to_float(__funnelshift_r(v[0], v[1], sh));
-    }
-    constexpr int NW = (KIND == kQ4Pair) ? 8 : 4;
-#pragma unroll
-    for (int k = 0; k < NW; ++k) {
-      const float d = k < 4 ? dA : dB;
-      const float c = -136.f * d;
-      const uint32_t lo = q[k] & 0x0F0F0F0Fu, hi = (q[k] >> 4) & 0x0F0F0F0Fu;
-      // (128 + q) * d - 136 d = (q - 8) * d, exact in fp32
-      w[8 * k + 0] = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4055u)), d, c);
-      w[8 * k + 1] = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4055u)), d, c);
-      w[8 * k + 2] = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4155u)), d, c);
-      w[8 * k + 3] = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4155u)), d, c);
-      w[8 * k + 4] = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4255u)), d, c);
-      w[8 * k + 5] = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4255u)), d, c);
-      w[8 * k + 6] = fmaf(__uint_as_float(__byte_perm(lo, 0x43u, 0x4355u)), d, c);
-      w[8 * k + 7] = fmaf(__uint_as_float(__byte_perm(hi, 0x43u, 0x4355u)), d, c);
-    }
-  } else if constexpr (KIND == kQ8Pair || KIND == kQ8One) {
-    uint32_t v[17];
-    uint32_t q[16];
-    float dA, dB = 0.f;
-    if constexpr (KIND == kQ8Pair) {
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(u);
-#pragma unroll
-      for (int i = 0; i < 17; ++i) v[i] = p[i];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q[k] = __funnelshift_r(v[k], v[k + 1], 16);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q[8 + k] = v[9 + k];
-      dA = half_bits_to_float(v[0]);
-      dB = half_bits_to_float(v[8] >> 16);
-    } else {
-      const uintptr_t a = reinterpret_cast<uintptr_t>(u);
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(a & ~uintptr_t(3));
-      const uint32_t sh = uint32_t(a & 2) * 8;
-#pragma unroll
-      for (int i = 0; i < 9; ++i) v[i] = p[i];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q[k] = __funnelshift_rc(v[k], v[k + 1], 16 + sh);
-      dA = half_bits_to_float(__funnelshift_r(v[0], v[1], sh));
-    }
-    constexpr int NW = (KIND == kQ8Pair) ? 16 : 8;
-    const float off = 8388736.0f;  // 2^23 + 128
-#pragma unroll
-    for (int k = 0; k < NW; ++k) {
-      const float d = k < 8 ? dA : dB;
-      const uint32_t s = q[k] ^ 0x80808080u;
-      w[4 * k + 0] = (__uint_as_float(__byte_perm(s, 0x4Bu, 0x4550u)) - off) * d;
-      w[4 * k + 1] = (__uint_as_float(__byte_perm(s, 0x4Bu, 0x4551u)) - off) * d;
-      w[4 * k + 2] = (__uint_as_float(__byte_perm(s, 0x4Bu, 0x4552u)) - off) * d;
-      w[4 * k + 3] = (__uint_as_float(__byte_perm(s, 0x4Bu, 0x4553u)) - off) * d;
-    }
-  } else {  // int4 with per-row scale (applied after the dot product)
-    constexpr int NW = (KIND == kI4x64) ? 8 : 4;
-    const uint4* p = reinterpret_cast<const uint4*>(u);
-    uint32_t q[8];
-    const uint4 a = p[0];
-    q[0] = a.x; q[1] = a.y; q[2] = a.z; q[3] = a.w;
-    if constexpr (NW == 8) {
-      const uint4 b = p[1];
-      q[4] = b.x; q[5] = b.y; q[6] = b.z; q[7] = b.w;
-    }
-#pragma unroll
-    for (int k = 0; k < NW; ++k) {
-      const uint32_t lo = (q[k] ^ 0x08080808u) & 0x0F0F0F0Fu, hi = ((q[k] >> 4) ^ 0x08080808u) & 0x0F0F0F0Fu;
-      w[8 * k + 0] = __uint_as_float(__byte_perm(lo, 0x43u, 0x4055u)) - 136.f;
-      w[8 * k + 1] = __uint_as_float(__byte_perm(hi, 0x43u, 0x4055u)) - 136.f;
-      w[8 * k + 2] = __uint_as_float(__byte_perm(lo, 0x43u, 0x4155u)) - 136.f;
-      w[8 * k + 3] = __uint_as_float(__byte_perm(hi, 0x43u, 0x4155u)) - 136.f;
-      w[8 * k + 4] = __uint_as_float(__byte_perm(lo, 0x43u, 0x4255u)) - 136.f;
-      w[8 * k + 5] = __uint_as_float(__byte_perm(hi, 0x43u, 0x4255u)) - 136.f;
-      w[8 * k + 6] = __uint_as_float(__byte_perm(lo, 0x43u, 0x4355u)) - 136.f;
-      w[8 * k + 7] = __uint_as_float(__byte_perm(hi, 0x43u, 0x4355u)) - 136.f;
-    }
-  }
-}
-
-__device__ __forceinline__ void unit_decode_any(int kind, const uint8_t* u, float (&w)[64]) {
-  switch (kind) {
-    case kQ4Pair: unit_decode<kQ4Pair>(u, w); break;
-    case kQ8Pair: unit_decode<kQ8Pair>(u, w); break;
-    case kI4x64: unit_decode<kI4x64>(u, w); break;
-    case kQ4One: unit_decode<kQ4One>(u, w); break;
-    case kQ8One: unit_decode<kQ8One>(u, w); break;
-    default: unit_decode<kI4x32>(u, w); break;
-  }
-}
-
-// Work item -> (which list, expert, tile).  Routed items first, then the shared expert's.
-struct MoeItem {
-  int shared;   // 0 routed, 1 shared
-  int expert;   // routed expert id
-  int tile;
-  int ntok;     // tokens of this expert
-  int tok0;     // offset into perm (routed)
-};
-
-__device__ __forceinline__ bool moe_item(const MoePhase& P, int n_active, int item, MoeItem& it) {
-  const int routed = n_active * P.tiles;
-  if (item < routed) {
-    const int a = item / P.tiles;
-    it.shared = 0;
-    it.expert = P.route.active[a];
-    it.tile = item - a * P.tiles;
-    it.tok0 = P.route.offsets[it.expert];
-    it.ntok = P.route.counts[it.expert];
-    return true;
-  }
-  item -= routed;
-  if (P.s_present && item < P.s_tiles) {
-    it.shared = 1;
-    it.expert = 0;
-    it.tile = item;
-    it.tok0 = 0;
-    it.ntok = P.tokens;
-    return true;
-  }
-  return false;
-}
-
-struct TileGeom {
-  const MoeMat* m[2];
-  int nmat, lpr, tile_rows, tb, r0, r1;
-};
-
-__device__ __forceinline__ TileGeom tile_geom(const MoePhase& P, const MoeItem& it) {
-  TileGeom g;
-  if (!it.shared) {
-    g.m[0] = &P.m0; g.m[1] = &P.m1; g.nmat = P.nmat; g.lpr = P.lpr; g.tile_rows = P.tile_rows; g.tb = P.tb;
+// Block 0 groups the routes; the other blocks convert x (jobs in Q).
+__global__ void __launch_bounds__(kRouteThreads, 1) k_moe_prep(const int32_t* __restrict__ idx, int pairs,
+                                                            int n_experts, RouteWs ws,
+                                                            const __grid_constant__ QuantJobs Q) {
+  if (blockIdx.x == 0) {
+    moe_route(idx, pairs, n_experts, ws);
   } else {
-    g.m[0] = &P.s0; g.m[1] = &P.s1; g.nmat = P.nmat; g.lpr = P.s_lpr; g.tile_rows = P.s_tile_rows; g.tb = P.s_tb;
-  }
-  g.r0 = it.tile * g.tile_rows;
-  g.r1 = min(g.r0 + g.tile_rows, g.m[0]->rows);
-  return g;
-}
-
-// Byte offset of matrix m's rows inside a slot (16-byte aligned sub-buffers).
-__device__ __forceinline__ int slot_sub_offset(const TileGeom& g, int m) {
-  return m == 0 ? 0 : ((g.tile_rows * g.m[0]->row_bytes + 47) / 16) * 16;
-}
-
-// Producer side: issue the bulk copies of one item's weight tile into `slot` (thread 0).
-__device__ __forceinline__ void issue_tile(const MoeItem& it, const TileGeom& g, uint8_t* slot, uint64_t* bar,
-                                           uint64_t pol) {
-  uint32_t total = 0;
-  for (int m = 0; m < g.nmat; ++m) {
-    const MoeMat& M = *g.m[m];
-    const uintptr_t wbeg = reinterpret_cast<uintptr_t>(M.base) + (it.shared ? 0 : size_t(it.expert) * M.stride);
-    const uintptr_t wend = wbeg + size_t(M.rows) * M.row_bytes;
-    const uintptr_t src = wbeg + size_t(g.r0) * M.row_bytes;
-    const uintptr_t end = src + size_t(g.r1 - g.r0) * M.row_bytes;
-    const uintptr_t a0 = src & ~uintptr_t(15);
-    const uintptr_t lim = wend & ~uintptr_t(15);
-    uintptr_t a1 = (end + 15) & ~uintptr_t(15);
-    if (a1 > lim) a1 = lim;
-    if (a1 < a0) a1 = a0;
-    uint8_t* dst = slot + slot_sub_offset(g, m);
-    for (uintptr_t b = (a1 > src ? a1 : src); b < end; ++b) dst[b - a0] = *reinterpret_cast<const uint8_t*>(b);
-    total += uint32_t(a1 - a0);
-  }
-  mbar_arrive_expect_tx(bar, total);
-  for (int m = 0; m < g.nmat; ++m) {
-    const MoeMat& M = *g.m[m];
-    const uintptr_t wbeg = reinterpret_cast<uintptr_t>(M.base) + (it.shared ? 0 : size_t(it.expert) * M.stride);
-    const uintptr_t wend = wbeg + size_t(M.rows) * M.row_bytes;
-    const uintptr_t src = wbeg + size_t(g.r0) * M.row_bytes;
-    const uintptr_t end = src + size_t(g.r1 - g.r0) * M.row_bytes;
-    const uintptr_t a0 = src & ~uintptr_t(15);
-    const uintptr_t lim = wend & ~uintptr_t(15);
-    uintptr_t a1 = (end + 15) & ~uintptr_t(15);
-    if (a1 > lim) a1 = lim;
-    if (a1 < a0) a1 = a0;
-    if (a1 > a0) bulk_g2s(slot + slot_sub_offset(g, m), reinterpret_cast<const void*>(a0), uint32_t(a1 - a0), bar, pol);
+    quant_jobs(Q, (long long)(blockIdx.x - 1) * blockDim.x + threadIdx.x, (long long)(gridDim.x - 1) * blockDim.x);
   }
 }
 
-__global__ void __launch_bounds__(kMoeThreads, 1) k_moe_grouped(const __grid_constant__ MoePhase P) {
+// ---------------------------------------------------------------- 2/4. grouped GEMV
+// The same producer/consumer structure, stage ring and integer dot products as k_qgemv; a
+// work item is one stage of rows of one matrix, applied to all the tokens routed to it.
+struct MgMat {            // one family of stacked matrices (gate, up or down of all experts)
+  const uint8_t* base;    // expert e's matrix at base + e * stride (stride 0: the shared expert)
+  long long stride;
+  int rows, cols;         // of one expert's matrix
+  int kind, row_bytes, units, scale_off;
+  int stage_rows, nstages;
+};
+
+struct MgPhase {
+  MgMat m[4];             // 0, 1: routed families; 2, 3: shared families
+  int nmat;               // routed families (1 or 2; they share one shape)
+  int s_nmat;             // shared families (0, 1 or 2; they share one shape)
+  const uint4* xq;        // routed input records [input rows][units of m[0]]
+  const uint4* s_xq;      // shared input records [tokens][units of m[2]]
+  float* out[4];          // per family: routed [pairs][rows], shared [tokens][rows]
+  int x_by_token;         // routed input row = pair / top_k (gate/up) or the pair (down)
+  int top_k, tokens;
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* active;
+  const int32_t* n_active;
+  const int32_t* perm;
+  uint32_t* ctr;          // work item counter (zeroed by k_moe_prep)
+};
+
+__device__ __forceinline__ int4 ld_desc(const int4* d) {
+  int4 v;
+  asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(d))
+               : "memory");
+  return v;
+}
+
+constexpr size_t kMgSmemBytes = size_t(kGemvStages) * kGemvStageAlloc +
+                                size_t(2 * kGemvConsumerWarps * kGemvRedRows) * sizeof(float) +
+                                (2 * kGemvStages) * sizeof(uint64_t) + size_t(kGemvStages) * sizeof(int4);
+
+// Consumer side of one item (stage `slot` holds rows [r0, r1) of family fam, expert e).
+// q counts token iterations (selects the group reduction buffer).
+template <int KIND>
+__device__ __forceinline__ void mg_item(const MgPhase& P, int fam, int e, int r0, int r1, uint32_t stage_s,
+                                        float* red, int& q) {
+  const MgMat& M = P.m[fam];
+  const bool shared = fam >= 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = M.units, row_bytes = M.row_bytes;
+  const int gw = gemv_group_warps(units);
+  const int groups = gemv_groups(units);
+  const int g = warp / gw, j = warp - g * gw;
+  const int p = 32 * j + lane;
+  const bool in_group = g < groups;
+  const bool active = in_group && p < units;
+  constexpr int UB = unit_bytes(KIND);
+  const uint8_t* wbase = M.base + (shared ? 0 : size_t(e) * M.stride);
+  const uint32_t src_lo = uint32_t(reinterpret_cast<uintptr_t>(wbase) + size_t(r0) * row_bytes) & 15u;
+  const uint32_t base = stage_s + src_lo + uint32_t(p) * UB;
+  const float* scales = reinterpret_cast<const float*>(wbase + M.scale_off);
+  const int nrows = r1 - r0;
+  const int ntok = shared ? P.tokens : P.counts[e];
+  const int32_t* list = shared ? nullptr : P.perm + P.offsets[e];
+  const uint4* xq = shared ? P.s_xq : P.xq;
+  float* out = P.out[fam];
+  for (int tt = 0; tt < ntok; ++tt, ++q) {
+    const int pid = shared ? tt : __ldg(list + tt);
+    const int xrow = (shared || !P.x_by_token) ? pid : pid / P.top_k;
+    XUnit X;
+    if (active) load_xunit<KIND>(xq + (size_t(xrow) * units + p) * xrec_chunks(KIND), X);
+    float* orow = out + size_t(pid) * M.rows + r0;
+    const int par = q & 1;
+    int nmine = 0;
+    if (in_group) {
+      for (int i = g; i < nrows; i += 2 * groups) {
+        const bool two = i + groups < nrows;
+        float v[2] = {0.f, 0.f};
+        if (active) {
+          if (two) {
+            const uint32_t u2[2] = {base + uint32_t(i) * row_bytes, base + uint32_t(i + groups) * row_bytes};
+            units_dot<KIND, 2>(u2, X, v);
+          } else {
+            const uint32_t u1[1] = {base + uint32_t(i) * row_bytes};
+            float o1[1];
+            units_dot<KIND, 1>(u1, X, o1);
+            v[0] = o1[0];
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+          v[1] += __shfl_xor_sync(0xffffffffu, v[1], o);
+        }
+        if (lane == 0) {
+          if (gw == 1) {
+            if (is_i4(KIND)) v[0] *= __ldg(scales + r0 + i);
+            orow[i] = v[0];
+            if (two) {
+              if (is_i4(KIND)) v[1] *= __ldg(scales + r0 + i + groups);
+              orow[i + groups] = v[1];
+            }
+          } else {
+            red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine] = v[0];
+            if (two) red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine + 1] = v[1];
+          }
+        }
+        nmine += two ? 2 : 1;
+      }
+    }
+    if (gw > 1 && in_group) {
+      named_bar_sync(2 + g, 32 * gw);
+      if (j == 0 && lane < nmine) {
+        float v = 0.f;
+        for (int jj = 0; jj < gw; ++jj) v += red[(par * kGemvConsumerWarps + g * gw + jj) * kGemvRedRows + lane];
+        const int i = g + lane * groups;
+        if (is_i4(KIND)) v *= __ldg(scales + r0 + i);
+        orow[i] = v;
+      }
+    }
+  }
+}
+
+// KR: unit kind of the routed families, KS: of the shared ones (one kernel per pair keeps each
+// consumer path within the register budget).
+template <int KR, int KS>
+__global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_constant__ MgPhase P) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* slots[2] = {smem, smem + kMoeSlotBytes + 64};
-  float* xs = reinterpret_cast<float*>(smem + 2 * size_t(kMoeSlotBytes + 64));
-  float* epi = xs + kMoeXBytes / 4;                       // [2][kMoeMaxTok][kMoeMaxVRows]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(epi + 2 * kMoeMaxTok * kMoeMaxVRows);
-  __shared__ int s_tok[kMoeMaxTok];                       // token (or pair) of each tile slot
+  uint8_t* ring = smem;
+  float* red = reinterpret_cast<float*>(smem + size_t(kGemvStages) * kGemvStageAlloc);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kGemvConsumerWarps * kGemvRedRows);
+  uint64_t* empty = full + kGemvStages;
+  int4* desc = reinterpret_cast<int4*>(empty + kGemvStages);  // (family, expert, r0, r1)
 
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGemvStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kGemvConsumerWarps);
+    }
     fence_barrier_init();
   }
   __syncthreads();
-  const int n_active = *P.route.n_active;
-  const uint64_t pol = policy_evict_first();
 
-  int item = blockIdx.x;
-  MoeItem it;
-  bool have = moe_item(P, n_active, item, it);
-  if (have && tid == 0) issue_tile(it, tile_geom(P, it), slots[0], &bars[0], pol);
-  int phase[2] = {0, 0};
-  int cur = 0;
-  while (have) {
-    const TileGeom g = tile_geom(P, it);
-    // prefetch the next item into the other slot (its previous contents were consumed and
-    // released by the __syncthreads at the end of the last iteration)
-    MoeItem nx;
-    const int nitem = item + gridDim.x;
-    const bool nhave = moe_item(P, n_active, nitem, nx);
-    if (nhave && tid == 0) issue_tile(nx, tile_geom(P, nx), slots[cur ^ 1], &bars[cur ^ 1], pol);
-
-    if (!mbar_wait(&bars[cur], uint32_t(phase[cur]))) return;
-    phase[cur] ^= 1;
-
-    // geometry of this tile
-    const MoeMat& M0 = *g.m[0];
-    const int kind = M0.kind, units = M0.units, ub = unit_bytes(kind), uw = unit_weights(kind);
-    const int xstride_u = uw + 4;                 // padded floats per unit in the x tile
-    const int rows_per_pass = kMoeThreads / g.lpr;
-    const int nrows = g.r1 - g.r0;
-    const int vrows = nrows * g.nmat;             // rows of both matrices
-    const int my_vr = tid / g.lpr, my_l = tid % g.lpr;
-    const int cols = M0.cols;
-    const float* xin = it.shared ? P.s_xin : P.xin;
-    const int xin_stride = it.shared ? P.s_xin_stride : P.xin_stride;
-
-    for (int j0 = 0; j0 < it.ntok; j0 += g.tb) {
-      const int nt = min(g.tb, it.ntok - j0);
-      // token ids of this token tile
-      if (tid < nt) {
-        const int jj = j0 + tid;
-        s_tok[tid] = it.shared ? jj : P.route.perm[it.tok0 + jj];
+  if (warp == kGemvConsumerWarps) {
+    // ------------------------------------------------ producer (one elected lane)
+    if (lane != 0) return;
+    const uint64_t pol = policy_evict_first();
+    const int na = *P.n_active;
+    const int n_sh = P.s_nmat * P.m[2].nstages;
+    const int per_expert = P.nmat * P.m[0].nstages;
+    const int n_items = n_sh + na * per_expert;
+    int s = 0;
+    bool ok = true;
+    int item = int(atomicAdd(P.ctr, 1u));
+    while (item < n_items) {
+      const int next = int(atomicAdd(P.ctr, 1u));  // claimed one item ahead
+      int fam, e = 0, k;
+      if (item < n_sh) {
+        fam = 2 + item / P.m[2].nstages;
+        k = item - (fam - 2) * P.m[2].nstages;
+      } else {
+        int r = item - n_sh;
+        const int a = r / per_expert;
+        r -= a * per_expert;
+        fam = r / P.m[0].nstages;
+        k = r - fam * P.m[0].nstages;
+        e = __ldg(P.active + a);
       }
-      __syncthreads();
-      // stage x rows into the padded tile layout: unit u at u * (uw + 4) floats
-      const int c4 = cols / 4;
-      for (int i = tid; i < nt * c4; i += kMoeThreads) {
-        const int j = i / c4, c = (i - j * c4) * 4;
-        const int pid = s_tok[j];
-        // gate/up reads x of the token; down reads h of the pair (or of the token if shared)
-        const int row = (P.gateup && !it.shared) ? pid / P.top_k : pid;
-        const float4 v = *reinterpret_cast<const float4*>(xin + size_t(row) * xin_stride + c);
-        const int u = c / uw, o = c - u * uw;
-        *reinterpret_cast<float4*>(xs + j * (units * xstride_u) + u * xstride_u + o) = v;
+      const MgMat& M = P.m[fam];
+      const int r0 = k * M.stage_rows;
+      const int r1 = min(r0 + M.stage_rows, M.rows);
+      const int slot = s % kGemvStages;
+      if (s >= kGemvStages && !mbar_wait(&empty[slot], uint32_t(s / kGemvStages - 1) & 1u)) {
+        ok = false;
+        break;
       }
-      __syncthreads();
-
-      // dot products: virtual row vr (matrix vr / nrows, row vr % nrows), lanes split units
-      for (int vr0 = 0; vr0 < vrows; vr0 += rows_per_pass) {
-        const int vr = vr0 + my_vr;
-        float acc[kMoeMaxTok];
-#pragma unroll
-        for (int j = 0; j < kMoeMaxTok; ++j) acc[j] = 0.f;
-        if (vr < vrows) {
-          const int m = vr / nrows, r = vr - m * nrows;
-          const MoeMat& M = *g.m[m];
-          const uintptr_t wbeg = reinterpret_cast<uintptr_t>(M.base) + (it.shared ? 0 : size_t(it.expert) * M.stride);
-          const uintptr_t src = wbeg + size_t(g.r0) * M.row_bytes;
-          const uint8_t* rowp = slots[cur] + slot_sub_offset(g, m) + (src & 15) + size_t(r) * M.row_bytes;
-          for (int u = my_l; u < units; u += g.lpr) {
-            float w[64];
-            unit_decode_any(kind, rowp + size_t(u) * ub, w);
-#pragma unroll
-            for (int j = 0; j < kMoeMaxTok; ++j) {
-              if (j < nt) {
-                const float4* xv = reinterpret_cast<const float4*>(xs + j * (units * xstride_u) + u * xstride_u);
-                float a = acc[j];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                  if (q < uw / 4) {
-                    const float4 x4 = xv[q];
-                    a = fmaf(w[4 * q], x4.x, a);
-                    a = fmaf(w[4 * q + 1], x4.y, a);
-                    a = fmaf(w[4 * q + 2], x4.z, a);
-                    a = fmaf(w[4 * q + 3], x4.w, a);
-                  }
-                }
-                acc[j] = a;
-              }
-            }
-          }
-        }
-        // reduce over the lanes of this row (fixed butterfly inside aligned lane groups)
-#pragma unroll
-        for (int j = 0; j < kMoeMaxTok; ++j) {
-          float a = acc[j];
-          for (int o = g.lpr / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-          acc[j] = a;
-        }
-        if (vr < vrows && my_l == 0) {
-          const int m = vr / nrows, r = vr - m * nrows;
-          const MoeMat& M = *g.m[m];
-          float sc = 1.f;
-          if (M.kind == kI4x64 || M.kind == kI4x32) {
-            const uint8_t* mb = M.base + (it.shared ? 0 : size_t(it.expert) * M.stride);
-            sc = __ldg(reinterpret_cast<const float*>(mb + M.scale_off) + g.r0 + r);
-          }
-#pragma unroll
-          for (int j = 0; j < kMoeMaxTok; ++j) {
-            if (j >= nt) break;
-            const float v = acc[j] * sc;
-            if (P.gateup) {
-              epi[(m * kMoeMaxTok + j) * kMoeMaxVRows + r] = v;
-            } else {
-              float* o = it.shared ? P.s_out : P.out;
-              const int ostride = it.shared ? P.s_out_stride : P.out_stride;
-              o[size_t(s_tok[j]) * ostride + g.r0 + r] = v;
-            }
-          }
-        }
+      fence_proxy_async_smem();
+      desc[slot] = make_int4(fam, e, r0, r1);
+      const uintptr_t wbeg = reinterpret_cast<uintptr_t>(M.base) + (fam >= 2 ? 0 : size_t(e) * M.stride);
+      const uintptr_t wend = wbeg + size_t(M.rows) * M.row_bytes;
+      const uintptr_t src = wbeg + size_t(r0) * M.row_bytes;
+      const uintptr_t end = src + size_t(r1 - r0) * M.row_bytes;
+      const uintptr_t a0 = src & ~uintptr_t(15);
+      const uintptr_t lim = wend & ~uintptr_t(15);
+      uintptr_t a1 = (end + 15) & ~uintptr_t(15);
+      if (a1 > lim) a1 = lim;
+      if (a1 < a0) a1 = a0;
+      uint8_t* dst = ring + size_t(slot) * kGemvStageAlloc;
+      for (uintptr_t b = (a1 > src ? a1 : src); b < end; ++b) dst[b - a0] = *reinterpret_cast<const uint8_t*>(b);
+      const uint32_t nb = uint32_t(a1 - a0);
+      if (nb > 0) {
+        mbar_arrive_expect_tx(&full[slot], nb);
+        bulk_g2s(dst, reinterpret_cast<const void*>(a0), nb, &full[slot], pol);
+      } else {
+        mbar_arrive(&full[slot]);
       }
-      if (P.gateup) {
-        __syncthreads();
-        for (int i = tid; i < nt * nrows; i += kMoeThreads) {
-          const int j = i / nrows, r = i - j * nrows;
-          const float gv = epi[(0 * kMoeMaxTok + j) * kMoeMaxVRows + r];
-          const float uv = epi[(1 * kMoeMaxTok + j) * kMoeMaxVRows + r];
-          float* o = it.shared ? P.s_out : P.out;
-          const int ostride = it.shared ? P.s_out_stride : P.out_stride;
-          o[size_t(s_tok[j]) * ostride + g.r0 + r] = act_fn(P.act, gv) * uv;
-        }
-      }
-      __syncthreads();
+      ++s;
+      item = next;
     }
-    item = nitem;
-    it = nx;
-    have = nhave;
-    cur ^= 1;
+    {  // end marker
+      const int slot = s % kGemvStages;
+      if (ok && (s < kGemvStages || mbar_wait(&empty[slot], uint32_t(s / kGemvStages - 1) & 1u))) {
+        desc[slot] = make_int4(-1, 0, 0, 0);
+        mbar_arrive(&full[slot]);
+      }
+    }
+    if (!ok) {
+      for (int qq = (s > kGemvStages ? s - kGemvStages : 0); qq < s; ++qq)
+        mbar_wait(&full[qq % kGemvStages], uint32_t(qq / kGemvStages) & 1u);
+    }
+    return;
+  }
+
+  // ------------------------------------------------ consumers
+  const uint32_t ring_s = smem_u32(ring);
+  int q = 0;
+  for (int s = 0;; ++s) {
+    const int slot = s % kGemvStages;
+    if (!mbar_wait(&full[slot], uint32_t(s / kGemvStages) & 1u)) return;
+    const int4 d = ld_desc(&desc[slot]);
+    if (d.x < 0) return;
+    // row groups may change from one item to the next: every consumer warp has finished the
+    // previous item (including its group reductions)
+    named_bar_sync(1, kGemvCompute);
+    const uint32_t stage_s = ring_s + uint32_t(slot) * kGemvStageAlloc;
+    if (d.x < 2) mg_item<KR>(P, d.x, d.y, d.z, d.w, stage_s, red, q);
+    else mg_item<KS>(P, d.x, d.y, d.z, d.w, stage_s, red, q);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
   }
 }
 

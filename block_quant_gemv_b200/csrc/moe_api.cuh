@@ -11,26 +11,91 @@ constexpr int kMoeMaxCols = 8192;  // hidden / inter / shared_inter limit of moe
 
 inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
+// Unit kind of a matrix format in the grouped GEMV: one block for Q8_0 and Q4_0 (a row of
+// hidden/inter values then fills more lanes than pairs of blocks would: 88 units for 2816
+// columns, 22 for 704), 64 values for int4 when the columns allow, else 32.
+inline int moe_kind(int fmt, int cols) {
+  if (fmt == BQG_Q8_0) return kQ8One;
+  if (fmt == BQG_Q4_0) return kQ4One;
+  return cols % 64 == 0 ? kI4x64 : kI4x32;
+}
+
+// Kernel instance for a (routed kind, shared kind) pair.
+using MgKernel = void (*)(MgPhase);
+template <int KR>
+inline MgKernel mg_kernel_ks(int ks) {
+  switch (ks) {
+    case kQ4One: return k_moe_gemv<KR, kQ4One>;
+    case kQ8One: return k_moe_gemv<KR, kQ8One>;
+    case kI4x64: return k_moe_gemv<KR, kI4x64>;
+    default: return k_moe_gemv<KR, kI4x32>;
+  }
+}
+inline MgKernel mg_kernel(int kr, int ks) {
+  switch (kr) {
+    case kQ4One: return mg_kernel_ks<kQ4One>(ks);
+    case kQ8One: return mg_kernel_ks<kQ8One>(ks);
+    case kI4x64: return mg_kernel_ks<kI4x64>(ks);
+    default: return mg_kernel_ks<kI4x32>(ks);
+  }
+}
+
+inline int mg_row_bytes(int fmt, int cols) {
+  return fmt == BQG_Q8_0 ? cols / 32 * 34 : fmt == BQG_Q4_0 ? cols / 32 * 18 : cols / 2;
+}
+
+// One family of stacked matrices [rows x cols] (expert e at base + e * stride).
+inline MgMat mg_mat(int fmt, const void* base, size_t stride, int rows, int cols) {
+  MgMat M{};
+  M.base = static_cast<const uint8_t*>(base);
+  M.stride = (long long)stride;
+  M.rows = rows;
+  M.cols = cols;
+  M.kind = moe_kind(fmt, cols);
+  M.row_bytes = mg_row_bytes(fmt, cols);
+  M.units = cols / unit_weights(M.kind);
+  M.scale_off = fmt == BQG_I4_ROW ? int((size_t(rows) * M.row_bytes + 15) / 16 * 16) : 0;
+  M.stage_rows = gemv_stage_rows(M.units, M.row_bytes);
+  M.nstages = (rows + M.stage_rows - 1) / M.stage_rows;
+  return M;
+}
+
+inline size_t xrec_bytes(int fmt, int rows, int cols) {
+  const int kind = moe_kind(fmt, cols);
+  return size_t(rows) * (cols / unit_weights(kind)) * xrec_chunks(kind) * 16;
+}
+
 struct MoeWsLayout {
-  size_t counts, offsets, active, n_active, perm, h, part, hs, sout, total;
+  size_t counts, offsets, active, n_active, ctr, perm;
+  size_t xq, s_xq, g, u, gs, us, hq, hsq, part, sout, total;
 };
 
 inline MoeWsLayout moe_ws_layout(const bqg_moe_layer* L, int tokens) {
   MoeWsLayout o{};
-  const size_t E = size_t(L->n_experts), pairs = size_t(tokens) * L->top_k;
+  const size_t E = size_t(L->n_experts), T = size_t(tokens), pairs = T * L->top_k;
+  const bool sh = L->s_gate != nullptr;
   size_t off = 0;
-  o.counts = off; off += 4 * E;
-  o.offsets = off; off += 4 * (E + 1);
-  o.active = off; off += 4 * E;
-  o.n_active = off; off += 4;
-  o.perm = off; off += 4 * pairs;
-  off = align256(off);
-  o.h = off; off = align256(off + 4 * pairs * L->inter);
-  o.part = off; off = align256(off + 4 * pairs * L->hidden);
-  if (L->s_gate != nullptr) {
-    o.hs = off; off = align256(off + 4 * size_t(tokens) * L->shared_inter);
-    o.sout = off; off = align256(off + 4 * size_t(tokens) * L->hidden);
-  }
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  o.counts = take(4 * E);
+  o.offsets = take(4 * (E + 1));
+  o.active = take(4 * E);
+  o.n_active = take(4);
+  o.ctr = take(8);
+  o.perm = take(4 * pairs);
+  o.xq = take(xrec_bytes(L->expert_fmt, tokens, L->hidden));
+  o.s_xq = sh ? take(xrec_bytes(L->shared_fmt, tokens, L->hidden)) : 0;
+  o.g = take(4 * pairs * L->inter);
+  o.u = take(4 * pairs * L->inter);
+  o.gs = sh ? take(4 * T * L->shared_inter) : 0;
+  o.us = sh ? take(4 * T * L->shared_inter) : 0;
+  o.hq = take(xrec_bytes(L->expert_fmt, int(pairs), L->inter));
+  o.hsq = sh ? take(xrec_bytes(L->shared_fmt, tokens, L->shared_inter)) : 0;
+  o.part = take(4 * pairs * L->hidden);
+  o.sout = sh ? take(4 * T * L->hidden) : 0;
   o.total = off;
   return o;
 }
@@ -65,43 +130,16 @@ inline int check_layer(const bqg_moe_layer* L) {
   return BQG_OK;
 }
 
-// Matrix family description for the grouped kernel.
-inline int moe_mat(int fmt, const void* base, size_t stride, int rows, int cols, MoeMat* out) {
-  MoeMat M{};
-  GemvProb P{};
-  // reuse the GEMV unit selection (kind, row bytes, units, scale offset)
-  const int st = make_gemv_prob(fmt, base, reinterpret_cast<const float*>(base),
-                                reinterpret_cast<float*>(const_cast<void*>(base)), rows, cols, &P);
-  if (st != BQG_OK) return st;
-  M.base = static_cast<const uint8_t*>(base);
-  M.stride = (long long)stride;
-  M.rows = rows;
-  M.cols = cols;
-  M.kind = P.kind;
-  M.row_bytes = P.row_bytes;
-  M.units = P.units;
-  M.scale_off = P.scale_off;
-  *out = M;
-  return BQG_OK;
-}
+// one attribute cache per kernel instance (4 x 4)
+inline SmemAttrOnce g_moe_attr[16];
+inline int moe_kind_index(int kind) { return kind == kQ4One ? 0 : kind == kQ8One ? 1 : kind == kI4x64 ? 2 : 3; }
 
-// Lanes per row, rows per tile and tokens per token tile for one matrix family.
-inline void moe_plan(const MoeMat& M, int nmat, int& lpr, int& tile_rows, int& tiles, int& tb) {
-  lpr = M.units <= 64 ? 8 : (M.units <= 128 ? 16 : 32);
-  const int rows_per_pass = kMoeThreads / lpr;
-  int tr = kMoeMaxVRows / nmat;
-  if (tr > rows_per_pass) tr = rows_per_pass;
-  while (tr > 1 && nmat * (((tr * M.row_bytes + 47) / 16) * 16) > kMoeSlotBytes) --tr;
-  if (tr > M.rows) tr = M.rows;
-  tile_rows = tr;
-  tiles = (M.rows + tr - 1) / tr;
-  const int uw = unit_weights(M.kind);
-  const int per_tok = M.units * (uw + 4) * 4;
-  tb = kMoeXBytes / per_tok;
-  if (tb > kMoeMaxTok) tb = kMoeMaxTok;
+inline int quant_grid(long long units, int cap) {
+  long long g = (units + 255) / 256;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return int(g);
 }
-
-inline SmemAttrOnce g_moe_attr;
 
 }  // namespace bqg
 
@@ -112,96 +150,130 @@ extern "C" size_t moe_workspace_size(const bqg_moe_layer* L, int tokens) {
 
 extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
                            int tokens, void* workspace, size_t ws_bytes, void* stream) {
-  int st = bqg::check_layer(L);
+  using namespace bqg;
+  int st = check_layer(L);
   if (st != BQG_OK) return st;
   if (x == nullptr || idx == nullptr || w == nullptr || y == nullptr || tokens < 1) return BQG_ERR_ARG;
   if ((long long)tokens * L->top_k > (1 << 24)) return BQG_ERR_LIMIT;
-  if (!bqg::aligned(x, 16) || !bqg::aligned(y, 16) || !bqg::aligned(idx, 4) || !bqg::aligned(w, 4))
-    return BQG_ERR_ALIGN;
-  const bqg::MoeWsLayout lay = bqg::moe_ws_layout(L, tokens);
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(idx, 4) || !aligned(w, 4)) return BQG_ERR_ALIGN;
+  const MoeWsLayout lay = moe_ws_layout(L, tokens);
   if (workspace == nullptr || ws_bytes < lay.total) return BQG_ERR_WORKSPACE;
-  if (!bqg::aligned(workspace, 256)) return BQG_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return BQG_ERR_ALIGN;
   int dev;
-  bqg::DeviceInfo* info;
-  st = bqg::current_device(&dev, &info);
-  if (st != BQG_OK) return st;
-  st = bqg::g_moe_attr.ensure(dev, bqg::k_moe_grouped, bqg::kMoeSmemBytes);
+  DeviceInfo* info;
+  st = current_device(&dev, &info);
   if (st != BQG_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto F = [&](size_t o) { return reinterpret_cast<float*>(ws + o); };
+  auto R = [&](size_t o) { return reinterpret_cast<uint4*>(ws + o); };
+  const bool sh = L->s_gate != nullptr;
+  const int pairs = tokens * L->top_k;
 
-  bqg::RouteWs route;
+  RouteWs route;
   route.counts = reinterpret_cast<int32_t*>(ws + lay.counts);
   route.offsets = reinterpret_cast<int32_t*>(ws + lay.offsets);
   route.active = reinterpret_cast<int32_t*>(ws + lay.active);
   route.n_active = reinterpret_cast<int32_t*>(ws + lay.n_active);
   route.perm = reinterpret_cast<int32_t*>(ws + lay.perm);
-  float* h = reinterpret_cast<float*>(ws + lay.h);
-  float* part = reinterpret_cast<float*>(ws + lay.part);
-  const bool has_shared = L->s_gate != nullptr;
-  float* hs = has_shared ? reinterpret_cast<float*>(ws + lay.hs) : nullptr;
-  float* sout = has_shared ? reinterpret_cast<float*>(ws + lay.sout) : nullptr;
-  const int pairs = tokens * L->top_k;
+  route.ctr = reinterpret_cast<uint32_t*>(ws + lay.ctr);
 
-  // 1. route grouping
-  bqg::k_moe_route<<<1, bqg::kRouteThreads, 0, s>>>(idx, pairs, L->n_experts, route);
-  if ((st = bqg::launch_status()) != BQG_OK) return st;
-
-  // 2. gate/up + activation, 3. down
-  for (int phase = 0; phase < 2; ++phase) {
-    bqg::MoePhase P{};
-    P.route = route;
-    P.tokens = tokens;
-    P.top_k = L->top_k;
-    P.act = L->act;
-    P.gateup = phase == 0;
-    if (phase == 0) {
-      if ((st = bqg::moe_mat(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden, &P.m0)) != BQG_OK) return st;
-      if ((st = bqg::moe_mat(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden, &P.m1)) != BQG_OK) return st;
-      P.nmat = 2;
-      P.xin = x;
-      P.xin_stride = L->hidden;
-      P.out = h;
-      P.out_stride = L->inter;
-    } else {
-      if ((st = bqg::moe_mat(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, &P.m0)) != BQG_OK) return st;
-      P.m1 = P.m0;
-      P.nmat = 1;
-      P.xin = h;
-      P.xin_stride = L->inter;
-      P.out = part;
-      P.out_stride = L->hidden;
-    }
-    bqg::moe_plan(P.m0, P.nmat, P.lpr, P.tile_rows, P.tiles, P.tb);
-    if (P.tb < 1) return BQG_ERR_LIMIT;
-    if (has_shared) {
-      P.s_present = 1;
-      if (phase == 0) {
-        if ((st = bqg::moe_mat(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden, &P.s0)) != BQG_OK) return st;
-        if ((st = bqg::moe_mat(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden, &P.s1)) != BQG_OK) return st;
-        P.s_xin = x;
-        P.s_xin_stride = L->hidden;
-        P.s_out = hs;
-        P.s_out_stride = L->shared_inter;
-      } else {
-        if ((st = bqg::moe_mat(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, &P.s0)) != BQG_OK) return st;
-        P.s1 = P.s0;
-        P.s_xin = hs;
-        P.s_xin_stride = L->shared_inter;
-        P.s_out = sout;
-        P.s_out_stride = L->hidden;
-      }
-      bqg::moe_plan(P.s0, P.nmat, P.s_lpr, P.s_tile_rows, P.s_tiles, P.s_tb);
-      if (P.s_tb < 1) return BQG_ERR_LIMIT;
-    }
-    const int grid = info->sm_count;
-    bqg::k_moe_grouped<<<grid, bqg::kMoeThreads, bqg::kMoeSmemBytes, s>>>(P);
-    if ((st = bqg::launch_status()) != BQG_OK) return st;
+  // routed and shared matrix families
+  const MgMat gate = mg_mat(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden);
+  const MgMat up = mg_mat(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden);
+  const MgMat down = mg_mat(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter);
+  MgMat s_gate{}, s_up{}, s_down{};
+  if (sh) {
+    s_gate = mg_mat(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden);
+    s_up = mg_mat(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden);
+    s_down = mg_mat(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter);
   }
 
-  // 4. combine in slot order, plus the shared output
+  // 1. route grouping + x in integer form
+  QuantJobs qx{};
+  qx.j[0] = QuantJob{x, nullptr, R(lay.xq), tokens, L->hidden, gate.kind, L->act};
+  qx.n = 1;
+  if (sh) qx.j[qx.n++] = QuantJob{x, nullptr, R(lay.s_xq), tokens, L->hidden, s_gate.kind, L->act};
+  const long long xunits = (long long)tokens * (gate.units + (sh ? s_gate.units : 0));
+  const int prep_grid = 1 + int((xunits + kRouteThreads - 1) / kRouteThreads < info->sm_count
+                                    ? (xunits + kRouteThreads - 1) / kRouteThreads
+                                    : info->sm_count);
+  k_moe_prep<<<prep_grid, kRouteThreads, 0, s>>>(idx, pairs, L->n_experts, route, qx);
+  if ((st = launch_status()) != BQG_OK) return st;
+
+  MgPhase P{};
+  P.top_k = L->top_k;
+  P.tokens = tokens;
+  P.counts = route.counts;
+  P.offsets = route.offsets;
+  P.active = route.active;
+  P.n_active = route.n_active;
+  P.perm = route.perm;
+
+  // 2. gate/up of the touched experts (and of the shared expert)
+  P.m[0] = gate;
+  P.m[1] = up;
+  P.nmat = 2;
+  P.xq = R(lay.xq);
+  P.out[0] = F(lay.g);
+  P.out[1] = F(lay.u);
+  P.x_by_token = 1;
+  if (sh) {
+    P.m[2] = s_gate;
+    P.m[3] = s_up;
+    P.s_nmat = 2;
+    P.s_xq = R(lay.s_xq);
+    P.out[2] = F(lay.gs);
+    P.out[3] = F(lay.us);
+  }
+  P.ctr = route.ctr;
+  {
+    const int kr = gate.kind, ks = sh ? s_gate.kind : gate.kind;
+    const MgKernel k = mg_kernel(kr, ks);
+    if ((st = g_moe_attr[moe_kind_index(kr) * 4 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
+      return st;
+    k<<<info->sm_count, kGemvThreads, kMgSmemBytes, s>>>(P);
+    if ((st = launch_status()) != BQG_OK) return st;
+  }
+
+  // 3. h = act(g) * u in integer form
+  QuantJobs qh{};
+  qh.j[0] = QuantJob{F(lay.g), F(lay.u), R(lay.hq), pairs, L->inter, down.kind, L->act};
+  qh.n = 1;
+  if (sh) qh.j[qh.n++] = QuantJob{F(lay.gs), F(lay.us), R(lay.hsq), tokens, L->shared_inter, s_down.kind, L->act};
+  const long long hunits = (long long)pairs * down.units + (sh ? (long long)tokens * s_down.units : 0);
+  k_moe_quant<<<quant_grid(hunits, 4 * info->sm_count), 256, 0, s>>>(qh);
+  if ((st = launch_status()) != BQG_OK) return st;
+
+  // 4. down of the touched experts (and of the shared expert)
+  MgPhase D = P;
+  D.m[0] = down;
+  D.nmat = 1;
+  D.xq = R(lay.hq);
+  D.out[0] = F(lay.part);
+  D.out[1] = nullptr;
+  D.x_by_token = 0;
+  D.s_nmat = 0;
+  if (sh) {
+    D.m[2] = s_down;
+    D.s_nmat = 1;
+    D.s_xq = R(lay.hsq);
+    D.out[2] = F(lay.sout);
+    D.out[3] = nullptr;
+  }
+  D.ctr = route.ctr + 1;
+  {
+    const int kr = down.kind, ks = sh ? s_down.kind : down.kind;
+    const MgKernel k = mg_kernel(kr, ks);
+    if ((st = g_moe_attr[moe_kind_index(kr) * 4 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
+      return st;
+    k<<<info->sm_count, kGemvThreads, kMgSmemBytes, s>>>(D);
+    if ((st = launch_status()) != BQG_OK) return st;
+  }
+
+  // 5. combine
   const long long n = (long long)tokens * L->hidden;
-  bqg::k_moe_combine<<<int((n + 255) / 256), 256, 0, s>>>(part, idx, w, sout, y, tokens, L->top_k, L->hidden,
-                                                            L->n_experts);
-  return bqg::launch_status();
+  k_moe_combine<<<unsigned((n + 255) / 256), 256, 0, s>>>(F(lay.part), idx, w, sh ? F(lay.sout) : nullptr, y, tokens,
+                                                           L->top_k, L->hidden, L->n_experts);
+  return launch_status();
 }

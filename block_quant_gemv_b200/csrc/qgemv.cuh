@@ -154,19 +154,10 @@ __device__ __forceinline__ uint32_t pack_byte(int a, int b, int c, int d, int k)
   return __byte_perm(__byte_perm(uint32_t(a), uint32_t(b), sel), __byte_perm(uint32_t(c), uint32_t(d), sel), 0x5410u);
 }
 
-// Loads one unit's x from xs and converts it (see XUnit).
+// Converts one unit's x values (see XUnit).
 template <int KIND>
-__device__ __forceinline__ void build_x(const float* xs, XUnit& X) {
+__device__ __forceinline__ void quantize_unit(const float (&xv)[unit_weights(KIND)], XUnit& X) {
   constexpr int UW = unit_weights(KIND);
-  float xv[UW];
-#pragma unroll
-  for (int i = 0; i < UW / 4; ++i) {
-    const float4 v = reinterpret_cast<const float4*>(xs)[i];
-    xv[4 * i] = v.x;
-    xv[4 * i + 1] = v.y;
-    xv[4 * i + 2] = v.z;
-    xv[4 * i + 3] = v.w;
-  }
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < UW; ++i) amax = fmaxf(amax, fabsf(xv[i]));
@@ -198,6 +189,22 @@ __device__ __forceinline__ void build_x(const float* xs, XUnit& X) {
     X.c0 = -8 * s0;
     X.c1 = -8 * s1;
   }
+}
+
+// Loads one unit's x from xs (shared or global memory, 16-byte aligned) and converts it.
+template <int KIND>
+__device__ __forceinline__ void build_x(const float* xs, XUnit& X) {
+  constexpr int UW = unit_weights(KIND);
+  float xv[UW];
+#pragma unroll
+  for (int i = 0; i < UW / 4; ++i) {
+    const float4 v = reinterpret_cast<const float4*>(xs)[i];
+    xv[4 * i] = v.x;
+    xv[4 * i + 1] = v.y;
+    xv[4 * i + 2] = v.z;
+    xv[4 * i + 3] = v.w;
+  }
+  quantize_unit<KIND>(xv, X);
 }
 
 // sum over the 8 elements of one nibble word of u * X (u the unsigned nibble), into (h, l).
