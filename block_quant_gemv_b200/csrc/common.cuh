@@ -19,6 +19,12 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void flag_error(int bits) { atomicOr(&g_dev_errors, bits); }
 
+// Dependent launches: wait until the previous kernel on the stream has completed and its writes
+// are visible (a no-op when the kernel was launched without programmatic serialization), and
+// allow the next kernel to be scheduled early (it still waits for this one before its reads).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

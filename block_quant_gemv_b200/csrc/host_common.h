@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "bqg.h"
 
@@ -46,6 +47,30 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 inline int launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? BQG_OK : BQG_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialization (dependent launch): the kernel may be
+// scheduled before the previous kernel on the stream has finished, and waits for it with
+// griddep_wait() before reading anything that kernel wrote.  Launch processing and the
+// kernel's prologue then overlap the previous kernel's tail.
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BQG_ERR_CUDA;
+  }
+  return launch_status();
 }
 
 // Per-device "dynamic shared memory attribute already set" flags for one kernel.

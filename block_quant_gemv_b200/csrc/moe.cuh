@@ -91,55 +91,100 @@ struct QuantJobs {
   int n;
 };
 
+// One 8-value segment of a unit: the UW/8 segments of a unit sit on consecutive lanes of one
+// warp, which share max|x| and the block sums by shuffles.  Every lane of the warp must call
+// this (valid = false for lanes past the end).
 template <int KIND>
-__device__ __forceinline__ void quant_one(const QuantJob& J, int row, int u) {
-  constexpr int UW = unit_weights(KIND);
-  const size_t off = size_t(row) * J.cols + size_t(u) * UW;
-  float xv[UW];
+__device__ __forceinline__ void quant_seg(const QuantJob& J, long long gs, bool valid) {
+  constexpr int UW = unit_weights(KIND), G = UW / 8, NW = UW / 4;
+  const int lane = threadIdx.x & 31;
+  const int units = J.cols / UW;
+  const long long unit = gs / G;
+  const int m = int(gs - unit * G);
+  float xv[8];
 #pragma unroll
-  for (int i = 0; i < UW / 4; ++i) {
-    const float4 v = *reinterpret_cast<const float4*>(J.a + off + 4 * i);
-    xv[4 * i] = v.x;
-    xv[4 * i + 1] = v.y;
-    xv[4 * i + 2] = v.z;
-    xv[4 * i + 3] = v.w;
-  }
-  if (J.b != nullptr) {
+  for (int i = 0; i < 8; ++i) xv[i] = 0.f;
+  if (valid) {
+    const int row = int(unit / units), u = int(unit - (long long)row * units);
+    const size_t off = size_t(row) * J.cols + size_t(u) * UW + 8 * m;
+    const float4 v0 = *reinterpret_cast<const float4*>(J.a + off);
+    const float4 v1 = *reinterpret_cast<const float4*>(J.a + off + 4);
+    xv[0] = v0.x; xv[1] = v0.y; xv[2] = v0.z; xv[3] = v0.w;
+    xv[4] = v1.x; xv[5] = v1.y; xv[6] = v1.z; xv[7] = v1.w;
+    if (J.b != nullptr) {
+      const float4 b0 = *reinterpret_cast<const float4*>(J.b + off);
+      const float4 b1 = *reinterpret_cast<const float4*>(J.b + off + 4);
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int i = 0; i < UW / 4; ++i) {
-      const float4 v = *reinterpret_cast<const float4*>(J.b + off + 4 * i);
-      xv[4 * i] = act_fn(J.act, xv[4 * i]) * v.x;
-      xv[4 * i + 1] = act_fn(J.act, xv[4 * i + 1]) * v.y;
-      xv[4 * i + 2] = act_fn(J.act, xv[4 * i + 2]) * v.z;
-      xv[4 * i + 3] = act_fn(J.act, xv[4 * i + 3]) * v.w;
+      for (int i = 0; i < 8; ++i) xv[i] = act_fn(J.act, xv[i]) * bv[i];
     }
   }
-  XUnit X;
-  quantize_unit<KIND>(xv, X);
-  store_xunit<KIND>(X, J.dst + (size_t(row) * (J.cols / UW) + u) * xrec_chunks(KIND));
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(xv[i]));
+#pragma unroll
+  for (int o = 1; o < G; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+  int xi[8];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    xi[i] = __float2int_rn(xv[i] * inv);
+    sum += xi[i];
+  }
+  uint32_t h0, h1, l0, l1;
+  if constexpr (is_q8(KIND)) {  // words 2m, 2m+1 = elements 8m..8m+3, 8m+4..8m+7
+    h0 = pack_byte(xi[0], xi[1], xi[2], xi[3], 1);
+    h1 = pack_byte(xi[4], xi[5], xi[6], xi[7], 1);
+    l0 = pack_byte(xi[0], xi[1], xi[2], xi[3], 0);
+    l1 = pack_byte(xi[4], xi[5], xi[6], xi[7], 0);
+  } else {  // words 2m, 2m+1 = even, odd elements of 8m..8m+7
+    h0 = pack_byte(xi[0], xi[2], xi[4], xi[6], 1);
+    h1 = pack_byte(xi[1], xi[3], xi[5], xi[7], 1);
+    l0 = pack_byte(xi[0], xi[2], xi[4], xi[6], 0);
+    l1 = pack_byte(xi[1], xi[3], xi[5], xi[7], 0);
+  }
+  // block sums: 4 segments of 32 values per block
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  const int sum_b1 = __shfl_sync(0xffffffffu, sum, (lane & ~(G - 1)) + (G == 8 ? 4 : 0));
+  if (valid) {
+    uint32_t* rec = reinterpret_cast<uint32_t*>(J.dst + unit * xrec_chunks(KIND));
+    *reinterpret_cast<uint2*>(rec + 2 * m) = make_uint2(h0, h1);
+    *reinterpret_cast<uint2*>(rec + NW + 2 * m) = make_uint2(l0, l1);
+    if (m == 0) {
+      const int c0 = is_q8(KIND) ? 0 : -8 * sum;
+      const int c1 = (is_q8(KIND) || G == 4) ? 0 : -8 * sum_b1;
+      *reinterpret_cast<uint4*>(rec + 2 * NW) = make_uint4(uint32_t(c0), uint32_t(c1), __float_as_uint(amax * (1.f / 32767.f)), 0u);
+    }
+  }
 }
 
-// Converts every unit of the jobs; thread i of nthreads takes units i, i + nthreads, ...
+// Converts every unit of the jobs: thread i of nthreads (a multiple of 32, warps aligned)
+// takes segments i, i + nthreads, ...
 __device__ __forceinline__ void quant_jobs(const QuantJobs& Q, long long i0, long long nthreads) {
   for (int jn = 0; jn < Q.n; ++jn) {
     const QuantJob& J = Q.j[jn];
-    const int units = J.cols / unit_weights(J.kind);
-    const long long total = (long long)J.rows * units;
-    for (long long i = i0; i < total; i += nthreads) {
-      const int row = int(i / units), u = int(i - (long long)row * units);
+    const int G = unit_weights(J.kind) / 8;
+    const long long total = (long long)J.rows * (J.cols / unit_weights(J.kind)) * G;
+    const long long padded = (total + 31) / 32 * 32;
+    for (long long i = i0; i < padded; i += nthreads) {
+      const bool valid = i < total;
       switch (J.kind) {
-        case kQ4Pair: quant_one<kQ4Pair>(J, row, u); break;
-        case kQ4One: quant_one<kQ4One>(J, row, u); break;
-        case kQ8Pair: quant_one<kQ8Pair>(J, row, u); break;
-        case kQ8One: quant_one<kQ8One>(J, row, u); break;
-        case kI4x64: quant_one<kI4x64>(J, row, u); break;
-        default: quant_one<kI4x32>(J, row, u); break;
+        case kQ4Pair: quant_seg<kQ4Pair>(J, i, valid); break;
+        case kQ4One: quant_seg<kQ4One>(J, i, valid); break;
+        case kQ8Pair: quant_seg<kQ8Pair>(J, i, valid); break;
+        case kQ8One: quant_seg<kQ8One>(J, i, valid); break;
+        case kI4x64: quant_seg<kI4x64>(J, i, valid); break;
+        default: quant_seg<kI4x32>(J, i, valid); break;
       }
     }
   }
 }
 
 __global__ void __launch_bounds__(256) k_moe_quant(const __grid_constant__ QuantJobs Q) {
+  griddep_launch_dependents();
+  griddep_wait();
   quant_jobs(Q, (long long)blockIdx.x * blockDim.x + threadIdx.x, (long long)gridDim.x * blockDim.x);
 }
 
@@ -172,17 +217,43 @@ __device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int p
   }
   if (bad) flag_error(BQG_DEVERR_EXPERT_ID);
   __syncthreads();
-  if (tid == 0) {
-    int off = 0, na = 0;
-    for (int e = 0; e < n_experts; ++e) {
-      ws.counts[e] = cnt[e];
-      ws.offsets[e] = off;
-      base[e] = off;
-      if (cnt[e] > 0) ws.active[na++] = e;
-      off += cnt[e];
+  if (warp == 0) {
+    // exclusive scan of the counts and the list of touched experts: lane l owns experts
+    // 8l .. 8l+7 (n_experts <= 256)
+    int c[8], tot = 0, nact = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = 8 * lane + i;
+      c[i] = e < n_experts ? cnt[e] : 0;
+      tot += c[i];
+      nact += c[i] > 0 ? 1 : 0;
     }
-    ws.offsets[n_experts] = off;
-    ws.n_active[0] = na;
+    int incl = tot, ainc = nact;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      const int a = __shfl_up_sync(0xffffffffu, ainc, o);
+      if (lane >= o) {
+        incl += v;
+        ainc += a;
+      }
+    }
+    int off = incl - tot, na = ainc - nact;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = 8 * lane + i;
+      if (e < n_experts) {
+        ws.counts[e] = c[i];
+        ws.offsets[e] = off;
+        base[e] = off;
+        if (c[i] > 0) ws.active[na++] = e;
+      }
+      off += c[i];
+    }
+    if (lane == 31) {
+      ws.offsets[n_experts] = incl;
+      ws.n_active[0] = ainc;
+    }
   }
   __syncthreads();
   // stable placement, one chunk of kRouteThreads pairs at a time
@@ -220,6 +291,8 @@ __device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int p
 __global__ void __launch_bounds__(kRouteThreads, 1) k_moe_prep(const int32_t* __restrict__ idx, int pairs,
                                                             int n_experts, RouteWs ws,
                                                             const __grid_constant__ QuantJobs Q) {
+  griddep_launch_dependents();
+  griddep_wait();
   if (blockIdx.x == 0) {
     moe_route(idx, pairs, n_experts, ws);
   } else {
@@ -264,16 +337,23 @@ __device__ __forceinline__ int4 ld_desc(const int4* d) {
   return v;
 }
 
-constexpr size_t kMgSmemBytes = size_t(kGemvStages) * kGemvStageAlloc +
+constexpr int kMgStages = 3;  // no x staging buffer here: room for a third 72 KB stage
+constexpr size_t kMgSmemBytes = size_t(kMgStages) * kGemvStageAlloc +
                                 size_t(2 * kGemvConsumerWarps * kGemvRedRows) * sizeof(float) +
-                                (2 * kGemvStages) * sizeof(uint64_t) + size_t(kGemvStages) * sizeof(int4);
+                                (3 * kMgStages) * sizeof(uint64_t) + size_t(kMgStages) * sizeof(int4);
+static_assert(kMgSmemBytes <= 227 * 1024, "grouped GEMV shared memory");
+static_assert((size_t(kMgStages) * kGemvStageAlloc + size_t(2 * kGemvConsumerWarps * kGemvRedRows) * 4) % 16 == 0,
+              "descriptors must be 16-byte aligned");
 
 // Consumer side of one item (stage `slot` holds rows [r0, r1) of family fam, expert e).
 // q counts token iterations (selects the group reduction buffer).
+// The weight stage may still be in flight on entry: the first token's x is loaded before
+// waiting for it (full, parity).  Returns false if that wait gave up.
+// With `reuse` (same matrix as the previous item) and a single token, X already holds it.
 template <int KIND>
-__device__ __forceinline__ void mg_item(const MgPhase& P, int fam, int e, int r0, int r1, uint32_t stage_s,
-                                        float* red, int& q) {
-  const MgMat& M = P.m[fam];
+__device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int fam, int e, int r0, int r1,
+                                        uint32_t stage_s, float* red, int& q, uint64_t* full, uint32_t parity, XUnit& X,
+                                        bool reuse) {
   const bool shared = fam >= 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = M.units, row_bytes = M.row_bytes;
@@ -296,8 +376,8 @@ __device__ __forceinline__ void mg_item(const MgPhase& P, int fam, int e, int r0
   for (int tt = 0; tt < ntok; ++tt, ++q) {
     const int pid = shared ? tt : __ldg(list + tt);
     const int xrow = (shared || !P.x_by_token) ? pid : pid / P.top_k;
-    XUnit X;
-    if (active) load_xunit<KIND>(xq + (size_t(xrow) * units + p) * xrec_chunks(KIND), X);
+    if (active && !(reuse && ntok == 1)) load_xunit<KIND>(xq + (size_t(xrow) * units + p) * xrec_chunks(KIND), X);
+    if (tt == 0 && !mbar_wait(full, parity)) return false;
     float* orow = out + size_t(pid) * M.rows + r0;
     const int par = q & 1;
     int nmine = 0;
@@ -348,6 +428,8 @@ __device__ __forceinline__ void mg_item(const MgPhase& P, int fam, int e, int r0
       }
     }
   }
+  if (ntok == 0) return mbar_wait(full, parity);
+  return true;
 }
 
 // KR: unit kind of the routed families, KS: of the shared ones (one kernel per pair keeps each
@@ -356,56 +438,84 @@ template <int KR, int KS>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_constant__ MgPhase P) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
-  float* red = reinterpret_cast<float*>(smem + size_t(kGemvStages) * kGemvStageAlloc);
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kGemvConsumerWarps * kGemvRedRows);
-  uint64_t* empty = full + kGemvStages;
-  int4* desc = reinterpret_cast<int4*>(empty + kGemvStages);  // (family, expert, r0, r1)
+  float* red = reinterpret_cast<float*>(smem + size_t(kMgStages) * kGemvStageAlloc);
+  int4* desc = reinterpret_cast<int4*>(red + 2 * kGemvConsumerWarps * kGemvRedRows);  // (family, expert, r0, r1)
+  __shared__ MgMat fams[4];  // the phase's matrix families, indexed per item from shared memory
+  uint64_t* full = reinterpret_cast<uint64_t*>(desc + kMgStages);
+  uint64_t* empty = full + kMgStages;
+  uint64_t* dready = empty + kMgStages;  // the slot's descriptor is written (stage may be in flight)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kGemvStages; ++i) {
+    for (int i = 0; i < kMgStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kGemvConsumerWarps);
+      mbar_init(&dready[i], 1);
     }
+    for (int i = 0; i < 4; ++i) fams[i] = P.m[i];
     fence_barrier_init();
   }
   __syncthreads();
+  griddep_launch_dependents();
+  griddep_wait();  // route lists, counters and input records come from earlier kernels
 
   if (warp == kGemvConsumerWarps) {
     // ------------------------------------------------ producer (one elected lane)
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
     const int na = *P.n_active;
-    const int n_sh = P.s_nmat * P.m[2].nstages;
-    const int per_expert = P.nmat * P.m[0].nstages;
+    const int n_sh = P.s_nmat * fams[2].nstages;
+    const int per_expert = P.nmat * fams[0].nstages;
     const int n_items = n_sh + na * per_expert;
     int s = 0;
     bool ok = true;
-    int item = int(atomicAdd(P.ctr, 1u));
-    while (item < n_items) {
-      const int next = int(atomicAdd(P.ctr, 1u));  // claimed one item ahead
+    // With one token every item costs about the same: items are claimed in runs (guided:
+    // about 1/(2 * grid) of what is left, at least one), so a CTA mostly stays on one matrix
+    // and keeps its x in registers.  With several tokens item costs differ (an expert's token
+    // count, the shared expert's all tokens): one item per claim balances them.
+    const int grid = int(gridDim.x);
+    int est = 0;  // this CTA's estimate of the counter (end of its last claim)
+    auto claim = [&](int& first) -> int {
+      int want = (n_items - est) / (2 * grid);
+      if (want < 1 || P.tokens > 1) want = 1;
+      first = int(atomicAdd(P.ctr, unsigned(want)));
+      est = first + want;
+      return first >= n_items ? 0 : min(want, n_items - first);
+    };
+    int first = 0, nfirst = 0;
+    int cnt = claim(first);
+    int ncnt = cnt > 0 ? claim(nfirst) : 0;  // the next run, claimed one run ahead
+    for (int item = first;; ++item) {
+      if (item >= first + cnt) {
+        first = nfirst;
+        cnt = ncnt;
+        if (cnt <= 0) break;
+        ncnt = claim(nfirst);
+        item = first;
+      }
       int fam, e = 0, k;
       if (item < n_sh) {
-        fam = 2 + item / P.m[2].nstages;
-        k = item - (fam - 2) * P.m[2].nstages;
+        fam = 2 + item / fams[2].nstages;
+        k = item - (fam - 2) * fams[2].nstages;
       } else {
         int r = item - n_sh;
         const int a = r / per_expert;
         r -= a * per_expert;
-        fam = r / P.m[0].nstages;
-        k = r - fam * P.m[0].nstages;
+        fam = r / fams[0].nstages;
+        k = r - fam * fams[0].nstages;
         e = __ldg(P.active + a);
       }
-      const MgMat& M = P.m[fam];
+      const MgMat& M = fams[fam];
       const int r0 = k * M.stage_rows;
       const int r1 = min(r0 + M.stage_rows, M.rows);
-      const int slot = s % kGemvStages;
-      if (s >= kGemvStages && !mbar_wait(&empty[slot], uint32_t(s / kGemvStages - 1) & 1u)) {
+      const int slot = s % kMgStages;
+      if (s >= kMgStages && !mbar_wait(&empty[slot], uint32_t(s / kMgStages - 1) & 1u)) {
         ok = false;
         break;
       }
       fence_proxy_async_smem();
       desc[slot] = make_int4(fam, e, r0, r1);
+      mbar_arrive(&dready[slot]);
       const uintptr_t wbeg = reinterpret_cast<uintptr_t>(M.base) + (fam >= 2 ? 0 : size_t(e) * M.stride);
       const uintptr_t wend = wbeg + size_t(M.rows) * M.row_bytes;
       const uintptr_t src = wbeg + size_t(r0) * M.row_bytes;
@@ -425,18 +535,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
         mbar_arrive(&full[slot]);
       }
       ++s;
-      item = next;
     }
     {  // end marker
-      const int slot = s % kGemvStages;
-      if (ok && (s < kGemvStages || mbar_wait(&empty[slot], uint32_t(s / kGemvStages - 1) & 1u))) {
+      const int slot = s % kMgStages;
+      if (ok && (s < kMgStages || mbar_wait(&empty[slot], uint32_t(s / kMgStages - 1) & 1u))) {
         desc[slot] = make_int4(-1, 0, 0, 0);
-        mbar_arrive(&full[slot]);
+        mbar_arrive(&dready[slot]);
       }
     }
     if (!ok) {
-      for (int qq = (s > kGemvStages ? s - kGemvStages : 0); qq < s; ++qq)
-        mbar_wait(&full[qq % kGemvStages], uint32_t(qq / kGemvStages) & 1u);
+      for (int qq = (s > kMgStages ? s - kMgStages : 0); qq < s; ++qq)
+        mbar_wait(&full[qq % kMgStages], uint32_t(qq / kMgStages) & 1u);
     }
     return;
   }
@@ -444,17 +553,25 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
   // ------------------------------------------------ consumers
   const uint32_t ring_s = smem_u32(ring);
   int q = 0;
+  int prev_fam = -1, prev_e = -1;
+  XUnit X;
   for (int s = 0;; ++s) {
-    const int slot = s % kGemvStages;
-    if (!mbar_wait(&full[slot], uint32_t(s / kGemvStages) & 1u)) return;
+    const int slot = s % kMgStages;
+    const uint32_t par = uint32_t(s / kMgStages) & 1u;
+    if (!mbar_wait(&dready[slot], par)) return;
     const int4 d = ld_desc(&desc[slot]);
     if (d.x < 0) return;
-    // row groups may change from one item to the next: every consumer warp has finished the
-    // previous item (including its group reductions)
-    named_bar_sync(1, kGemvCompute);
+    // Another matrix: row groups may change, so every consumer warp must have finished the
+    // previous item (including its group reductions).  The same matrix (next stage of a run):
+    // same groups, and with one token its x is still in registers.
+    const bool same = d.x == prev_fam && d.y == prev_e;
+    if (!same) named_bar_sync(1, kGemvCompute);
+    prev_fam = d.x;
+    prev_e = d.y;
     const uint32_t stage_s = ring_s + uint32_t(slot) * kGemvStageAlloc;
-    if (d.x < 2) mg_item<KR>(P, d.x, d.y, d.z, d.w, stage_s, red, q);
-    else mg_item<KS>(P, d.x, d.y, d.z, d.w, stage_s, red, q);
+    const bool ok = d.x < 2 ? mg_item<KR>(P, fams[d.x], d.x, d.y, d.z, d.w, stage_s, red, q, &full[slot], par, X, same)
+                            : mg_item<KS>(P, fams[d.x], d.x, d.y, d.z, d.w, stage_s, red, q, &full[slot], par, X, same);
+    if (!ok) return;
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
   }
@@ -466,16 +583,30 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
 __global__ void k_moe_combine(const float* __restrict__ part, const int32_t* __restrict__ idx,
                               const float* __restrict__ w, const float* __restrict__ sout, float* __restrict__ y,
                               int tokens, int top_k, int hidden, int n_experts) {
+  griddep_wait();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)tokens * hidden) return;
   const int t = int(i / hidden), c = int(i - (long long)t * hidden);
-  float acc = 0.f;
-  for (int j = 0; j < top_k; ++j) {
-    const int e = idx[t * top_k + j];
-    if (e >= 0 && e < n_experts) acc = fmaf(w[t * top_k + j], part[(size_t(t) * top_k + j) * hidden + c], acc);
+  // all loads first (top_k <= BQG_MAX_TOPK), then the slot-order sum
+  float wv[BQG_MAX_TOPK], pv[BQG_MAX_TOPK];
+#pragma unroll
+  for (int j = 0; j < BQG_MAX_TOPK; ++j) {
+    wv[j] = 0.f;
+    pv[j] = 0.f;
+    if (j < top_k) {
+      const int e = __ldg(idx + t * top_k + j);
+      if (e >= 0 && e < n_experts) {
+        wv[j] = __ldg(w + t * top_k + j);
+        pv[j] = part[(size_t(t) * top_k + j) * hidden + c];
+      }
+    }
   }
-  if (sout != nullptr) acc += sout[size_t(t) * hidden + c];
-  y[i] = acc;
+  const float s = sout != nullptr ? sout[size_t(t) * hidden + c] : 0.f;
+  float acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < BQG_MAX_TOPK; ++j)
+    if (j < top_k) acc = fmaf(wv[j], pv[j], acc);
+  y[i] = acc + s;
 }
 
 }  // namespace bqg

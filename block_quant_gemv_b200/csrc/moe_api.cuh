@@ -134,8 +134,8 @@ inline int check_layer(const bqg_moe_layer* L) {
 inline SmemAttrOnce g_moe_attr[16];
 inline int moe_kind_index(int kind) { return kind == kQ4One ? 0 : kind == kQ8One ? 1 : kind == kI4x64 ? 2 : 3; }
 
-inline int quant_grid(long long units, int cap) {
-  long long g = (units + 255) / 256;
+inline int quant_grid(long long threads, int cap) {
+  long long g = (threads + 255) / 256;
   if (g < 1) g = 1;
   if (g > cap) g = cap;
   return int(g);
@@ -194,12 +194,14 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   qx.j[0] = QuantJob{x, nullptr, R(lay.xq), tokens, L->hidden, gate.kind, L->act};
   qx.n = 1;
   if (sh) qx.j[qx.n++] = QuantJob{x, nullptr, R(lay.s_xq), tokens, L->hidden, s_gate.kind, L->act};
-  const long long xunits = (long long)tokens * (gate.units + (sh ? s_gate.units : 0));
-  const int prep_grid = 1 + int((xunits + kRouteThreads - 1) / kRouteThreads < info->sm_count
-                                    ? (xunits + kRouteThreads - 1) / kRouteThreads
+  // one thread per 8 values
+  const long long xsegs = (long long)tokens * L->hidden / 8 * (sh ? 2 : 1);
+  const int prep_grid = 1 + int((xsegs + kRouteThreads - 1) / kRouteThreads < info->sm_count
+                                    ? (xsegs + kRouteThreads - 1) / kRouteThreads
                                     : info->sm_count);
-  k_moe_prep<<<prep_grid, kRouteThreads, 0, s>>>(idx, pairs, L->n_experts, route, qx);
-  if ((st = launch_status()) != BQG_OK) return st;
+  if ((st = launch_pdl(k_moe_prep, dim3(prep_grid), dim3(kRouteThreads), 0, s, idx, pairs, L->n_experts, route, qx)) !=
+      BQG_OK)
+    return st;
 
   MgPhase P{};
   P.top_k = L->top_k;
@@ -232,8 +234,7 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
     const MgKernel k = mg_kernel(kr, ks);
     if ((st = g_moe_attr[moe_kind_index(kr) * 4 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
       return st;
-    k<<<info->sm_count, kGemvThreads, kMgSmemBytes, s>>>(P);
-    if ((st = launch_status()) != BQG_OK) return st;
+    if ((st = launch_pdl(k, dim3(info->sm_count), dim3(kGemvThreads), kMgSmemBytes, s, P)) != BQG_OK) return st;
   }
 
   // 3. h = act(g) * u in integer form
@@ -241,9 +242,9 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   qh.j[0] = QuantJob{F(lay.g), F(lay.u), R(lay.hq), pairs, L->inter, down.kind, L->act};
   qh.n = 1;
   if (sh) qh.j[qh.n++] = QuantJob{F(lay.gs), F(lay.us), R(lay.hsq), tokens, L->shared_inter, s_down.kind, L->act};
-  const long long hunits = (long long)pairs * down.units + (sh ? (long long)tokens * s_down.units : 0);
-  k_moe_quant<<<quant_grid(hunits, 4 * info->sm_count), 256, 0, s>>>(qh);
-  if ((st = launch_status()) != BQG_OK) return st;
+  const long long hsegs = ((long long)pairs * L->inter + (sh ? (long long)tokens * L->shared_inter : 0)) / 8;
+  if ((st = launch_pdl(k_moe_quant, dim3(quant_grid(hsegs, 4 * info->sm_count)), dim3(256), 0, s, qh)) != BQG_OK)
+    return st;
 
   // 4. down of the touched experts (and of the shared expert)
   MgPhase D = P;
@@ -267,13 +268,11 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
     const MgKernel k = mg_kernel(kr, ks);
     if ((st = g_moe_attr[moe_kind_index(kr) * 4 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
       return st;
-    k<<<info->sm_count, kGemvThreads, kMgSmemBytes, s>>>(D);
-    if ((st = launch_status()) != BQG_OK) return st;
+    if ((st = launch_pdl(k, dim3(info->sm_count), dim3(kGemvThreads), kMgSmemBytes, s, D)) != BQG_OK) return st;
   }
 
   // 5. combine
   const long long n = (long long)tokens * L->hidden;
-  k_moe_combine<<<unsigned((n + 255) / 256), 256, 0, s>>>(F(lay.part), idx, w, sh ? F(lay.sout) : nullptr, y, tokens,
-                                                           L->top_k, L->hidden, L->n_experts);
-  return launch_status();
+  return launch_pdl(k_moe_combine, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s, F(lay.part), idx, w,
+                    sh ? F(lay.sout) : nullptr, y, tokens, L->top_k, L->hidden, L->n_experts);
 }

@@ -13,29 +13,31 @@
 namespace bqg {
 
 // ---------------------------------------------------------------- router logits
-// One warp per expert row e; the CTA's 4 warps cover 4 experts and a tile of up to 8
-// tokens.  Each warp streams R[e, :] once with 16-byte loads and keeps one accumulator per
-// token; x rows are shared by the CTA's warps through L1.  Lanes are reduced with a fixed
-// butterfly, so results are deterministic.
-constexpr int kRouterWarps = 4;
+// One CTA per (expert row e, tile of up to TT tokens), 256 threads striding over the row in
+// 16-byte loads (unrolled so that several loads are in flight per thread).  Each thread keeps
+// one accumulator per token; lanes are reduced with a fixed butterfly and the 8 warps in a
+// fixed order through shared memory, so results are deterministic.
+constexpr int kRouterThreads = 256;
 constexpr int kRouterTok = 8;
 
 template <int TT>
-__global__ void __launch_bounds__(kRouterWarps * 32) k_router_logits(const float* __restrict__ R,
-                                                                     const float* __restrict__ x,
-                                                                     float* __restrict__ logits, int tokens,
-                                                                     int n_experts, int hidden) {
+__global__ void __launch_bounds__(kRouterThreads) k_router_logits(const float* __restrict__ R,
+                                                                  const float* __restrict__ x,
+                                                                  float* __restrict__ logits, int tokens,
+                                                                  int n_experts, int hidden) {
+  __shared__ float part[kRouterThreads / 32][TT];
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * kRouterWarps + warp;
+  const int e = blockIdx.x;
   const int t0 = blockIdx.y * TT;
-  if (e >= n_experts) return;
   const int nt = min(TT, tokens - t0);
   float acc[TT];
 #pragma unroll
   for (int t = 0; t < TT; ++t) acc[t] = 0.f;
   const float4* r4 = reinterpret_cast<const float4*>(R + size_t(e) * hidden);
   const int h4 = hidden / 4;
-  for (int k = lane; k < h4; k += 32) {
+#pragma unroll 4
+  for (int k = threadIdx.x; k < h4; k += kRouterThreads) {
     const float4 r = __ldg(r4 + k);
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
@@ -51,7 +53,14 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_logits(const float
 #pragma unroll
   for (int t = 0; t < TT; ++t) {
     const float s = warp_sum(acc[t]);
-    if (lane == 0 && t < nt) logits[size_t(t0 + t) * n_experts + e] = s;
+    if (lane == 0) part[warp][t] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x < nt) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRouterThreads / 32; ++w) s += part[w][threadIdx.x];
+    logits[size_t(t0 + threadIdx.x) * n_experts + e] = s;
   }
 }
 
@@ -70,6 +79,8 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 __global__ void __launch_bounds__(kTopkWarps * 32) k_router_topk(const float* __restrict__ logits, int tokens,
                                                                  int n_experts, int k, int32_t* __restrict__ idx,
                                                                  float* __restrict__ weights) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + warp;
   if (t >= tokens) return;
@@ -159,18 +170,19 @@ extern "C" int moe_router_logits(const float* R, const float* x, float* logits, 
   const int st = bqg::current_device(&dev, &info);
   if (st != BQG_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int gx = (n_experts + bqg::kRouterWarps - 1) / bqg::kRouterWarps;
+  const int gx = n_experts;
+  const int threads = bqg::kRouterThreads;
   if (tokens == 1) {
-    bqg::k_router_logits<1><<<dim3(gx, 1), bqg::kRouterWarps * 32, 0, s>>>(R, x, logits, tokens, n_experts, hidden);
+    return bqg::launch_pdl(bqg::k_router_logits<1>, dim3(gx, 1), dim3(threads), 0, s, R, x, logits, tokens, n_experts, hidden);
   } else if (tokens <= 2) {
-    bqg::k_router_logits<2><<<dim3(gx, 1), bqg::kRouterWarps * 32, 0, s>>>(R, x, logits, tokens, n_experts, hidden);
+    return bqg::launch_pdl(bqg::k_router_logits<2>, dim3(gx, 1), dim3(threads), 0, s, R, x, logits, tokens, n_experts, hidden);
   } else if (tokens <= 4) {
-    bqg::k_router_logits<4><<<dim3(gx, 1), bqg::kRouterWarps * 32, 0, s>>>(R, x, logits, tokens, n_experts, hidden);
+    return bqg::launch_pdl(bqg::k_router_logits<4>, dim3(gx, 1), dim3(threads), 0, s, R, x, logits, tokens, n_experts, hidden);
   } else {
     const int gy = (tokens + bqg::kRouterTok - 1) / bqg::kRouterTok;
     if (gy > 65535) return BQG_ERR_LIMIT;
-    bqg::k_router_logits<bqg::kRouterTok>
-        <<<dim3(gx, gy), bqg::kRouterWarps * 32, 0, s>>>(R, x, logits, tokens, n_experts, hidden);
+    return bqg::launch_pdl(bqg::k_router_logits<bqg::kRouterTok>, dim3(gx, gy), dim3(threads), 0, s, R, x, logits, tokens,
+                           n_experts, hidden);
   }
   return bqg::launch_status();
 }
@@ -187,7 +199,6 @@ extern "C" int moe_router_topk(const float* logits, int tokens, int n_experts, i
   const int st = bqg::current_device(&dev, &info);
   if (st != BQG_OK) return st;
   const int grid = (tokens + bqg::kTopkWarps - 1) / bqg::kTopkWarps;
-  bqg::k_router_topk<<<grid, bqg::kTopkWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(logits, tokens, n_experts,
-                                                                                          k, idx, weights);
-  return bqg::launch_status();
+  return bqg::launch_pdl(bqg::k_router_topk, dim3(grid), dim3(bqg::kTopkWarps * 32), 0,
+                         static_cast<cudaStream_t>(stream), logits, tokens, n_experts, k, idx, weights);
 }
