@@ -125,6 +125,15 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first(self, timeout: float = 15.0):
+        """Blocks until nvidia-smi has printed its first sample: its start-up (driver
+        initialisation) can stall this process's CUDA calls, so it must not overlap the timed
+        region."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.05)
+        self.lines.clear()
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
@@ -277,6 +286,9 @@ def time_decode_step(args, world, dev):
     W = wl.build_gemv_workload(specs, seed=args.seed, device=dev)
     batch = bqg.GemvBatch(W.items())
     stream = torch.cuda.current_stream()
+    clocks = ClockSampler(physical_gpu(torch.cuda.current_device()))
+    clocks.start()
+    clocks.wait_first()
     for _ in range(max(3, args.warmup)):
         batch.run()
     torch.cuda.synchronize()
@@ -285,11 +297,8 @@ def time_decode_step(args, world, dev):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(physical_gpu(torch.cuda.current_device()))
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.2)
     torch.cuda.nvtx.range_push("timed")  # lets a profiler select exactly the timed launches
     t_begin.record(stream)
     for i in range(args.steps):

@@ -198,6 +198,7 @@ struct RouteWs {
   int32_t* n_active;  // [1]
   int32_t* perm;      // [T * k] pair ids (t * k + j) grouped by expert, token order inside
   uint32_t* ctr;      // [2] work item counters of the two grouped GEMV launches
+  int4* act_info;     // [E] per touched expert (in active order): (expert, count, offset, first pair)
 };
 
 __device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int pairs, int n_experts,
@@ -285,6 +286,13 @@ __device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int p
     }
     __syncthreads();
   }
+  // one record per touched expert, so a work item needs a single load to find its tokens
+  const int na = ws.n_active[0];
+  for (int a = tid; a < na; a += kRouteThreads) {
+    const int e = ws.active[a];
+    const int off = ws.offsets[e];
+    ws.act_info[a] = make_int4(e, ws.counts[e], off, ws.perm[off]);
+  }
 }
 
 // Block 0 groups the routes; the other blocks convert x (jobs in Q).
@@ -325,6 +333,7 @@ struct MgPhase {
   const int32_t* active;
   const int32_t* n_active;
   const int32_t* perm;
+  const int4* act_info;   // per touched expert: (expert, count, offset, first pair)
   uint32_t* ctr;          // work item counter (zeroed by k_moe_prep)
 };
 
@@ -340,7 +349,7 @@ __device__ __forceinline__ int4 ld_desc(const int4* d) {
 constexpr int kMgStages = 3;  // no x staging buffer here: room for a third 72 KB stage
 constexpr size_t kMgSmemBytes = size_t(kMgStages) * kGemvStageAlloc +
                                 size_t(2 * kGemvConsumerWarps * kGemvRedRows) * sizeof(float) +
-                                (3 * kMgStages) * sizeof(uint64_t) + size_t(kMgStages) * sizeof(int4);
+                                (3 * kMgStages) * sizeof(uint64_t) + size_t(2 * kMgStages) * sizeof(int4);
 static_assert(kMgSmemBytes <= 227 * 1024, "grouped GEMV shared memory");
 static_assert((size_t(kMgStages) * kGemvStageAlloc + size_t(2 * kGemvConsumerWarps * kGemvRedRows) * 4) % 16 == 0,
               "descriptors must be 16-byte aligned");
@@ -351,9 +360,9 @@ static_assert((size_t(kMgStages) * kGemvStageAlloc + size_t(2 * kGemvConsumerWar
 // waiting for it (full, parity).  Returns false if that wait gave up.
 // With `reuse` (same matrix as the previous item) and a single token, X already holds it.
 template <int KIND>
-__device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int fam, int e, int r0, int r1,
-                                        uint32_t stage_s, float* red, int& q, uint64_t* full, uint32_t parity, XUnit& X,
-                                        bool reuse) {
+__device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int4 d, int4 dt, uint32_t stage_s,
+                                        float* red, int& q, uint64_t* full, uint32_t parity, XUnit& X, bool reuse) {
+  const int fam = d.x, e = d.y, r0 = d.z, r1 = d.w;
   const bool shared = fam >= 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = M.units, row_bytes = M.row_bytes;
@@ -369,12 +378,20 @@ __device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int fa
   const uint32_t base = stage_s + src_lo + uint32_t(p) * UB;
   const float* scales = reinterpret_cast<const float*>(wbase + M.scale_off);
   const int nrows = r1 - r0;
-  const int ntok = shared ? P.tokens : P.counts[e];
-  const int32_t* list = shared ? nullptr : P.perm + P.offsets[e];
+  const int ntok = dt.x;                   // tokens of this expert (all tokens: shared)
+  const int32_t* list = P.perm + dt.y;     // their pairs, in token order
   const uint4* xq = shared ? P.s_xq : P.xq;
   float* out = P.out[fam];
+  // int4 row scales: lane l of a group holds the scale of the group's l-th row of the stage
+  float sc = 1.f;
+  if constexpr (is_i4(KIND)) {
+    const int rr = g + lane * groups;
+    if (in_group && rr < nrows) sc = __ldg(scales + r0 + rr);
+  }
+  int pid = shared ? 0 : dt.z;
   for (int tt = 0; tt < ntok; ++tt, ++q) {
-    const int pid = shared ? tt : __ldg(list + tt);
+    int next_pid = tt + 1;  // prefetched for the next token
+    if (!shared && tt + 1 < ntok) next_pid = __ldg(list + tt + 1);
     const int xrow = (shared || !P.x_by_token) ? pid : pid / P.top_k;
     if (active && !(reuse && ntok == 1)) load_xunit<KIND>(xq + (size_t(xrow) * units + p) * xrec_chunks(KIND), X);
     if (tt == 0 && !mbar_wait(full, parity)) return false;
@@ -401,14 +418,20 @@ __device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int fa
           v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
           v[1] += __shfl_xor_sync(0xffffffffu, v[1], o);
         }
+        float s0 = 1.f, s1 = 1.f;
+        if constexpr (is_i4(KIND)) {
+          if (gw == 1) {  // rows i and i + groups are the group's rows (i - g) / groups and + 1
+            const int n0 = (i - g) / groups;
+            s0 = __shfl_sync(0xffffffffu, sc, n0 & 31);
+            s1 = __shfl_sync(0xffffffffu, sc, (n0 + 1) & 31);
+            if (n0 >= 32) s0 = __ldg(scales + r0 + i);
+            if (n0 + 1 >= 32) s1 = __ldg(scales + r0 + i + groups);
+          }
+        }
         if (lane == 0) {
           if (gw == 1) {
-            if (is_i4(KIND)) v[0] *= __ldg(scales + r0 + i);
-            orow[i] = v[0];
-            if (two) {
-              if (is_i4(KIND)) v[1] *= __ldg(scales + r0 + i + groups);
-              orow[i + groups] = v[1];
-            }
+            orow[i] = v[0] * s0;
+            if (two) orow[i + groups] = v[1] * s1;
           } else {
             red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine] = v[0];
             if (two) red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine + 1] = v[1];
@@ -423,10 +446,10 @@ __device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int fa
         float v = 0.f;
         for (int jj = 0; jj < gw; ++jj) v += red[(par * kGemvConsumerWarps + g * gw + jj) * kGemvRedRows + lane];
         const int i = g + lane * groups;
-        if (is_i4(KIND)) v *= __ldg(scales + r0 + i);
-        orow[i] = v;
+        orow[i] = v * sc;  // lane l writes the group's l-th row (its scale prefetched above)
       }
     }
+    pid = next_pid;
   }
   if (ntok == 0) return mbar_wait(full, parity);
   return true;
@@ -439,9 +462,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   float* red = reinterpret_cast<float*>(smem + size_t(kMgStages) * kGemvStageAlloc);
-  int4* desc = reinterpret_cast<int4*>(red + 2 * kGemvConsumerWarps * kGemvRedRows);  // (family, expert, r0, r1)
+  // per slot: (family, expert, r0, r1), (tokens, offset in perm, first pair, 0)
+  int4* desc = reinterpret_cast<int4*>(red + 2 * kGemvConsumerWarps * kGemvRedRows);
   __shared__ MgMat fams[4];  // the phase's matrix families, indexed per item from shared memory
-  uint64_t* full = reinterpret_cast<uint64_t*>(desc + kMgStages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(desc + 2 * kMgStages);
   uint64_t* empty = full + kMgStages;
   uint64_t* dready = empty + kMgStages;  // the slot's descriptor is written (stage may be in flight)
 
@@ -494,6 +518,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
         item = first;
       }
       int fam, e = 0, k;
+      int4 tok = make_int4(P.tokens, 0, 0, 0);  // shared expert: all tokens in order
       if (item < n_sh) {
         fam = 2 + item / fams[2].nstages;
         k = item - (fam - 2) * fams[2].nstages;
@@ -503,7 +528,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
         r -= a * per_expert;
         fam = r / fams[0].nstages;
         k = r - fam * fams[0].nstages;
-        e = __ldg(P.active + a);
+        const int4 ai = __ldg(P.act_info + a);
+        e = ai.x;
+        tok = make_int4(ai.y, ai.z, ai.w, 0);
       }
       const MgMat& M = fams[fam];
       const int r0 = k * M.stage_rows;
@@ -514,7 +541,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
         break;
       }
       fence_proxy_async_smem();
-      desc[slot] = make_int4(fam, e, r0, r1);
+      desc[2 * slot] = make_int4(fam, e, r0, r1);
+      desc[2 * slot + 1] = tok;
       mbar_arrive(&dready[slot]);
       const uintptr_t wbeg = reinterpret_cast<uintptr_t>(M.base) + (fam >= 2 ? 0 : size_t(e) * M.stride);
       const uintptr_t wend = wbeg + size_t(M.rows) * M.row_bytes;
@@ -539,7 +567,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
     {  // end marker
       const int slot = s % kMgStages;
       if (ok && (s < kMgStages || mbar_wait(&empty[slot], uint32_t(s / kMgStages - 1) & 1u))) {
-        desc[slot] = make_int4(-1, 0, 0, 0);
+        desc[2 * slot] = make_int4(-1, 0, 0, 0);
         mbar_arrive(&dready[slot]);
       }
     }
@@ -559,8 +587,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
     const int slot = s % kMgStages;
     const uint32_t par = uint32_t(s / kMgStages) & 1u;
     if (!mbar_wait(&dready[slot], par)) return;
-    const int4 d = ld_desc(&desc[slot]);
+    const int4 d = ld_desc(&desc[2 * slot]);
     if (d.x < 0) return;
+    const int4 dt = ld_desc(&desc[2 * slot + 1]);
     // Another matrix: row groups may change, so every consumer warp must have finished the
     // previous item (including its group reductions).  The same matrix (next stage of a run):
     // same groups, and with one token its x is still in registers.
@@ -569,8 +598,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
     prev_fam = d.x;
     prev_e = d.y;
     const uint32_t stage_s = ring_s + uint32_t(slot) * kGemvStageAlloc;
-    const bool ok = d.x < 2 ? mg_item<KR>(P, fams[d.x], d.x, d.y, d.z, d.w, stage_s, red, q, &full[slot], par, X, same)
-                            : mg_item<KS>(P, fams[d.x], d.x, d.y, d.z, d.w, stage_s, red, q, &full[slot], par, X, same);
+    const bool ok = d.x < 2 ? mg_item<KR>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same)
+                            : mg_item<KS>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same);
     if (!ok) return;
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);

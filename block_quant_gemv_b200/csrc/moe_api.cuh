@@ -66,7 +66,7 @@ inline size_t xrec_bytes(int fmt, int rows, int cols) {
 }
 
 struct MoeWsLayout {
-  size_t counts, offsets, active, n_active, ctr, perm;
+  size_t counts, offsets, active, n_active, ctr, act_info, perm;
   size_t xq, s_xq, g, u, gs, us, hq, hsq, part, sout, total;
 };
 
@@ -85,6 +85,7 @@ inline MoeWsLayout moe_ws_layout(const bqg_moe_layer* L, int tokens) {
   o.active = take(4 * E);
   o.n_active = take(4);
   o.ctr = take(8);
+  o.act_info = take(16 * E);
   o.perm = take(4 * pairs);
   o.xq = take(xrec_bytes(L->expert_fmt, tokens, L->hidden));
   o.s_xq = sh ? take(xrec_bytes(L->shared_fmt, tokens, L->hidden)) : 0;
@@ -177,6 +178,7 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   route.n_active = reinterpret_cast<int32_t*>(ws + lay.n_active);
   route.perm = reinterpret_cast<int32_t*>(ws + lay.perm);
   route.ctr = reinterpret_cast<uint32_t*>(ws + lay.ctr);
+  route.act_info = reinterpret_cast<int4*>(ws + lay.act_info);
 
   // routed and shared matrix families
   const MgMat gate = mg_mat(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden);
@@ -211,6 +213,7 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   P.active = route.active;
   P.n_active = route.n_active;
   P.perm = route.perm;
+  P.act_info = route.act_info;
 
   // 2. gate/up of the touched experts (and of the shared expert)
   P.m[0] = gate;
