@@ -480,7 +480,7 @@ def time_moe_gemma(dev, seed, peak, copies=8):
 
 def time_moe_glm(dev, seed, peak):
     """GLM-like stack: 8 resident layers of 256 int4-row SwiGLU experts (38.7 GB), given N(0,1)
-    logits, top-8, layers chained (x of layer l+1 = y of layer l); T = 1, 8, 64."""
+    logits, top-8, run back to back, each layer on its own seeded N(0,1) input; T = 1, 8, 64."""
     import torch
 
     import block_quant_gemv_b200 as bqg
@@ -491,18 +491,19 @@ def time_moe_glm(dev, seed, peak):
     expert_bytes = sum(spec.mat_bytes(w) for w in ("gate", "up", "down"))
     resident = sum(T.gate.numel() + T.up.numel() + T.down.numel() for T in Ts)
     out = {"workload": f"glm_moe: {wl.GLM_LAYERS} layers x 256 int4-row experts (hidden 6144, SwiGLU 2048), "
-                       f"top-8 of given N(0,1) logits, chained; {resident / 1e9:.1f} GB resident"}
+                       f"top-8 of given N(0,1) logits, layers back to back; {resident / 1e9:.1f} GB resident"}
     for T in (1, 8, 64):
         logits = [wl.moe_logits(spec, seed, l, T).to(dev) for l in range(len(Ls))]
         idx = [torch.empty(T, spec.top_k, dtype=torch.int32, device=dev) for _ in Ls]
         w = [torch.empty(T, spec.top_k, device=dev) for _ in Ls]
-        xs = [wl.moe_tokens(spec, seed, T).to(dev)] + [torch.empty(T, spec.hidden, device=dev) for _ in Ls]
+        xs = [wl.moe_tokens(spec, seed, T, layer=l).to(dev) for l in range(len(Ls))]
+        ys = [torch.empty(T, spec.hidden, device=dev) for _ in Ls]
         ws = torch.empty(bqg.moe_workspace_size(Ls[0], T), dtype=torch.uint8, device=dev)
 
         def fn():
             for l in range(len(Ls)):
                 bqg.moe_router_topk(logits[l], spec.top_k, idx[l], w[l])
-                bqg.moe_forward(Ls[l], xs[l], idx[l], w[l], xs[l + 1], ws)
+                bqg.moe_forward(Ls[l], xs[l], idx[l], w[l], ys[l], ws)
         us = graph_us(fn, reps=5) / len(Ls)
         distinct = sum(int(torch.unique(i).numel()) for i in idx) / len(Ls)
         nbytes = distinct * expert_bytes + 8 * T * spec.hidden + 4 * T * spec.n_experts

@@ -7,8 +7,8 @@
 // "Engine status" (GPU-resident single-shot prefill).
 //
 // One CTA computes a 128 (tokens, padded) x 128 (output features) tile over a range of k.
-//   warp 0     TMA: X tiles (128 rows x 64 k, fp16, 128-byte swizzle) and raw Q4_0 row chunks
-//              (128 rows x 144 bytes = 256 k) into shared-memory rings.
+//   warp 0     TMA: X tiles (128 rows x 64 k, fp16, 128-byte swizzle; 5-deep ring) and raw Q4_0
+//              row chunks (128 rows x 144 bytes = 256 k; 3-deep ring) into shared memory.
 //   warp 1     allocates the 128-column fp32 accumulator in tensor memory and issues the
 //              tcgen05.mma instructions (M=128, N=128, K=16 each, both operands K-major in
 //              shared memory); tcgen05.commit frees each stage when its MMAs have read it.
@@ -32,7 +32,7 @@ constexpr int kPfThreads = 192;           // 6 warps
 constexpr int kPfTileN = 128;             // output features per CTA
 constexpr int kPfTileM = 128;             // tokens per CTA (MMA M)
 constexpr int kPfStageK = 64;             // k per stage (one 128-byte swizzle row of fp16)
-constexpr int kPfStages = 4;              // A/B stage ring depth
+constexpr int kPfStages = 5;              // A/B stage ring depth
 constexpr int kPfRawK = 256;              // k per raw Q4_0 chunk (8 blocks = 144 bytes per row)
 constexpr int kPfRawBytesRow = kPfRawK / 32 * 18;  // 144
 constexpr int kPfRawStages = 3;
@@ -43,6 +43,9 @@ constexpr int kPfMaxSplit = 8;            // k-splits per tile (cluster size)
 // smem: [A ring | B ring] (1024-aligned), raw ring, barriers, tmem address; + 1 KB alignment slack
 constexpr size_t kPfSmemBytes = 1024 + size_t(kPfStages) * (kPfABytes + kPfBBytes) +
                                 size_t(kPfRawStages) * kPfRawBytes + 256;
+static_assert(kPfSmemBytes <= 227 * 1024, "prefill shared memory");
+static_assert(size_t(kPfStages) * kPfABytes >= size_t(kPfTileN + 4) * kPfTileM * 4, "split-k partial tile parks in the A ring");
+static_assert((2 * kPfStages + 2 * kPfRawStages + 1) * 8 + 8 <= 256, "barrier area");
 
 struct PfParams {
   void* Y;           // fp16 [tokens x n]
@@ -136,11 +139,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t rank) {
+// 16 bytes at the same shared-memory offset in cluster rank `rank` (its own rank included).
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_saddr, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(remote)
+               : "memory");
   return v;
 }
 
@@ -302,9 +309,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   // ------------------------------------------------ epilogue: accumulator -> fp16 Y
   // Warps 2-5 own the accumulator rows (tensor-memory lanes 32*(warp%4) .. +31 = tokens).  With a
-  // k-split cluster every CTA parks its partial tile in its (now idle) A ring and rank 0 sums the
-  // ranks in order through distributed shared memory; every thread of every CTA takes part in the
-  // two cluster barriers.
+  // k-split cluster every CTA parks its partial tile in its (now idle) A ring; rank r then sums
+  // its slice of the columns over all ranks, in rank order, through distributed shared memory.
+  // Every thread of every CTA takes part in the two cluster barriers.
   const bool epi_warp = warp >= 2;
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;  // token
@@ -313,7 +320,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     have = !*abort_flag && mbar_wait(done, 0);
     tc_fence_after();
   }
-  float* park = reinterpret_cast<float*>(a_ring);  // [kPfTileN][kPfTileM] fp32 = 64 KB
+  // partial tile, row-major with a 4-float pad per row (conflict-free 16-byte accesses)
+  constexpr int kPitch = kPfTileN + 4;
+  float* park = reinterpret_cast<float*>(a_ring);  // [kPfTileM][kPitch] fp32 = 66 KB
   const uint32_t tm_row = tmem + (uint32_t(quarter * 32) << 16);
   if (prm.ksplit > 1) {
     if (epi_warp) {
@@ -322,22 +331,34 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint32_t r16[16];
         if (have) tmem_ld16(tm_row + uint32_t(c), r16);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) park[(c + i) * kPfTileM + row] = have ? __uint_as_float(r16[i]) : 0.f;
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(&park[row * kPitch + c + i]) =
+              have ? make_float4(__uint_as_float(r16[i]), __uint_as_float(r16[i + 1]), __uint_as_float(r16[i + 2]),
+                                 __uint_as_float(r16[i + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     __syncwarp();
     cluster_sync();
-    if (epi_warp && cluster_ctarank() == 0 && row < prm.tokens) {
-      __half* y = static_cast<__half*>(prm.Y) + size_t(row) * prm.n + n0;
-      const int ncols = min(kPfTileN, prm.n - n0);
+    // rank r sums columns [r * cw, (r + 1) * cw) of every rank's tile, in rank order
+    const int cw = kPfTileN / prm.ksplit;  // 16, 32 or 64
+    const int rank = int(cluster_ctarank());
+    const int c0 = rank * cw;
+    const int ncols = min(cw, prm.n - n0 - c0);
+    if (epi_warp && row < prm.tokens && ncols > 0) {
+      __half* y = static_cast<__half*>(prm.Y) + size_t(row) * prm.n + n0 + c0;
 #pragma unroll 1
       for (int c = 0; c < ncols; c += 8) {
         float v[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = park[(c + i) * kPfTileM + row];
-        for (int rk = 1; rk < prm.ksplit; ++rk)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] += ld_dsmem_f32(smem_u32(&park[(c + i) * kPfTileM + row]), uint32_t(rk));
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+        for (int rk = 0; rk < prm.ksplit; ++rk) {
+          const uint32_t a = smem_u32(&park[row * kPitch + c0 + c]);
+          const float4 lo = ld_dsmem_f32x4(a, uint32_t(rk));
+          const float4 hi = ld_dsmem_f32x4(a + 16, uint32_t(rk));
+          v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
+          v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
+        }
         uint4 pk;
         pk.x = h2_bits(__floats2half2_rn(v[0], v[1]));
         pk.y = h2_bits(__floats2half2_rn(v[2], v[3]));
@@ -347,7 +368,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
     __syncwarp();
-    cluster_sync();  // peers keep their shared memory until rank 0 has read it
+    cluster_sync();  // every rank keeps its shared memory until all ranks have read it
   } else if (epi_warp && have) {
     // tcgen05.ld is warp-collective: every lane loads, only rows < tokens store
     __half* y = static_cast<__half*>(prm.Y) + size_t(row) * prm.n + n0;

@@ -139,7 +139,9 @@ class MoESpec:
 # shared dense GeGLU expert of 2112 in Q8_0, fp32 router 128 x 2816.
 GEMMA_MOE = MoESpec("gemma_moe", 128, 8, 2816, 704, FMT_Q4_0, 1, 2112, FMT_Q8_0, True)
 # GLM-style layer: hidden 6144, 256 experts, top-8, SwiGLU experts of 2048 in packed int4 with
-# fp32 row scales, no shared expert, logits given (N(0,1)); 8 such layers are stacked.
+# fp32 row scales, no shared expert, logits given (N(0,1)); 8 such layers are stacked, resident
+# together, and run back to back, each on its own seeded N(0,1) input (feeding a layer's output
+# straight into the next, with no norm in between, overflows fp32 by the fifth layer).
 GLM_MOE = MoESpec("glm_moe", 256, 8, 6144, 2048, FMT_I4_ROW, 2, 0, 0, False)
 GLM_LAYERS = 8
 
@@ -192,9 +194,11 @@ def build_moe_layer(spec: MoESpec, seed: int, layer: int = 0, device="cuda") -> 
                       shared, R)
 
 
-def moe_tokens(spec: MoESpec, seed: int, tokens: int) -> torch.Tensor:
-    """Host fp32 activations x ~ N(0, 1), [tokens, hidden]."""
-    return normal_f32(seed, stream_id(f"{spec.name}/x/T{tokens}"), tokens * spec.hidden).view(tokens, spec.hidden)
+def moe_tokens(spec: MoESpec, seed: int, tokens: int, layer: Optional[int] = None) -> torch.Tensor:
+    """Host fp32 activations x ~ N(0, 1), [tokens, hidden]; with `layer`, the input of that
+    layer of a stack (each layer of the stack takes its own seeded input)."""
+    name = f"{spec.name}/x/T{tokens}" if layer is None else f"{spec.name}/L{layer}/x/T{tokens}"
+    return normal_f32(seed, stream_id(name), tokens * spec.hidden).view(tokens, spec.hidden)
 
 
 def moe_logits(spec: MoESpec, seed: int, layer: int, tokens: int) -> torch.Tensor:

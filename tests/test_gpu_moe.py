@@ -129,3 +129,35 @@ def test_gemma_like_moe_layer_full_size(tokens):
     assert_close(y.cpu().numpy()[same], ref[same], what=f"gemma-like MoE T={tokens}")
     ref_routed = om.moe_layer(lay, x.numpy(), ridx, rw, with_shared=False)
     assert_close(y_routed.cpu().numpy()[same], ref_routed[same], what=f"gemma-like routed branch T={tokens}")
+
+
+def _glm_layer_check(L, spec, layer, tokens, sample=None):
+    x = wl.moe_tokens(spec, 0, tokens, layer=layer)
+    lg = wl.moe_logits(spec, 0, layer, tokens)
+    idx, w = bqg.moe_router_topk(lg.cuda(), spec.top_k)
+    y = bqg.moe_forward(device_layer(L), x.cuda(), idx, w)
+    torch.cuda.synchronize()
+    ridx, rw = om.router_topk(lg.numpy(), spec.top_k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)            # same fp32 logits: bit-exact
+    sel = np.arange(tokens) if sample is None else np.asarray(sample)
+    ref = om.moe_layer(oracle_layer(spec, 0, layer), x.numpy()[sel], ridx[sel], rw[sel])
+    assert_close(y.cpu().numpy()[sel], ref, what=f"glm-like layer {layer} T={tokens}")
+    assert_close(y.cpu().numpy()[sel], ref, tol=1e-4, what=f"glm-like layer {layer} T={tokens} (x fixed point)")
+
+
+def test_glm_like_stack_full_size():
+    """Hidden 6144, 256 int4-row SwiGLU experts of 2048, top-8 of given N(0,1) logits: all 8
+    layers resident at once (38.7 GB); every layer at T=1 against the oracle, and one layer at
+    T=8 and T=64 on sampled tokens."""
+    need_gpu()
+    spec = wl.GLM_MOE
+    layers = [wl.build_moe_layer(spec, 0, l, device="cuda") for l in range(wl.GLM_LAYERS)]
+    resident = sum(T.gate.numel() + T.up.numel() + T.down.numel() for T in layers)
+    assert resident == 8 * 256 * 18_915_328
+    for l, L in enumerate(layers):
+        _glm_layer_check(L, spec, l, 1)
+    _glm_layer_check(layers[3], spec, 3, 8, sample=[0, 7])
+    _glm_layer_check(layers[5], spec, 5, 64, sample=[13, 50])
+    del layers
+    torch.cuda.empty_cache()
+    assert bqg.bqg_device_errors() == 0
