@@ -347,6 +347,21 @@ __device__ __forceinline__ int4 ld_desc(const int4* d) {
 }
 
 constexpr int kMgStages = 3;  // no x staging buffer here: room for a third 72 KB stage
+// The 15 consumer warps form two teams of 7 that take alternate items of the ring (the 15th
+// warp idles): two items are in progress per SM, so one team's x loads, barrier and
+// descriptor waits overlap the other team's dot products.
+constexpr int kMgTeams = 2;
+constexpr int kMgTeamWarps = 7;
+constexpr int kMgMaxUnits = 32 * kMgTeamWarps;  // units per row a team can cover
+__host__ __device__ constexpr int mg_groups(int units) { return kMgTeamWarps / gemv_group_warps(units); }
+// Rows per stage: as many whole rows as fit 72 KB, a multiple of the team's row groups, and
+// (when a group spans several warps) at most 32 rows per group (one reducing lane per row).
+__host__ __device__ constexpr int mg_stage_rows(int units, int row_bytes) {
+  return ((gemv_group_warps(units) > 1 && kGemvStageBytes / row_bytes > 32 * mg_groups(units))
+              ? 32 * mg_groups(units)
+              : kGemvStageBytes / row_bytes) /
+         mg_groups(units) * mg_groups(units);
+}
 constexpr size_t kMgSmemBytes = size_t(kMgStages) * kGemvStageAlloc +
                                 size_t(2 * kGemvConsumerWarps * kGemvRedRows) * sizeof(float) +
                                 (3 * kMgStages) * sizeof(uint64_t) + size_t(2 * kMgStages) * sizeof(int4);
@@ -361,14 +376,16 @@ static_assert((size_t(kMgStages) * kGemvStageAlloc + size_t(2 * kGemvConsumerWar
 // With `reuse` (same matrix as the previous item) and a single token, X already holds it.
 template <int KIND>
 __device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int4 d, int4 dt, uint32_t stage_s,
-                                        float* red, int& q, uint64_t* full, uint32_t parity, XUnit& X, bool reuse) {
+                                        float* red, int& q, uint64_t* full, uint32_t parity, XUnit& X, bool reuse,
+                                        int team) {
   const int fam = d.x, e = d.y, r0 = d.z, r1 = d.w;
   const bool shared = fam >= 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tw = warp - team * kMgTeamWarps;  // warp within the team
   const int units = M.units, row_bytes = M.row_bytes;
   const int gw = gemv_group_warps(units);
-  const int groups = gemv_groups(units);
-  const int g = warp / gw, j = warp - g * gw;
+  const int groups = mg_groups(units);
+  const int g = tw / gw, j = tw - g * gw;
   const int p = 32 * j + lane;
   const bool in_group = g < groups;
   const bool active = in_group && p < units;
@@ -441,10 +458,11 @@ __device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int4 d
       }
     }
     if (gw > 1 && in_group) {
-      named_bar_sync(2 + g, 32 * gw);
+      named_bar_sync(3 + 3 * team + g, 32 * gw);  // gw > 1: at most 3 groups per team
       if (j == 0 && lane < nmine) {
         float v = 0.f;
-        for (int jj = 0; jj < gw; ++jj) v += red[(par * kGemvConsumerWarps + g * gw + jj) * kGemvRedRows + lane];
+        for (int jj = 0; jj < gw; ++jj)
+          v += red[(par * kGemvConsumerWarps + team * kMgTeamWarps + g * gw + jj) * kGemvRedRows + lane];
         const int i = g + lane * groups;
         orow[i] = v * sc;  // lane l writes the group's l-th row (its scale prefetched above)
       }
@@ -473,7 +491,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMgStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kGemvConsumerWarps);
+      mbar_init(&empty[i], kMgTeamWarps);  // the team that takes the slot's item
       mbar_init(&dready[i], 1);
     }
     for (int i = 0; i < 4; ++i) fams[i] = P.m[i];
@@ -564,12 +582,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
       }
       ++s;
     }
-    {  // end marker
+    // end markers, one for each team (the next item of each team)
+    for (int t = 0; t < kMgTeams && ok; ++t, ++s) {
       const int slot = s % kMgStages;
-      if (ok && (s < kMgStages || mbar_wait(&empty[slot], uint32_t(s / kMgStages - 1) & 1u))) {
-        desc[2 * slot] = make_int4(-1, 0, 0, 0);
-        mbar_arrive(&dready[slot]);
+      if (s >= kMgStages && !mbar_wait(&empty[slot], uint32_t(s / kMgStages - 1) & 1u)) {
+        ok = false;
+        break;
       }
+      desc[2 * slot] = make_int4(-1, 0, 0, 0);
+      mbar_arrive(&dready[slot]);
     }
     if (!ok) {
       for (int qq = (s > kMgStages ? s - kMgStages : 0); qq < s; ++qq)
@@ -579,11 +600,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
   }
 
   // ------------------------------------------------ consumers
+  const int team = warp / kMgTeamWarps;
+  if (team >= kMgTeams) return;  // the odd warp out
   const uint32_t ring_s = smem_u32(ring);
   int q = 0;
   int prev_fam = -1, prev_e = -1;
   XUnit X;
-  for (int s = 0;; ++s) {
+  for (int s = team;; s += kMgTeams) {
     const int slot = s % kMgStages;
     const uint32_t par = uint32_t(s / kMgStages) & 1u;
     if (!mbar_wait(&dready[slot], par)) return;
@@ -594,12 +617,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
     // previous item (including its group reductions).  The same matrix (next stage of a run):
     // same groups, and with one token its x is still in registers.
     const bool same = d.x == prev_fam && d.y == prev_e;
-    if (!same) named_bar_sync(1, kGemvCompute);
+    if (!same) named_bar_sync(1 + team, 32 * kMgTeamWarps);
     prev_fam = d.x;
     prev_e = d.y;
     const uint32_t stage_s = ring_s + uint32_t(slot) * kGemvStageAlloc;
-    const bool ok = d.x < 2 ? mg_item<KR>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same)
-                            : mg_item<KS>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same);
+    const bool ok = d.x < 2 ? mg_item<KR>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same, team)
+                            : mg_item<KS>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same, team);
     if (!ok) return;
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);

@@ -7,13 +7,15 @@
 
 namespace bqg {
 
-constexpr int kMoeMaxCols = 8192;  // hidden / inter / shared_inter limit of moe_forward
+constexpr int kMoeMaxCols = BQG_MAX_MOE_COLS;  // hidden / inter / shared_inter limit of moe_forward
+static_assert(kMoeMaxCols / 32 <= kMgMaxUnits, "one-block units of the widest row must fit a consumer team");
 
 inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 // Unit kind of a matrix format in the grouped GEMV: one block for Q8_0 and Q4_0 (a row of
 // hidden/inter values then fills more lanes than pairs of blocks would: 88 units for 2816
-// columns, 22 for 704), 64 values for int4 when the columns allow, else 32.
+// columns, 22 for 704), 64 values for int4 when the columns allow, else 32.  Rows of up to
+// BQG_MAX_MOE_COLS values give at most 224 units, one per lane of a 7-warp consumer team.
 inline int moe_kind(int fmt, int cols) {
   if (fmt == BQG_Q8_0) return kQ8One;
   if (fmt == BQG_Q4_0) return kQ4One;
@@ -55,7 +57,7 @@ inline MgMat mg_mat(int fmt, const void* base, size_t stride, int rows, int cols
   M.row_bytes = mg_row_bytes(fmt, cols);
   M.units = cols / unit_weights(M.kind);
   M.scale_off = fmt == BQG_I4_ROW ? int((size_t(rows) * M.row_bytes + 15) / 16 * 16) : 0;
-  M.stage_rows = gemv_stage_rows(M.units, M.row_bytes);
+  M.stage_rows = mg_stage_rows(M.units, M.row_bytes);
   M.nstages = (rows + M.stage_rows - 1) / M.stage_rows;
   return M;
 }

@@ -71,7 +71,7 @@ enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 #define BQG_MAX_BATCH 256        /* largest descriptor count of one qgemv_batched call     */
 #define BQG_MAX_EXPERTS 256      /* largest n_experts of the router / MoE calls            */
 #define BQG_MAX_TOPK 8           /* largest k of the router / MoE calls                    */
-#define BQG_MAX_MOE_COLS 8192    /* largest hidden / inter / shared_inter of moe_forward   */
+#define BQG_MAX_MOE_COLS 7168    /* largest hidden / inter / shared_inter of moe_forward   */
 
 /* Device-side error bits, reported by bqg_device_errors(). */
 #define BQG_DEVERR_TIMEOUT 0x1   /* a bounded in-kernel wait gave up (the kernel returned early) */
