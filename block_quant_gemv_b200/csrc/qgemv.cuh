@@ -6,8 +6,9 @@
 //                y_r = s_r * sum_i q_ri x_i                 (int4 with per-row scale).
 //
 // Design (B200):
-//  * The problem list is one byte stream.  Each CTA (one per SM) owns a contiguous,
-//    byte-balanced range of rows (computed on the host), cut into stages of whole rows.
+//  * The problem list is one stream of rows.  Each CTA (one per SM) owns a contiguous range of
+//    rows of about equal cost (bytes, with nibble-format bytes weighted 1.5; computed on the
+//    host), cut into stages of whole rows.
 //  * A producer warp streams the stages with 1-D bulk copies (TMA) into two 72 KB shared-memory
 //    slots (double buffering), completing on mbarriers.  Rows keep their canonical byte
 //    layout (18/34-byte blocks); an unaligned start is copied from the 16-byte boundary below.
@@ -63,7 +64,7 @@ struct GemvProb {
   const uint8_t* W;
   const float* x;
   float* y;
-  long long byte_start;  // offset of this matrix's rows in the concatenated stream
+  long long byte_start;  // host: the matrix's first cost unit in the whole list (partitioning)
   int rows;
   int cols;
   int kind;       // UnitKind

@@ -52,6 +52,12 @@ inline int make_gemv_prob(int fmt, const void* W, const float* x, float* y, int 
   return BQG_OK;
 }
 
+// Cost of a Q4_0 / int4 byte relative to a Q8_0 byte, in sixteenths (1.5 measured best on the
+// decode step: 115.0 us against 117.2 us for a pure byte split; 2.0 gives 134 us).
+#ifndef BQG_GEMV_NIBBLE_COST16
+#define BQG_GEMV_NIBBLE_COST16 24
+#endif
+
 inline SmemAttrOnce g_gemv_attr1, g_gemv_attrN;
 
 template <int MAXP>
@@ -63,26 +69,31 @@ inline int launch_gemv(GemvParams<MAXP>& prm, long long total_rows, cudaStream_t
   SmemAttrOnce& attr = (MAXP == 1) ? g_gemv_attr1 : g_gemv_attrN;
   st = attr.ensure(dev, k_qgemv<MAXP>, kGemvSmemBytes);
   if (st != BQG_OK) return st;
+  // Cost-balanced split: a row costs its bytes times a per-format weight in sixteenths (the
+  // nibble formats carry about twice the weights per byte of Q8_0, so more integer dot work per
+  // byte).  CTA c owns the rows whose first cost unit lies in [c*T/G, (c+1)*T/G).
   long long total = 0;
+  long long row_cost[MAXP];
   for (int i = 0; i < prm.n; ++i) {
-    prm.p[i].byte_start = total;
-    total += (long long)prm.p[i].rows * prm.p[i].row_bytes;
+    const int w16 = is_q8(prm.p[i].kind) ? 16 : BQG_GEMV_NIBBLE_COST16;
+    row_cost[i] = (long long)prm.p[i].row_bytes * w16;
+    prm.p[i].byte_start = total;  // here: the matrix's first cost unit
+    total += (long long)prm.p[i].rows * row_cost[i];
   }
   prm.total_bytes = total;
   long long g = total_rows < info->sm_count ? total_rows : info->sm_count;
   if (g > kGemvMaxGrid) g = kGemvMaxGrid;
   const int grid = int(g);
-  // Byte-balanced split: CTA c owns the rows whose first byte lies in [c*T/G, (c+1)*T/G).
-  // first_row(b) = the first (problem, row) whose start byte is >= b; b grows with c, so one
+  // first_row(b) = the first (problem, row) whose start cost is >= b; b grows with c, so one
   // forward sweep over the problems serves all CTAs.
   int sweep = 0;
   auto first_row = [&](long long b, int& p, int& r) {
     for (p = sweep; p < prm.n; ++p) {
       const GemvProb& P = prm.p[p];
-      const long long end = P.byte_start + (long long)P.rows * P.row_bytes;
+      const long long end = P.byte_start + (long long)P.rows * row_cost[p];
       if (b < end) {
         const long long off = b - P.byte_start;
-        r = off <= 0 ? 0 : int((off + P.row_bytes - 1) / P.row_bytes);
+        r = off <= 0 ? 0 : int((off + row_cost[p] - 1) / row_cost[p]);
         if (r < P.rows) {
           sweep = p;
           return;
