@@ -143,6 +143,14 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=5)
+        if not self.lines:
+            # a timed region shorter than the sampling period: one query right after it
+            try:
+                out = subprocess.run(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                      "-i", str(self.gpu)], capture_output=True, text=True, timeout=10).stdout
+                self.lines = [ln.strip() for ln in out.splitlines() if ln.strip()]
+            except (OSError, subprocess.SubprocessError):
+                pass
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
