@@ -22,7 +22,10 @@
  *   - Arguments are validated on the host before any launch.  A failed check returns a
  *     negative bqg_status and launches nothing.  A failed launch returns BQG_ERR_CUDA.
  *   - Sizes are element counts unless named *_bytes.  Matrices are row-major.
- *   - Float outputs are fp32 (fp16 for the prefill GEMM).  Accumulation is fp32.
+ *   - Float outputs are fp32 (fp16 for the prefill GEMM).  The GEMV and MoE kernels hold each
+ *     32 or 64 activation values as 16-bit fixed point with their own scale
+ *     (|x - s X| <= max|x| / 65534), sum each block's products exactly in int32 and the blocks
+ *     in fp32; the prefill GEMM multiplies fp16 operands with fp32 accumulation.
  *
  * Weight formats (the byte layout of one matrix with `rows` rows of `cols` weights; rows are
  * stored one after another, row r holding its cols/32 blocks in order):
@@ -67,7 +70,7 @@ enum bqg_status {
 enum bqg_fmt { BQG_Q8_0 = 1, BQG_Q4_0 = 2, BQG_I4_ROW = 3 };
 enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 
-#define BQG_MAX_COLS 15360       /* largest cols (K) accepted by the GEMV and MoE calls     */
+#define BQG_MAX_COLS 15360       /* largest cols (K) of the GEMV, router and prefill calls  */
 #define BQG_MAX_BATCH 256        /* largest descriptor count of one qgemv_batched call     */
 #define BQG_MAX_EXPERTS 256      /* largest n_experts of the router / MoE calls            */
 #define BQG_MAX_TOPK 8           /* largest k of the router / MoE calls                    */
