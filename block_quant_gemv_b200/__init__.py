@@ -25,7 +25,7 @@ __all__ = [
 
 Q8_0, Q4_0, I4_ROW = 1, 2, 3
 ACT_GELU_TANH, ACT_SILU = 1, 2
-MAX_COLS, MAX_BATCH, MAX_EXPERTS, MAX_TOPK = 15360, 256, 256, 8
+MAX_COLS, MAX_BATCH, MAX_EXPERTS, MAX_TOPK, MAX_MOE_COLS = 15360, 256, 256, 8, 7168
 DEVERR_TIMEOUT, DEVERR_EXPERT_ID = 0x1, 0x2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

@@ -147,3 +147,14 @@ def test_moe_argument_errors(L):
     assert fwd(ctypes.byref(c), A, A, A, A, 16, A, size, None) == -1
     c.act, c.hidden = 1, 2820
     assert L.lib().moe_workspace_size(ctypes.byref(c), 16) == 0
+
+
+def test_binding_limits_match_header():
+    import re
+    import block_quant_gemv_b200 as bqg
+    text = open(os.path.join(ROOT, "include", "bqg.h")).read()
+    for name, val in (("BQG_MAX_COLS", bqg.MAX_COLS), ("BQG_MAX_BATCH", bqg.MAX_BATCH),
+                      ("BQG_MAX_EXPERTS", bqg.MAX_EXPERTS), ("BQG_MAX_TOPK", bqg.MAX_TOPK),
+                      ("BQG_MAX_MOE_COLS", bqg.MAX_MOE_COLS)):
+        m = re.search(rf"#define {name} (\d+)", text)
+        assert m and int(m.group(1)) == val, name
