@@ -111,9 +111,12 @@ def test_tinyllama_decode_step_full_size_sampled():
     need_gpu()
     specs = wl.decode_step_specs()
     W = wl.build_gemv_workload(specs, seed=0, device="cuda")
+    W.y_all.fill_(float("nan"))
     batch = bqg.GemvBatch(W.items())
     batch.run()
     torch.cuda.synchronize()
+    for i, s in enumerate(specs):  # every row of every matrix written (static ranges and claimed tail)
+        assert torch.isfinite(W.y(i)).all(), s.name
     rng = np.random.default_rng(0)
     xs = {}
     for i, s in enumerate(specs):
