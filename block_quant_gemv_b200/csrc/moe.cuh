@@ -373,7 +373,8 @@ static_assert((size_t(kMgStages) * kGemvStageAlloc + size_t(2 * kGemvConsumerWar
 // q counts token iterations (selects the group reduction buffer).
 // The weight stage may still be in flight on entry: the first token's x is loaded before
 // waiting for it (full, parity).  Returns false if that wait gave up.
-// With `reuse` (same matrix as the previous item) and a single token, X already holds it.
+// With `reuse` (a single token whose input record the team's previous item also used), X
+// already holds it.
 template <int KIND>
 __device__ __forceinline__ bool mg_item(const MgPhase& P, const MgMat& M, int4 d, int4 dt, uint32_t stage_s,
                                         float* red, int& q, uint64_t* full, uint32_t parity, XUnit& X, bool reuse,
@@ -604,7 +605,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
   if (team >= kMgTeams) return;  // the odd warp out
   const uint32_t ring_s = smem_u32(ring);
   int q = 0;
-  int prev_fam = -1, prev_e = -1;
+  int prev_units = -1, prev_routed = -1;  // row shape of the team's previous item
+  int prev_x = -1;                        // input record held in X (one-token items), else -1
   XUnit X;
   for (int s = team;; s += kMgTeams) {
     const int slot = s % kMgStages;
@@ -613,16 +615,27 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
     const int4 d = ld_desc(&desc[2 * slot]);
     if (d.x < 0) return;
     const int4 dt = ld_desc(&desc[2 * slot + 1]);
-    // Another matrix: row groups may change, so every consumer warp must have finished the
-    // previous item (including its group reductions).  The same matrix (next stage of a run):
-    // same groups, and with one token its x is still in registers.
-    const bool same = d.x == prev_fam && d.y == prev_e;
-    if (!same) named_bar_sync(1 + team, 32 * kMgTeamWarps);
-    prev_fam = d.x;
-    prev_e = d.y;
+    // Another row shape (units per row or unit kind): row groups may change, so every consumer
+    // warp of the team must have finished the previous item, including its group reductions.
+    // Items of the same shape (another stage, gate after up, another expert) keep the groups,
+    // and each group's own barrier orders its reduction buffers.
+    const int routed = d.x < 2 ? 1 : 0;
+    const int units = fams[d.x].units;
+    if (units != prev_units || routed != prev_routed) named_bar_sync(1 + team, 32 * kMgTeamWarps);
+    prev_units = units;
+    prev_routed = routed;
+    // One token: X may already hold its input record (the same token for every routed gate/up
+    // item, the same pair for every stage of one expert's down matrix).
+    int xkey = -1;
+    if (dt.x == 1) {
+      const int pid = routed ? dt.z : 0;
+      xkey = 2 * ((routed && P.x_by_token) ? pid / P.top_k : pid) + routed;
+    }
+    const bool reuse = xkey >= 0 && xkey == prev_x;
+    prev_x = xkey;
     const uint32_t stage_s = ring_s + uint32_t(slot) * kGemvStageAlloc;
-    const bool ok = d.x < 2 ? mg_item<KR>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same, team)
-                            : mg_item<KS>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, same, team);
+    const bool ok = routed ? mg_item<KR>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, reuse, team)
+                           : mg_item<KS>(P, fams[d.x], d, dt, stage_s, red, q, &full[slot], par, X, reuse, team);
     if (!ok) return;
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
