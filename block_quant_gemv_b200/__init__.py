@@ -194,11 +194,17 @@ def qgemm_prefill(fmt: int, W: torch.Tensor, X: torch.Tensor, n: int, k: int,
 def moe_router_logits(R: torch.Tensor, x: torch.Tensor, logits: Optional[torch.Tensor] = None) -> torch.Tensor:
     _need_cuda("R", R, torch.float32)
     _need_cuda("x", x, torch.float32)
+    if R.dim() != 2:
+        raise ValueError("R must be [n_experts, hidden]")
     n_experts, hidden = R.shape
     tokens = x.numel() // hidden
+    if tokens < 1 or x.numel() != tokens * hidden:
+        raise ValueError(f"x must hold whole tokens of {hidden} values")
     if logits is None:
         logits = torch.empty(tokens, n_experts, dtype=torch.float32, device=x.device)
     _need_cuda("logits", logits, torch.float32)
+    if logits.numel() < tokens * n_experts:
+        raise ValueError(f"logits must hold tokens x n_experts = {tokens} x {n_experts} values")
     _check(lib().moe_router_logits(_ptr(R), _ptr(x), _ptr(logits), tokens, n_experts, hidden, _stream(x)),
            "moe_router_logits")
     return logits
@@ -207,6 +213,8 @@ def moe_router_logits(R: torch.Tensor, x: torch.Tensor, logits: Optional[torch.T
 def moe_router_topk(logits: torch.Tensor, k: int, idx: Optional[torch.Tensor] = None,
                     weights: Optional[torch.Tensor] = None):
     _need_cuda("logits", logits, torch.float32)
+    if logits.dim() != 2:
+        raise ValueError("logits must be [tokens, n_experts]")
     tokens, n_experts = logits.shape
     if idx is None:
         idx = torch.empty(tokens, k, dtype=torch.int32, device=logits.device)
@@ -214,6 +222,8 @@ def moe_router_topk(logits: torch.Tensor, k: int, idx: Optional[torch.Tensor] = 
         weights = torch.empty(tokens, k, dtype=torch.float32, device=logits.device)
     _need_cuda("idx", idx, torch.int32)
     _need_cuda("weights", weights, torch.float32)
+    if idx.numel() < tokens * k or weights.numel() < tokens * k:
+        raise ValueError(f"idx and weights must hold tokens x k = {tokens} x {k} values")
     _check(lib().moe_router_topk(_ptr(logits), tokens, n_experts, k, _ptr(idx), _ptr(weights), _stream(logits)),
            "moe_router_topk")
     return idx, weights
@@ -230,6 +240,20 @@ class MoELayer:
                  gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor,
                  gate_stride: int, up_stride: int, down_stride: int, shared=None):
         self.tensors = [gate, up, down]
+
+        def need(name, t, fmt, rows, cols, count=1, stride=0):
+            # `count` matrices of rows x cols in fmt, `stride` bytes apart, must lie inside t
+            nb = bqg_weight_bytes(fmt, rows, cols)
+            if nb == 0:
+                return  # invalid shape or format: the library's own checks report it
+            if count > 1 and stride < nb:
+                raise ValueError(f"{name}: stride {stride} is smaller than one matrix ({nb} bytes)")
+            if t.numel() * t.element_size() < (count - 1) * stride + nb:
+                raise ValueError(f"{name}: {t.numel() * t.element_size()} bytes, "
+                                 f"{count} matrices need {(count - 1) * stride + nb}")
+        need("gate", gate, expert_fmt, inter, hidden, n_experts, gate_stride)
+        need("up", up, expert_fmt, inter, hidden, n_experts, up_stride)
+        need("down", down, expert_fmt, hidden, inter, n_experts, down_stride)
         c = MoELayerC()
         c.n_experts, c.top_k, c.hidden, c.inter = n_experts, top_k, hidden, inter
         c.expert_fmt, c.act = expert_fmt, act
@@ -237,6 +261,9 @@ class MoELayer:
         c.gate_stride, c.up_stride, c.down_stride = gate_stride, up_stride, down_stride
         if shared is not None:
             sfmt, sinter, sg, su, sd = shared
+            need("shared gate", sg, sfmt, sinter, hidden)
+            need("shared up", su, sfmt, sinter, hidden)
+            need("shared down", sd, sfmt, hidden, sinter)
             self.tensors += [sg, su, sd]
             c.shared_inter, c.shared_fmt = sinter, sfmt
             c.s_gate, c.s_up, c.s_down = sg.data_ptr(), su.data_ptr(), sd.data_ptr()
@@ -248,15 +275,26 @@ def moe_workspace_size(layer: MoELayer, tokens: int) -> int:
     return int(lib().moe_workspace_size(ctypes.byref(layer.c), tokens))
 
 
+def _moe_tokens(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, y: torch.Tensor) -> int:
+    tokens = x.numel() // layer.hidden
+    if tokens < 1 or x.numel() != tokens * layer.hidden:
+        raise ValueError(f"x must hold whole tokens of hidden = {layer.hidden} values")
+    if idx.numel() < tokens * layer.top_k or w.numel() < tokens * layer.top_k:
+        raise ValueError(f"idx and w must hold tokens x top_k = {tokens} x {layer.top_k} values")
+    if y.numel() < tokens * layer.hidden:
+        raise ValueError(f"y must hold tokens x hidden = {tokens} x {layer.hidden} values")
+    return tokens
+
+
 def moe_forward(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor,
                 y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     _need_cuda("x", x, torch.float32)
     _need_cuda("idx", idx, torch.int32)
     _need_cuda("w", w, torch.float32)
-    tokens = x.numel() // layer.hidden
     if y is None:
-        y = torch.empty(tokens, layer.hidden, dtype=torch.float32, device=x.device)
+        y = torch.empty(max(x.numel() // layer.hidden, 1), layer.hidden, dtype=torch.float32, device=x.device)
     _need_cuda("y", y, torch.float32)
+    tokens = _moe_tokens(layer, x, idx, w, y)
     need = moe_workspace_size(layer, tokens)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
@@ -278,7 +316,7 @@ def moe_forward_noalloc(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: 
     _need_cuda("idx", idx, torch.int32)
     _need_cuda("w", w, torch.float32)
     _need_cuda("y", y, torch.float32)
-    tokens = x.numel() // layer.hidden
+    tokens = _moe_tokens(layer, x, idx, w, y)
     _check(lib().moe_forward_noalloc(ctypes.byref(layer.c), _ptr(x), _ptr(idx), _ptr(w), _ptr(y), tokens, _stream(x)),
            "moe_forward_noalloc")
     return y

@@ -158,3 +158,22 @@ def test_binding_limits_match_header():
                       ("BQG_MAX_MOE_COLS", bqg.MAX_MOE_COLS)):
         m = re.search(rf"#define {name} (\d+)", text)
         assert m and int(m.group(1)) == val, name
+
+
+def test_moe_layer_binding_rejects_short_tensors():
+    """The binding checks every stacked expert tensor against n_experts x stride before any
+    pointer reaches the library (the C ABI cannot see buffer sizes)."""
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    from tests.moe_util import device_layer
+    spec = wl.MoESpec("abi_small", 4, 2, 64, 32, bqg.Q4_0, bqg.ACT_GELU_TANH, 32, bqg.Q8_0, False)
+    T = wl.build_moe_layer(spec, 0, device="cpu")
+    device_layer(T)  # the builder's layout passes
+    with pytest.raises(ValueError):
+        bqg.MoELayer(4, 2, 64, 32, bqg.Q4_0, 1, T.gate[:-1], T.up, T.down, T.gate_stride, T.up_stride, T.down_stride)
+    with pytest.raises(ValueError):  # stride below one matrix
+        bqg.MoELayer(4, 2, 64, 32, bqg.Q4_0, 1, T.gate, T.up, T.down, T.gate_stride - 16, T.up_stride, T.down_stride)
+    short_shared = (bqg.Q8_0, 32, T.shared[0], T.shared[1], T.shared[2][:-2])
+    with pytest.raises(ValueError):
+        bqg.MoELayer(4, 2, 64, 32, bqg.Q4_0, 1, T.gate, T.up, T.down, T.gate_stride, T.up_stride, T.down_stride,
+                     short_shared)

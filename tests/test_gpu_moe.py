@@ -161,3 +161,21 @@ def test_glm_like_stack_full_size():
     del layers
     torch.cuda.empty_cache()
     assert bqg.bqg_device_errors() == 0
+
+
+def test_binding_rejects_short_buffers():
+    """x, idx, w and y smaller than tokens x (hidden, top_k) are refused before any launch."""
+    need_gpu()
+    spec = SMALL[0]
+    lay = device_layer(wl.build_moe_layer(spec, 0, 0, device="cuda"))
+    x = torch.zeros(3, spec.hidden, device="cuda")
+    idx = torch.zeros(3, spec.top_k, dtype=torch.int32, device="cuda")
+    w = torch.zeros(3, spec.top_k, device="cuda")
+    with pytest.raises(ValueError):
+        bqg.moe_forward(lay, x.view(-1)[:-1], idx, w)
+    with pytest.raises(ValueError):
+        bqg.moe_forward(lay, x, idx[:2], w)
+    with pytest.raises(ValueError):
+        bqg.moe_forward(lay, x, idx, w, torch.empty(2, spec.hidden, device="cuda"))
+    with pytest.raises(ValueError):
+        bqg.moe_forward_noalloc(lay, x, idx, w[:1], torch.empty(3, spec.hidden, device="cuda"))

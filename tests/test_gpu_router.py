@@ -63,3 +63,18 @@ def test_topk_weights_sum_to_one():
     _, w = bqg.moe_router_topk(lg, 8)
     assert torch.allclose(w.sum(dim=1), torch.ones(512, device="cuda"), atol=1e-6)
     assert bool((w[:, :-1] >= w[:, 1:]).all())
+
+
+def test_binding_rejects_short_buffers():
+    """Buffers smaller than the shape needs are refused by the binding before any launch."""
+    need_gpu()
+    R = torch.zeros(8, 64, device="cuda")
+    with pytest.raises(ValueError):  # not a whole number of tokens
+        bqg.moe_router_logits(R, torch.zeros(100, device="cuda"))
+    with pytest.raises(ValueError):
+        bqg.moe_router_logits(R, torch.zeros(3, 64, device="cuda"), torch.empty(3, 7, device="cuda"))
+    lg = torch.zeros(3, 8, device="cuda")
+    with pytest.raises(ValueError):
+        bqg.moe_router_topk(lg, 2, torch.empty(3, 1, dtype=torch.int32, device="cuda"))
+    with pytest.raises(ValueError):
+        bqg.moe_router_topk(lg, 2, None, torch.empty(5, device="cuda"))
