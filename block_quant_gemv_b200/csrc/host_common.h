@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 #include <utility>
 
 #include "bqg.h"
@@ -19,22 +20,32 @@ struct DeviceInfo {
   int sm_count = 0;
   int cc_major = 0;
   int cc_minor = 0;
-  bool ready = false;
+  std::atomic<bool> ready{false};  // the fields above are set (written once, under g_device_mutex)
 };
 
 inline DeviceInfo g_devices[kMaxDevices];
+inline std::mutex g_device_mutex;
 
-// Attributes of the current device (queried once per device).  Returns BQG_OK,
-// BQG_ERR_CUDA or BQG_ERR_DEVICE (not compute capability 10.0).
+// Attributes of the current device (queried once per device; calls from several host threads
+// are safe, and a failed query is retried by the next call).  Returns BQG_OK, BQG_ERR_CUDA or
+// BQG_ERR_DEVICE (not compute capability 10.0).
 inline int current_device(int* dev_out, DeviceInfo** info) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BQG_ERR_CUDA;
   DeviceInfo& d = g_devices[dev];
-  if (!d.ready) {
-    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BQG_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return BQG_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return BQG_ERR_CUDA;
-    d.ready = true;
+  if (!d.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_device_mutex);
+    if (!d.ready.load(std::memory_order_relaxed)) {
+      int sm = 0, major = 0, minor = 0;
+      if (cudaDeviceGetAttribute(&sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return BQG_ERR_CUDA;
+      d.sm_count = sm;
+      d.cc_major = major;
+      d.cc_minor = minor;
+      d.ready.store(true, std::memory_order_release);
+    }
   }
   if (d.cc_major != 10 || d.cc_minor != 0) return BQG_ERR_DEVICE;
   *dev_out = dev;
