@@ -493,6 +493,9 @@ extern "C" int qgemm_prefill(int fmt, const void* W, const void* X, void* Y, int
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k_prefill_q4, tx, tw, prm) != cudaSuccess) return BQG_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, k_prefill_q4, tx, tw, prm) != cudaSuccess) {
+    (void)cudaGetLastError();  // not left behind for a later call's status check
+    return BQG_ERR_CUDA;
+  }
   return launch_status();
 }
