@@ -151,9 +151,15 @@ class ClockSampler:
                 self.lines = [ln.strip() for ln in out.splitlines() if ln.strip()]
             except (OSError, subprocess.SubprocessError):
                 pass
+        return self.summarize(self.lines)
+
+    @staticmethod
+    def summarize(lines):
+        """Median SM clock, maximum SM clock and the throttle reasons seen in `FIELDS` records
+        (malformed records are skipped)."""
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != 6:
                 continue
