@@ -6,7 +6,8 @@ fallback: if the library is not built, every call raises.
 
 The functions mirror the C ABI in include/bqg.h (same names):
     qgemv, qgemv_batched, qgemm_prefill, moe_router_logits, moe_router_topk,
-    moe_workspace_size, moe_forward, bqg_status_string, bqg_weight_bytes, bqg_device_errors
+    moe_workspace_size, moe_forward, moe_forward_noalloc, bqg_status_string, bqg_weight_bytes,
+    bqg_device_errors, bqg_selftest_wait_timeout
 """
 from __future__ import annotations
 
@@ -19,6 +20,7 @@ import torch
 __all__ = [
     "Q8_0", "Q4_0", "I4_ROW", "ACT_GELU_TANH", "ACT_SILU", "BQGError",
     "lib", "library_path", "bqg_status_string", "bqg_weight_bytes", "bqg_device_errors",
+    "bqg_selftest_wait_timeout",
     "qgemv", "qgemv_batched", "GemvBatch", "qgemm_prefill", "moe_router_logits",
     "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward", "moe_forward_noalloc",
 ]
@@ -68,6 +70,7 @@ _SIGNATURES = {
     "moe_workspace_size": (_sz, [ctypes.POINTER(MoELayerC), _i]),
     "moe_forward": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "moe_forward_noalloc": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp]),
+    "bqg_selftest_wait_timeout": (_i, [_vp]),
 }
 
 
@@ -106,6 +109,13 @@ def bqg_device_errors() -> int:
     bits = _i(0)
     _check(lib().bqg_device_errors(ctypes.byref(bits)), "bqg_device_errors")
     return int(bits.value)
+
+
+def bqg_selftest_wait_timeout() -> None:
+    """Launches the failure-detection self-test on the current device: one wait that nothing
+    completes gives up after its bound (2 s) and sets DEVERR_TIMEOUT (read it with
+    bqg_device_errors)."""
+    _check(lib().bqg_selftest_wait_timeout(_vp(torch.cuda.current_stream().cuda_stream)), "bqg_selftest_wait_timeout")
 
 
 def _check(status: int, what: str):

@@ -8,12 +8,14 @@
 //   router.cuh       router logits and softmax/top-k/renormalise kernels + entry points
 //   moe.cuh          grouped MoE layer kernels + moe_forward
 //   prefill.cuh      tcgen05 prefill-chunk GEMM + qgemm_prefill
+//   selftest.cuh     failure-detection self-test (a bounded wait that runs out)
 #include "common.cuh"
 #include "host_common.h"
 #include "qgemv_api.cuh"
 #include "router.cuh"
 #include "moe_api.cuh"
 #include "prefill.cuh"
+#include "selftest.cuh"
 
 extern "C" const char* bqg_status_string(int status) {
   switch (status) {

@@ -228,6 +228,15 @@ BQG_API int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* i
 BQG_API int moe_forward_noalloc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
                                 float* y, int tokens, void* stream);
 
+/* ---------------------------------------------------------------- failure-detection self-test
+ * bqg_selftest_wait_timeout: launches one kernel (one CTA) whose single mbarrier wait nothing
+ * completes.  The wait is the bounded wait every kernel of the library uses: after 2 s it gives
+ * up, sets BQG_DEVERR_TIMEOUT in the device error word and the kernel returns, so the context
+ * stays usable.  Read (and clear) the bit with bqg_device_errors.  The pages describe no such
+ * call; it shows that a stuck pipeline ends with a status instead of a hang.
+ *   stream  CUDA stream (NULL: the default stream).  Returns BQG_OK once launched. */
+BQG_API int bqg_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

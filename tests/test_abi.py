@@ -32,7 +32,7 @@ def test_header_declares_the_api():
     names = declared_functions()
     for want in ["qgemv", "qgemv_batched", "qgemm_prefill", "moe_router_logits", "moe_router_topk",
                  "moe_workspace_size", "moe_forward", "moe_forward_noalloc", "bqg_status_string", "bqg_weight_bytes",
-                 "bqg_device_errors", "bqg_version"]:
+                 "bqg_device_errors", "bqg_version", "bqg_selftest_wait_timeout"]:
         assert want in names
 
 
