@@ -80,7 +80,9 @@ enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 #define BQG_DEVERR_TIMEOUT 0x1   /* a bounded in-kernel wait gave up (the kernel returned early) */
 #define BQG_DEVERR_EXPERT_ID 0x2 /* moe_forward met an expert id outside [0, n_experts); skipped */
 
-/* Human-readable name of a bqg_status value (static string, never NULL). */
+/* Human-readable name of a bqg_status value (static string, never NULL).
+ *   Source: Camelid README, "Why" and "At a glance" (the engine fails closed with typed errors
+ *   instead of guessing); every call here returns one of the bqg_status values above. */
 BQG_API const char* bqg_status_string(int status);
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -188,7 +190,12 @@ typedef struct {
   const void* s_down;
 } bqg_moe_layer;
 
-/* Bytes of device workspace moe_forward needs for `tokens` tokens (0 on invalid arguments). */
+/* Bytes of device workspace moe_forward needs for `tokens` tokens (0 on invalid arguments).
+ *   Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (tokens are grouped by expert so that
+ *   each expert read serves every row routed to it): the workspace holds that grouping (counts,
+ *   offsets, the permutation of the (token, slot) pairs) and the per-pair intermediate rows.
+ *   The caller allocates it once (PyTorch allocator or cudaMalloc) and may reuse it for every
+ *   call with at most `tokens` tokens; its contents are scratch. */
 BQG_API size_t moe_workspace_size(const bqg_moe_layer* L, int tokens);
 
 /* moe_forward: y[t] = sum_{j<k} w[t, j] * FFN_{idx[t, j]}(x[t]) (+ shared FFN(x[t])), where

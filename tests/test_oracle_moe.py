@@ -109,6 +109,19 @@ def test_gelu_tanh_properties():
     assert abs(om.gelu_tanh(20.0) - 20.0) < 1e-12 and abs(om.gelu_tanh(-20.0)) < 1e-12
 
 
+def test_gelu_tanh_matches_library_routine():
+    """The tanh form against an independent implementation of the same formula: PyTorch's
+    gelu(approximate="tanh") evaluated in float64.  A slip in the cubic coefficient or in
+    sqrt(2/pi) (which the properties above cannot see) moves the values by far more than 1e-12."""
+    import torch
+    g = np.concatenate([np.linspace(-8, 8, 4001), [-3.3, -1e-3, 1e-3, 0.7, 2.5]])
+    ref = torch.nn.functional.gelu(torch.from_numpy(g), approximate="tanh").numpy()
+    np.testing.assert_allclose(om.gelu_tanh(g), ref, rtol=0, atol=1e-12)
+    # a plausible typo of the coefficient is caught at this tolerance
+    bad = 0.5 * g * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (g + 0.0447 * g ** 3)))
+    assert np.max(np.abs(bad - ref)) > 1e-6
+
+
 def test_silu_properties():
     g = np.linspace(-10, 10, 1001)
     s = om.silu(g)
