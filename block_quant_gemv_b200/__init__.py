@@ -19,6 +19,7 @@ import torch
 
 __all__ = [
     "Q8_0", "Q4_0", "I4_ROW", "ACT_GELU_TANH", "ACT_SILU", "BQGError",
+    "MOE_PATH_AUTO", "MOE_PATH_CUDA_CORES", "MOE_PATH_TENSOR_CORES",
     "lib", "library_path", "bqg_status_string", "bqg_weight_bytes", "bqg_device_errors",
     "bqg_selftest_wait_timeout",
     "qgemv", "qgemv_batched", "GemvBatch", "qgemm_prefill", "moe_router_logits",
@@ -27,6 +28,8 @@ __all__ = [
 
 Q8_0, Q4_0, I4_ROW = 1, 2, 3
 ACT_GELU_TANH, ACT_SILU = 1, 2
+MOE_PATH_AUTO, MOE_PATH_CUDA_CORES, MOE_PATH_TENSOR_CORES = 0, 1, 2
+MOE_TC_MIN_TOKENS = 16
 MAX_COLS, MAX_BATCH, MAX_EXPERTS, MAX_TOPK, MAX_MOE_COLS = 15360, 256, 256, 8, 7168
 DEVERR_TIMEOUT, DEVERR_EXPERT_ID = 0x1, 0x2
 
@@ -54,7 +57,7 @@ class MoELayerC(ctypes.Structure):
                 ("gate", _vp), ("up", _vp), ("down", _vp),
                 ("gate_stride", _sz), ("up_stride", _sz), ("down_stride", _sz),
                 ("shared_inter", _i), ("shared_fmt", _i),
-                ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp)]
+                ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp), ("path", _i)]
 
 
 _SIGNATURES = {
@@ -248,7 +251,7 @@ class MoELayer:
 
     def __init__(self, n_experts: int, top_k: int, hidden: int, inter: int, expert_fmt: int, act: int,
                  gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor,
-                 gate_stride: int, up_stride: int, down_stride: int, shared=None):
+                 gate_stride: int, up_stride: int, down_stride: int, shared=None, path: int = 0):
         self.tensors = [gate, up, down]
 
         def need(name, t, fmt, rows, cols, count=1, stride=0):
@@ -277,8 +280,19 @@ class MoELayer:
             self.tensors += [sg, su, sd]
             c.shared_inter, c.shared_fmt = sinter, sfmt
             c.s_gate, c.s_up, c.s_down = sg.data_ptr(), su.data_ptr(), sd.data_ptr()
+        c.path = path
         self.c = c
         self.hidden, self.top_k, self.n_experts = hidden, top_k, n_experts
+
+    def with_path(self, path: int) -> "MoELayer":
+        """The same layer (same tensors) with another expert path (MOE_PATH_*)."""
+        other = object.__new__(MoELayer)
+        other.__dict__.update(self.__dict__)
+        c = MoELayerC()
+        ctypes.memmove(ctypes.byref(c), ctypes.byref(self.c), ctypes.sizeof(c))
+        c.path = path
+        other.c = c
+        return other
 
 
 def moe_workspace_size(layer: MoELayer, tokens: int) -> int:
@@ -314,7 +328,7 @@ def moe_forward(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Te
     return y
 
 
-NOALLOC_SCRATCH_BYTES = 24 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def moe_forward_noalloc(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor,

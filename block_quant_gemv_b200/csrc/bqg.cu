@@ -56,9 +56,42 @@ extern "C" int bqg_device_errors(int* bits) {
 static __device__ __align__(256) uint8_t g_moe_noalloc_scratch[BQG_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-// Device address of g_moe_noalloc_scratch per device.  In host code the array's name is only a
-// host-side stand-in, so the address must be asked from the runtime (once per device).
-std::atomic<void*> g_noalloc_scratch_ptr[bqg::kMaxDevices];
+// Device address of g_moe_noalloc_scratch per device, with the id of the CUDA context it was
+// looked up in.  In host code the array's name is only a host-side stand-in, so the address is
+// asked from the runtime with that device current: once per device (the first call), and again
+// only if the device's context has been destroyed and re-created since (the module, and with it
+// the array, may then sit at another address).
+struct NoallocScratch {
+  std::atomic<void*> ptr{nullptr};
+  std::atomic<unsigned long long> ctx{0};
+};
+NoallocScratch g_noalloc_scratch[bqg::kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (false if the driver cannot tell).
+bool current_context_id(unsigned long long* id) {
+  static std::atomic<CtxGetCurrentFn> get_current{nullptr};
+  static std::atomic<CtxGetIdFn> get_id{nullptr};
+  CtxGetCurrentFn fc = get_current.load(std::memory_order_acquire);
+  CtxGetIdFn fi = get_id.load(std::memory_order_acquire);
+  if (fc == nullptr || fi == nullptr) {
+    void* p1 = nullptr;
+    void* p2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || p1 == nullptr || p2 == nullptr)
+      return false;
+    fc = reinterpret_cast<CtxGetCurrentFn>(p1);
+    fi = reinterpret_cast<CtxGetIdFn>(p2);
+    get_current.store(fc, std::memory_order_release);
+    get_id.store(fi, std::memory_order_release);
+  }
+  CUcontext c = nullptr;
+  return fc(&c) == CUDA_SUCCESS && c != nullptr && fi(c, id) == CUDA_SUCCESS;
+}
 }  // namespace
 
 extern "C" int moe_forward_noalloc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
@@ -71,12 +104,17 @@ extern "C" int moe_forward_noalloc(const bqg_moe_layer* L, const float* x, const
   if (need > size_t(BQG_NOALLOC_SCRATCH_BYTES)) return BQG_ERR_LIMIT;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= bqg::kMaxDevices) return BQG_ERR_CUDA;
-  void* scratch = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (scratch == nullptr) {
-    // first call on this device: look the array up with this device current
+  NoallocScratch& slot = g_noalloc_scratch[dev];
+  // The first call on a device (and the first after its context was re-created) does the
+  // set-up: make it before any stream capture that includes the call.
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  void* scratch = slot.ptr.load(std::memory_order_acquire);
+  if (scratch == nullptr || (have_ctx && slot.ctx.load(std::memory_order_acquire) != ctx)) {
     if (cudaGetSymbolAddress(&scratch, g_moe_noalloc_scratch) != cudaSuccess || scratch == nullptr)
       return BQG_ERR_CUDA;
-    g_noalloc_scratch_ptr[dev].store(scratch, std::memory_order_release);
+    slot.ctx.store(ctx, std::memory_order_release);
+    slot.ptr.store(scratch, std::memory_order_release);
   }
   // Every region of the scratch is written by the kernels before it is read, so nothing has to
   // be cleared between calls.

@@ -3,6 +3,7 @@
 
 #include "host_common.h"
 #include "moe.cuh"
+#include "moe_tc.cuh"
 #include "qgemv_api.cuh"
 
 namespace bqg {
@@ -103,6 +104,89 @@ inline MoeWsLayout moe_ws_layout(const bqg_moe_layer* L, int tokens) {
   return o;
 }
 
+// Workspace of the tensor-core path: the same routing tables, then fp16 activation rows (x in
+// expert-grouped order, x of the shared expert in token order, the gated hidden rows h) and the
+// fp32 per-pair and shared outputs that the combine sums.
+struct MoeTcLayout {
+  size_t counts, offsets, active, n_active, ctr, act_info, perm;
+  size_t xg, xs, hg, hs, part, sout, total;
+};
+
+inline MoeTcLayout moe_ws_layout_tc(const bqg_moe_layer* L, int tokens) {
+  MoeTcLayout o{};
+  const size_t E = size_t(L->n_experts), T = size_t(tokens), pairs = T * L->top_k;
+  const bool sh = L->s_gate != nullptr;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  o.counts = take(4 * E);
+  o.offsets = take(4 * (E + 1));
+  o.active = take(4 * E);
+  o.n_active = take(4);
+  o.ctr = take(8);
+  o.act_info = take(16 * E);
+  o.perm = take(4 * pairs);
+  o.xg = take(2 * pairs * L->hidden);
+  o.xs = sh ? take(2 * T * L->hidden) : 0;
+  o.hg = take(2 * pairs * L->inter);
+  o.hs = sh ? take(2 * T * L->shared_inter) : 0;
+  o.part = take(4 * pairs * L->hidden);
+  o.sout = sh ? take(4 * T * L->hidden) : 0;
+  o.total = off;
+  return o;
+}
+
+// The families of a layer on the tensor-core path; false when a shape does not fit it.
+struct TcLayer {
+  TcFam gate, up, down0, down1, s_gate, s_up, s_down0, s_down1;
+};
+
+inline bool tc_layer(const bqg_moe_layer* L, TcLayer* T) {
+  TcLayer t{};
+  if (!tc_fam(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden, 0, &t.gate) ||
+      !tc_fam(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden, 0, &t.up) ||
+      !tc_fam(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, 0, &t.down0) ||
+      !tc_fam(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, 128, &t.down1))
+    return false;
+  if (L->s_gate != nullptr) {
+    if (!tc_fam(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden, 0, &t.s_gate) ||
+        !tc_fam(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden, 0, &t.s_up) ||
+        !tc_fam(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, 0, &t.s_down0) ||
+        !tc_fam(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, 128, &t.s_down1))
+      return false;
+  }
+  if (T != nullptr) *T = t;
+  return true;
+}
+
+// Path for `tokens` tokens: BQG_MOE_PATH_CUDA_CORES or BQG_MOE_PATH_TENSOR_CORES (negative: error).
+inline int moe_path(const bqg_moe_layer* L, int tokens) {
+  if (L->path == BQG_MOE_PATH_CUDA_CORES) return BQG_MOE_PATH_CUDA_CORES;
+  const bool tc = tc_layer(L, nullptr);
+  if (L->path == BQG_MOE_PATH_TENSOR_CORES) return tc ? int(BQG_MOE_PATH_TENSOR_CORES) : int(BQG_ERR_SHAPE);
+  return (tc && tokens >= BQG_MOE_TC_MIN_TOKENS) ? BQG_MOE_PATH_TENSOR_CORES : BQG_MOE_PATH_CUDA_CORES;
+}
+
+// Workspace for every call of up to `tokens` tokens (each path's layout grows with the tokens;
+// with the automatic choice, fewer tokens may take the other path).
+inline size_t moe_ws_total(const bqg_moe_layer* L, int tokens) {
+  const int path = moe_path(L, tokens);
+  if (path < 0) return 0;
+  if (path == BQG_MOE_PATH_CUDA_CORES) return moe_ws_layout(L, tokens).total;
+  size_t need = moe_ws_layout_tc(L, tokens).total;
+  if (L->path == BQG_MOE_PATH_AUTO) {
+    const int below = tokens < BQG_MOE_TC_MIN_TOKENS ? tokens : BQG_MOE_TC_MIN_TOKENS - 1;
+    if (below >= 1) {
+      const size_t cc = moe_ws_layout(L, below).total;
+      if (cc > need) need = cc;
+    }
+  }
+  return need;
+}
+
 inline bool valid_fmt(int f) { return f == BQG_Q8_0 || f == BQG_Q4_0 || f == BQG_I4_ROW; }
 
 inline int check_layer(const bqg_moe_layer* L) {
@@ -112,6 +196,8 @@ inline int check_layer(const bqg_moe_layer* L) {
   if (L->top_k > L->n_experts) return BQG_ERR_SHAPE;
   if (!valid_fmt(L->expert_fmt)) return BQG_ERR_FMT;
   if (L->act != BQG_ACT_GELU_TANH && L->act != BQG_ACT_SILU) return BQG_ERR_ARG;
+  if (L->path != BQG_MOE_PATH_AUTO && L->path != BQG_MOE_PATH_CUDA_CORES && L->path != BQG_MOE_PATH_TENSOR_CORES)
+    return BQG_ERR_ARG;
   if (L->hidden % 32 || L->inter % 32) return BQG_ERR_SHAPE;
   if (L->hidden > kMoeMaxCols || L->inter > kMoeMaxCols) return BQG_ERR_LIMIT;
   if (L->gate == nullptr || L->up == nullptr || L->down == nullptr) return BQG_ERR_ARG;
@@ -144,11 +230,119 @@ inline int quant_grid(long long threads, int cap) {
   return int(g);
 }
 
+// One grouped-GEMM launch (phase 0 gate/up, 1 down) of the tensor-core path.
+inline int launch_moe_tc(const bqg_moe_layer* L, const TcLayer& TL, int phase, int tokens, const RouteWs& route,
+                         const __half* b_routed, const __half* b_shared, __half* h_routed, __half* h_shared,
+                         float* part, float* sout, int dev, const DeviceInfo* info, cudaStream_t s) {
+  const bool sh = L->s_gate != nullptr;
+  const int pairs = tokens * L->top_k;
+  TcParams P{};
+  int st;
+  if (phase == 0) {
+    P.fam[0] = TL.gate;
+    P.fam[1] = TL.up;
+    P.fam[2] = sh ? TL.s_gate : TL.gate;
+    P.fam[3] = sh ? TL.s_up : TL.up;
+  } else {
+    P.fam[0] = TL.down0;
+    P.fam[1] = TL.down1;
+    P.fam[2] = sh ? TL.s_down0 : TL.down0;
+    P.fam[3] = sh ? TL.s_down1 : TL.down1;
+  }
+  for (int i = 0; i < 4; ++i) {
+    const int ne = i < 2 ? L->n_experts : (sh ? 1 : L->n_experts);
+    if ((st = tc_encode_amap(&P.amap[i], P.fam[i], ne)) != BQG_OK) return st;
+  }
+  const int kb = phase == 0 ? L->hidden : L->inter;
+  const int kbs = phase == 0 ? L->hidden : L->shared_inter;
+  if ((st = tc_encode_bmap(&P.bmap[0], b_routed, pairs, kb)) != BQG_OK) return st;
+  if (sh) {
+    if ((st = tc_encode_bmap(&P.bmap[1], b_shared, tokens, kbs)) != BQG_OK) return st;
+  } else {
+    P.bmap[1] = P.bmap[0];
+  }
+  P.phase = phase;
+  P.act = L->act;
+  P.tokens = tokens;
+  P.has_shared = sh ? 1 : 0;
+  P.tiles_r = phase == 0 ? (L->inter + 127) / 128 : (L->hidden + 255) / 256;
+  P.tiles_s = phase == 0 ? (L->shared_inter + 127) / 128 : (L->hidden + 255) / 256;
+  int win = 0;
+  for (int i = 0; i < 4; ++i) win = P.fam[i].win > win ? P.fam[i].win : win;
+  tc_raw_ring(win, &P.raw_stages, &P.raw_stage_bytes);
+  P.act_info = route.act_info;
+  P.n_active = route.n_active;
+  P.perm = route.perm;
+  P.ctr = route.ctr + phase;
+  P.hout[0] = h_routed;
+  P.hout[1] = h_shared;
+  P.hstride[0] = L->inter;
+  P.hstride[1] = L->shared_inter;
+  P.hperm[0] = L->expert_fmt != BQG_Q8_0;
+  P.hperm[1] = sh && L->shared_fmt != BQG_Q8_0;
+  P.yout[0] = part;
+  P.yout[1] = sout;
+  P.ystride = L->hidden;
+  if ((st = g_tc_attr.ensure(dev, k_moe_tc, kTcMaxSmem)) != BQG_OK) return st;
+  return launch_pdl(k_moe_tc, dim3(info->sm_count), dim3(kTcThreads), tc_smem_bytes(P.raw_stages, P.raw_stage_bytes),
+                    s, P);
+}
+
+}  // namespace bqg
+
+namespace bqg {
+// The layer on the tensor-core path: route grouping (one block), fp16 activation rows, the
+// grouped gate/up GEMM with act(g) * u in its epilogue, the grouped down GEMM, the combine.
+inline int moe_forward_tc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
+                          int tokens, uint8_t* ws, int dev, const DeviceInfo* info, cudaStream_t s) {
+  TcLayer TL;
+  if (!tc_layer(L, &TL)) return BQG_ERR_SHAPE;
+  const MoeTcLayout lay = moe_ws_layout_tc(L, tokens);
+  const bool sh = L->s_gate != nullptr;
+  const int pairs = tokens * L->top_k;
+  RouteWs route;
+  route.counts = reinterpret_cast<int32_t*>(ws + lay.counts);
+  route.offsets = reinterpret_cast<int32_t*>(ws + lay.offsets);
+  route.active = reinterpret_cast<int32_t*>(ws + lay.active);
+  route.n_active = reinterpret_cast<int32_t*>(ws + lay.n_active);
+  route.perm = reinterpret_cast<int32_t*>(ws + lay.perm);
+  route.ctr = reinterpret_cast<uint32_t*>(ws + lay.ctr);
+  route.act_info = reinterpret_cast<int4*>(ws + lay.act_info);
+  auto H = [&](size_t o) { return reinterpret_cast<__half*>(ws + o); };
+  auto F = [&](size_t o) { return reinterpret_cast<float*>(ws + o); };
+  int st;
+  // 1. route grouping
+  QuantJobs none{};
+  none.n = 0;
+  if ((st = launch_pdl(k_moe_prep, dim3(1), dim3(kRouteThreads), 0, s, idx, pairs, L->n_experts, route, none)) !=
+      BQG_OK)
+    return st;
+  // 2. activation rows in fp16 (grouped order for the routed experts, token order for the shared one)
+  const long long chunks = (long long)(pairs + (sh ? tokens : 0)) * (L->hidden / 8);
+  if ((st = launch_pdl(k_moe_xprep, dim3(quant_grid(chunks, 4 * info->sm_count)), dim3(256), 0, s, x,
+                       (const int32_t*)route.perm, (const int32_t*)route.offsets, L->n_experts, L->top_k, tokens,
+                       L->hidden, H(lay.xg), int(L->expert_fmt != BQG_Q8_0), sh ? H(lay.xs) : (__half*)nullptr,
+                       int(sh && L->shared_fmt != BQG_Q8_0))) != BQG_OK)
+    return st;
+  // 3. gate/up with h = act(g) * u in the epilogue
+  if ((st = launch_moe_tc(L, TL, 0, tokens, route, H(lay.xg), sh ? H(lay.xs) : nullptr, H(lay.hg),
+                          sh ? H(lay.hs) : nullptr, nullptr, nullptr, dev, info, s)) != BQG_OK)
+    return st;
+  // 4. down
+  if ((st = launch_moe_tc(L, TL, 1, tokens, route, H(lay.hg), sh ? H(lay.hs) : nullptr, nullptr, nullptr, F(lay.part),
+                          sh ? F(lay.sout) : nullptr, dev, info, s)) != BQG_OK)
+    return st;
+  // 5. combine
+  const long long n = (long long)tokens * L->hidden;
+  return launch_pdl(k_moe_combine, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s, (const float*)F(lay.part), idx, w,
+                    sh ? (const float*)F(lay.sout) : (const float*)nullptr, y, tokens, L->top_k, L->hidden,
+                    L->n_experts);
+}
 }  // namespace bqg
 
 extern "C" size_t moe_workspace_size(const bqg_moe_layer* L, int tokens) {
   if (bqg::check_layer(L) != BQG_OK || tokens < 1) return 0;
-  return bqg::moe_ws_layout(L, tokens).total;
+  return bqg::moe_ws_total(L, tokens);
 }
 
 extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
@@ -159,8 +353,9 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   if (x == nullptr || idx == nullptr || w == nullptr || y == nullptr || tokens < 1) return BQG_ERR_ARG;
   if ((long long)tokens * L->top_k > (1 << 24)) return BQG_ERR_LIMIT;
   if (!aligned(x, 16) || !aligned(y, 16) || !aligned(idx, 4) || !aligned(w, 4)) return BQG_ERR_ALIGN;
-  const MoeWsLayout lay = moe_ws_layout(L, tokens);
-  if (workspace == nullptr || ws_bytes < lay.total) return BQG_ERR_WORKSPACE;
+  const int path = moe_path(L, tokens);
+  if (path < 0) return path;
+  if (workspace == nullptr || ws_bytes < moe_ws_total(L, tokens)) return BQG_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return BQG_ERR_ALIGN;
   int dev;
   DeviceInfo* info;
@@ -168,6 +363,8 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   if (st != BQG_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (path == BQG_MOE_PATH_TENSOR_CORES) return moe_forward_tc(L, x, idx, w, y, tokens, ws, dev, info, s);
+  const MoeWsLayout lay = moe_ws_layout(L, tokens);
   auto F = [&](size_t o) { return reinterpret_cast<float*>(ws + o); };
   auto R = [&](size_t o) { return reinterpret_cast<uint4*>(ws + o); };
   const bool sh = L->s_gate != nullptr;

@@ -1,0 +1,703 @@
+// Grouped expert GEMM of the MoE layer on the 5th-generation tensor cores (tcgen05), for steps
+// with many tokens (a prefill chunk, or a decode batch whose experts each serve several tokens):
+//   gate/up phase:  h[p, i] = act(G_e[i, :] x_t) * (U_e[i, :] x_t)   for every routed pair p = (t, j)
+//   down phase:     out[p, c] = D_e[c, :] h[p, :]
+// and the same for the shared expert over all tokens.
+//
+// Sources: TurboFieldfare wiki, "메모리·전문가 스트리밍" (prefill in chunks of at most 128 tokens;
+// each expert read serves every row routed to it; routed experts split from the dense shared
+// branch); Camelid README, "Gemma 4" (GeGLU experts; dense shared expert + sparse top-8 branch).
+//
+// One work item = up to 64 tokens of one expert (or of the shared expert) times two 128-row
+// weight tiles: the gate and up tiles of the same rows (gate/up phase), or two consecutive
+// tiles of the down matrix (down phase).  Weight rows sit on the MMA's M side (128), the item's
+// tokens on N (16..64, padded to 16), k along the matrix columns.  Each CTA (one per SM) runs
+// items claimed from a counter, with warp-specialised roles:
+//   warp 0      TMA: raw weight chunks (128 rows x 128 or 64 k of each tile, in their block
+//               format) through a ring in shared memory.  A 3-D tensor map with 8-byte elements
+//               views each family as [expert][super-row][bytes], a super-row being g = 1, 2 or 4
+//               consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of 704
+//               values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
+//   warp 14     TMA: the item's activation rows (fp16, 128-byte swizzle, k-major) per 64-k stage.
+//   warps 2-9   dequantize: thread (tile f, row r) turns its row's 64 weights of a stage into fp16
+//               and stores them with tcgen05.st straight into TENSOR MEMORY (lane r), where the
+//               MMA reads its A operand.  Keeping A out of shared memory matters: 4-bit weights
+//               expanded to fp16 in shared memory would cost ~4 bytes of shared-memory traffic
+//               per weight (store + MMA read), more than the SM moves at the HBM rate.
+//   warp 1      allocates all 512 tensor-memory columns and issues tcgen05.mma (kind::f16, A from
+//               tensor memory, B from shared memory, fp32 accumulation): 4 A stages of 2 x 32
+//               columns, and two accumulator buffers of 2 x 64 columns, so the epilogue of one
+//               item overlaps the MMAs of the next.
+//   warps 10-13 epilogue: read the accumulators (tcgen05.ld), apply int4 row scales, and write
+//               h = act(g) * u as fp16 (gate/up) or the fp32 per-pair outputs (down).
+//
+// Weights become fp16 exactly as stored values allow: Q4_0 (q - 8) and Q8_0 q exactly via the
+// fp16 exponent-bias identity (0x6400 | byte = 1024 + byte), then one rounding of the product by
+// d; int4 values -8..7 exactly (its row scale is applied to the fp32 accumulator).  Within each
+// group of 8 k, nibble formats store the weights in the order their bytes yield them
+// (elements 0,4,1,5,2,6,3,7); the activation rows are written in the same order, which leaves
+// every dot product unchanged.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "host_common.h"
+#include "moe.cuh"
+#include "tcgen05.cuh"
+
+namespace bqg {
+
+constexpr int kTcThreads = 480;            // 15 warps
+constexpr int kTcWarpRaw = 0, kTcWarpMma = 1, kTcWarpDq = 2, kTcWarpEpi = 10, kTcWarpB = 14;
+constexpr int kTcDqThreads = 256;          // 2 tiles x 128 rows
+constexpr int kTcNMax = 64;                // tokens per item (MMA N <= 64)
+constexpr int kTcAStages = 4;              // A stages in tensor memory
+constexpr int kTcBStages = 4;              // activation stages in shared memory
+constexpr int kTcBStageBytes = kTcNMax * 128;  // 64 rows x 64 k fp16
+constexpr int kTcDescs = 8;                // item descriptor ring
+constexpr int kTcRawMax = 12;              // raw weight ring depth (runtime, by window size)
+constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (A stages use 0..255)
+constexpr int kTcDescReaders = 1 + 1 + 8 + 4;  // B producer, MMA, dequant warps, epilogue warps
+// smem: [1 KB alignment slack][B ring][raw ring][barriers + descriptors]
+constexpr int kTcBarBytes = 1024;
+constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBStages) * kTcBStageBytes + kTcBarBytes;
+constexpr size_t kTcMaxSmem = 227 * 1024;
+static_assert((2 * kTcRawMax + 4 * kTcAStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <= kTcBarBytes,
+              "barrier area");
+
+// One family of stacked matrices as the kernel sees it (rows on M, cols = k).
+struct TcFam {
+  const uint8_t* base;  // expert 0's matrix (the shared expert: its only matrix)
+  long long stride;     // bytes between experts
+  int fmt, rows, cols;
+  int row_bytes;
+  int g;                // rows per super-row of the tensor map
+  int win;              // bytes fetched per row and raw chunk (a 16-byte-aligned window)
+  int cb;               // bytes of one raw chunk of one row
+  int raw_k;            // weights per raw chunk (128, or 64 for Q8_0)
+  int scale_off;        // int4: byte offset of the row scales in one matrix
+  int m_off;            // row offset of this tile inside an item (0, or 128 for the second down tile)
+};
+
+struct alignas(64) TcParams {
+  CUtensorMap amap[4];  // weight maps: 0, 1 routed tiles; 2, 3 shared tiles
+  CUtensorMap bmap[2];  // activation maps: 0 routed (rows in expert-grouped order), 1 shared (token order)
+  TcFam fam[4];
+  int phase;            // 0 gate/up, 1 down
+  int act;
+  int tokens, has_shared;
+  int tiles_r, tiles_s; // items' tile pairs per routed expert / for the shared expert
+  int raw_stages, raw_stage_bytes;
+  const int4* act_info; // per touched expert: (expert, count, offset, first pair)
+  const int32_t* n_active;
+  const int32_t* perm;  // pair ids in expert-grouped order
+  uint32_t* ctr;        // item counter (zeroed by the route kernel)
+  __half* hout[2];      // gate/up: h rows (routed: grouped order; shared: token order)
+  int hstride[2];       // inter, shared_inter
+  int hperm[2];         // 1: the down matrix is a nibble format (store h in nibble order)
+  float* yout[2];       // down: per-pair outputs [pairs][hidden], shared [tokens][hidden]
+  int ystride;          // hidden
+};
+
+// ---------------------------------------------------------------- dequantization of one 64-k stage
+// Four fp16 pairs of the 8 nibbles of word w (element 2m = low nibble of byte m), in the order
+// the bytes yield them: (e0, e4) (e1, e5) (e2, e6) (e3, e7); values (q - 8) * d.
+__device__ __forceinline__ void tc_nib8(uint32_t w, __half2 d2, uint32_t* o) {
+  const __half2 bias = __half2half2(__ushort_as_half(0x6408));  // 1032
+  uint32_t p[4] = {(w & 0x000F000Fu) | 0x64006400u, ((w >> 4) & 0x000F000Fu) | 0x64006400u,
+                   ((w >> 8) & 0x000F000Fu) | 0x64006400u, ((w >> 12) & 0x000F000Fu) | 0x64006400u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)  // (1024 + q) - 1032 = q - 8 exactly; times d rounds once
+    o[i] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p[i]), bias), d2));
+}
+// Same for two's-complement nibbles without a scale: t ^ 8 = t + 8, so (1024 + (t + 8)) - 1032 = t.
+__device__ __forceinline__ void tc_i4nib8(uint32_t w, uint32_t* o) {
+  const __half2 bias = __half2half2(__ushort_as_half(0x6408));
+  w ^= 0x88888888u;
+  uint32_t p[4] = {(w & 0x000F000Fu) | 0x64006400u, ((w >> 4) & 0x000F000Fu) | 0x64006400u,
+                   ((w >> 8) & 0x000F000Fu) | 0x64006400u, ((w >> 12) & 0x000F000Fu) | 0x64006400u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&p[i]), bias));
+}
+// Four int8 values of word w as two fp16 pairs (e0, e1) (e2, e3), values q * d:
+// q ^ 0x80 = q + 128 as an unsigned byte, 0x64 high byte gives 1024 + q + 128, minus 1152 is q.
+__device__ __forceinline__ void tc_q8x4(uint32_t w, __half2 d2, uint32_t* o) {
+  const __half2 bias = __half2half2(__ushort_as_half(0x6480));  // 1152
+  const uint32_t u = w ^ 0x80808080u;
+  uint32_t p0 = __byte_perm(u, 0x64646464u, 0x5140), p1 = __byte_perm(u, 0x64646464u, 0x7362);
+  o[0] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p0), bias), d2));
+  o[1] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p1), bias), d2));
+}
+
+// 64 weights of one row (two blocks, or 64 int4 values) at shared address a as 32 fp16 pairs.
+// Q4_0 and Q8_0: a is 4-byte aligned (the row's blocks start there); int4: 16-byte aligned.
+__device__ __forceinline__ void tc_dequant64(int fmt, uint32_t a, uint32_t (&o)[32]) {
+  if (fmt == BQG_Q4_0) {  // block A: d at bytes 0-1, qs at 2..17; block B: d at 18-19, qs at 20..35
+    uint32_t v[9];
+#pragma unroll
+    for (int i = 0; i < 9; ++i) v[i] = lds32(a + 4 * i);
+    const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
+    const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[4] >> 16)));
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_nib8(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[4 * m]);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_nib8(v[5 + m], dB, &o[16 + 4 * m]);
+  } else if (fmt == BQG_Q8_0) {  // block A: d 0-1, q 2..33; block B: d 34-35, q 36..67
+    uint32_t v[17];
+#pragma unroll
+    for (int i = 0; i < 17; ++i) v[i] = lds32(a + 4 * i);
+    const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
+    const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[8] >> 16)));
+#pragma unroll
+    for (int m = 0; m < 8; ++m) tc_q8x4(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[2 * m]);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) tc_q8x4(v[9 + m], dB, &o[16 + 2 * m]);
+  } else {
+    const uint4 p0 = lds128(a), p1 = lds128(a + 16);
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) tc_i4nib8(w[m], &o[4 * m]);
+  }
+}
+
+// Position of element k inside its activation row: nibble formats hold each group of 8 in
+// the order 0,4,1,5,2,6,3,7, i.e. element i of a group sits at position {0,2,4,6,1,3,5,7}[i].
+__host__ __device__ __forceinline__ int tc_kpos(int k, int nibble) {
+  if (!nibble) return k;
+  const int i = k & 7;
+  return (k & ~7) | ((i & 3) << 1) | (i >> 2);
+}
+
+// ---------------------------------------------------------------- the kernel
+// Item descriptor: d0 = (flags: bit0 shared, bit1 second tile present; expert; m0; tokens),
+//                  d1 = (first activation row; N; first output row; 64-k stages).
+__global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant__ TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_s & 1023)) & 1023);
+  uint8_t* bring = smem;                                            // kTcBStages x 8 KB
+  uint8_t* wring = bring + size_t(kTcBStages) * kTcBStageBytes;    // raw_stages x raw_stage_bytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wring + size_t(P.raw_stages) * P.raw_stage_bytes);
+  uint64_t* raw_full = bars;                        // [kTcRawMax] TMA bytes
+  uint64_t* raw_empty = raw_full + kTcRawMax;       // [kTcRawMax] 256 dequant threads
+  uint64_t* a_full = raw_empty + kTcRawMax;         // [kTcAStages] 256 dequant threads
+  uint64_t* a_empty = a_full + kTcAStages;          // [kTcAStages] MMA commit
+  uint64_t* b_full = a_empty + kTcAStages;          // [kTcBStages] TMA bytes
+  uint64_t* b_empty = b_full + kTcBStages;          // [kTcBStages] MMA commit
+  uint64_t* acc_full = b_empty + kTcBStages;        // [2] MMA commit
+  uint64_t* acc_empty = acc_full + 2;               // [2] 128 epilogue threads
+  uint64_t* d_full = acc_empty + 2;                 // [kTcDescs] producer
+  uint64_t* d_empty = d_full + kTcDescs;            // [kTcDescs] reader warps
+  uint64_t* done = d_empty + kTcDescs;              // final MMA commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int4* descs = reinterpret_cast<int4*>(bars + (kTcBarBytes - kTcDescs * 32) / 8);  // [kTcDescs][2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTcRawMax; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], kTcDqThreads);
+    }
+    for (int i = 0; i < kTcAStages; ++i) {
+      mbar_init(&a_full[i], kTcDqThreads);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < kTcBStages; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 128);
+    }
+    for (int i = 0; i < kTcDescs; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], kTcDescReaders);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kTcWarpRaw && lane == 0) {
+    for (int i = 0; i < 4; ++i) prefetch_tensormap(&P.amap[i]);
+    prefetch_tensormap(&P.bmap[0]);
+    prefetch_tensormap(&P.bmap[1]);
+  }
+  if (warp == kTcWarpMma) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+  griddep_wait();  // routing tables and activation rows come from earlier kernels
+
+  // Readers of the descriptor ring: wait for slot ds, copy, release (lane 0 of each reader warp).
+  // Called by lane 0 of a reader warp only (the other lanes get the values by shuffles).
+  auto read_desc = [&](int ds, int4& d0, int4& d1) -> bool {
+    const int slot = ds % kTcDescs;
+    if (!mbar_wait(&d_full[slot], uint32_t(ds / kTcDescs) & 1u)) {
+      *abort_flag = 1;
+      return false;
+    }
+    d0 = ld_desc(&descs[2 * slot]);
+    d1 = ld_desc(&descs[2 * slot + 1]);
+    mbar_arrive(&d_empty[slot]);
+    return true;
+  };
+
+  if (warp == kTcWarpRaw) {
+    // ------------------------------------------------ item claims + raw weight TMA
+    if (lane == 0) {
+      const int na = *P.n_active;
+      const int nch = (P.tokens + kTcNMax - 1) / kTcNMax;
+      const int n_sh = P.has_shared ? P.tiles_s * nch : 0;
+      const int per_e = P.tiles_r * nch;
+      const int n_items = n_sh + na * per_e;
+      const int tile_rows = P.phase == 0 ? 128 : 256;
+      int ds = 0, rp = 0;
+      bool ok = true;
+      int item = int(atomicAdd(P.ctr, 1u));
+      while (ok) {
+        const int next = item < n_items ? int(atomicAdd(P.ctr, 1u)) : n_items;  // one claim ahead
+        int4 d0, d1;
+        bool end = item >= n_items;
+        if (!end) {
+          int shared, e = 0, t, c, cnt, off;
+          if (item < n_sh) {
+            shared = 1;
+            t = item / nch;
+            c = item - t * nch;
+            cnt = P.tokens;
+            off = 0;
+          } else {
+            shared = 0;
+            const int r = item - n_sh;
+            const int a = r / per_e;
+            const int rem = r - a * per_e;
+            t = rem / nch;
+            c = rem - t * nch;
+            const int4 ai = __ldg(P.act_info + a);
+            e = ai.x;
+            cnt = ai.y;
+            off = ai.z;
+          }
+          const int ntok = min(kTcNMax, cnt - c * kTcNMax);
+          if (ntok <= 0) {  // an empty token chunk of a lightly routed expert
+            item = next;
+            continue;
+          }
+          const int fb = shared ? 2 : 0;
+          const int m0 = t * tile_rows;
+          const int two = (P.phase == 0 || m0 + 128 < P.fam[fb].rows) ? 1 : 0;
+          d0 = make_int4(shared | (two << 1), e, m0, ntok);
+          d1 = make_int4(off + c * kTcNMax, (ntok + 15) & ~15, off + c * kTcNMax, P.fam[fb].cols / 64);
+        } else {
+          d0 = make_int4(-1, 0, 0, 0);
+          d1 = make_int4(0, 0, 0, 0);
+        }
+        const int slot = ds % kTcDescs;
+        if (ds >= kTcDescs && !mbar_wait(&d_empty[slot], uint32_t(ds / kTcDescs - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        descs[2 * slot] = d0;
+        descs[2 * slot + 1] = d1;
+        mbar_arrive(&d_full[slot]);
+        ++ds;
+        if (end) break;
+        // raw chunks of this item: both tiles' rows, k range [kc * raw_k, (kc + 1) * raw_k)
+        const int fb = (d0.x & 1) ? 2 : 0;
+        const int ntiles = 1 + ((d0.x >> 1) & 1);
+        const TcFam& F0 = P.fam[fb];
+        const int nraw = (d1.w * 64 + F0.raw_k - 1) / F0.raw_k;
+        for (int kc = 0; kc < nraw; ++kc, ++rp) {
+          const int slot_r = rp % P.raw_stages;
+          if (rp >= P.raw_stages && !mbar_wait(&raw_empty[slot_r], uint32_t(rp / P.raw_stages - 1) & 1u)) {
+            ok = false;
+            break;
+          }
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&raw_full[slot_r], uint32_t(ntiles * 128 * F0.win));
+          uint8_t* dst0 = wring + size_t(slot_r) * P.raw_stage_bytes;
+          for (int f = 0; f < ntiles; ++f) {
+            const TcFam& F = P.fam[fb + f];
+            const int y = (d0.z + F.m_off) / F.g;
+            for (int j = 0; j < F.g; ++j) {
+              const int xb = (j * F.row_bytes + kc * F.cb) & ~15;
+              tma_load_3d(dst0 + size_t(f) * 128 * F.win + size_t(j) * (128 / F.g) * F.win, &P.amap[fb + f], xb / 8, y,
+                          d0.y, &raw_full[slot_r]);
+            }
+          }
+        }
+        item = next;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // bounded wait for the copies already issued, so none lands after the CTA exits
+        for (int q = (rp > P.raw_stages ? rp - P.raw_stages : 0); q < rp; ++q)
+          mbar_wait(&raw_full[q % P.raw_stages], uint32_t(q / P.raw_stages) & 1u);
+      }
+    }
+  } else if (warp == kTcWarpB) {
+    // ------------------------------------------------ activation rows (B operand) TMA
+    if (lane == 0) {
+      int bs = 0;
+      bool ok = true;
+      for (int ds = 0; ok; ++ds) {
+        int4 d0, d1;
+        if (!read_desc(ds, d0, d1)) break;
+        if (d0.x < 0) break;
+        const int sh = d0.x & 1;
+        const int N = d1.y;
+        for (int s = 0; s < d1.w; ++s, ++bs) {
+          const int slot = bs % kTcBStages;
+          if (bs >= kTcBStages && !mbar_wait(&b_empty[slot], uint32_t(bs / kTcBStages - 1) & 1u)) {
+            ok = false;
+            break;
+          }
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[slot], uint32_t(N * 128));
+          uint8_t* dst = bring + size_t(slot) * kTcBStageBytes;
+          for (int nb = 0; nb < N / 16; ++nb)
+            tma_load_2d(dst + nb * 2048, &P.bmap[sh], s * 64, d1.x + 16 * nb, &b_full[slot]);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        for (int q = (bs > kTcBStages ? bs - kTcBStages : 0); q < bs; ++q)
+          mbar_wait(&b_full[q % kTcBStages], uint32_t(q / kTcBStages) & 1u);
+      }
+    }
+  } else if (warp == kTcWarpMma) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int as = 0, bs = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        int4 d0, d1;
+        if (!read_desc(it, d0, d1)) break;
+        if (d0.x < 0) break;
+        const int two = (d0.x >> 1) & 1;
+        const int buf = it & 1;
+        if (it >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(it / 2 - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t idesc = umma_idesc_f16(128, d1.y);
+        const uint32_t dcol = tmem + uint32_t(kTcAccCol + buf * 128);
+        for (int s = 0; s < d1.w; ++s, ++as, ++bs) {
+          const int aslot = as % kTcAStages, bslot = bs % kTcBStages;
+          if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u) ||
+              !mbar_wait(&b_full[bslot], uint32_t(bs / kTcBStages) & 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t acol = tmem + uint32_t(aslot * 64);
+          const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 16 k per MMA: 8 tensor-memory columns, 32 bytes of B
+            const uint64_t bdesc = umma_desc_sw128(b_s + 32 * kk);
+            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+            umma_f16_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);
+            if (two) umma_f16_ts(dcol + 64, acol + 32 + 8 * kk, bdesc, idesc, acc);
+          }
+          umma_commit(&a_empty[aslot]);
+          umma_commit(&b_empty[bslot]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+      }
+      if (!ok) *abort_flag = 1;
+      umma_commit(done);  // every MMA issued above has completed once this arrives
+      mbar_wait(done, 0);
+    }
+  } else if (warp < kTcWarpEpi) {
+    // ------------------------------------------------ dequantize into tensor memory
+    const int f = (warp - kTcWarpDq) >> 2;    // tile 0 (warps 2-5) or tile 1 (warps 6-9)
+    const int qw = warp & 3;                  // tensor-memory lane quarter this warp may access
+    const int r = 32 * qw + lane;             // row of the tile = tensor-memory lane
+    const uint32_t tlane = uint32_t(32 * qw) << 16;
+    const uint32_t wring_s = smem_u32(wring);
+    int rp = 0, as = 0;
+    bool ok = true;
+    for (int ds = 0; ok; ++ds) {
+      int4 d0, d1;
+      int4 dd0 = make_int4(0, 0, 0, 0), dd1 = dd0;
+      if (lane == 0 && !read_desc(ds, dd0, dd1)) dd0.x = -2;
+      d0.x = __shfl_sync(0xffffffffu, dd0.x, 0);
+      d0.y = __shfl_sync(0xffffffffu, dd0.y, 0);
+      d0.z = __shfl_sync(0xffffffffu, dd0.z, 0);
+      d1.w = __shfl_sync(0xffffffffu, dd1.w, 0);
+      if (d0.x < 0) break;
+      const int fb = (d0.x & 1) ? 2 : 0;
+      const bool tile_on = f == 0 || ((d0.x >> 1) & 1);
+      const TcFam& F = P.fam[fb + f];
+      const TcFam& F0 = P.fam[fb];
+      const bool row_on = tile_on && d0.z + F.m_off + r < F.rows;  // warp-uniform (rows % 32 == 0)
+      const int g = F.g, j = r % g, q = r / g;
+      const uint32_t row_off = uint32_t(f * 128 * F.win + j * (128 / g) * F.win + q * F.win);
+      const int spr = F0.raw_k / 64;  // MMA stages per raw chunk
+      const int nraw = (d1.w + spr - 1) / spr;
+      for (int kc = 0; kc < nraw && ok; ++kc, ++rp) {
+        const int slot_r = rp % P.raw_stages;
+        if (!mbar_wait(&raw_full[slot_r], uint32_t(rp / P.raw_stages) & 1u)) {
+          ok = false;
+          break;
+        }
+        const uint32_t mis = uint32_t(j * F.row_bytes + kc * F.cb) & 15u;
+        const uint32_t rbase = wring_s + uint32_t(slot_r) * P.raw_stage_bytes + row_off + mis;
+        for (int h = 0; h < spr && kc * spr + h < d1.w; ++h, ++as) {
+          const int aslot = as % kTcAStages;
+          if (as >= kTcAStages && !mbar_wait(&a_empty[aslot], uint32_t(as / kTcAStages - 1) & 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (row_on) {
+            uint32_t o[32];
+            tc_dequant64(F.fmt, rbase + uint32_t(h * (F.cb / spr)), o);
+            const uint32_t taddr = tmem + tlane + uint32_t(aslot * 64 + f * 32);
+            tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(&o[0]));
+            tmem_st16(taddr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&o[16]));
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          mbar_arrive(&a_full[aslot]);
+        }
+        mbar_arrive(&raw_empty[slot_r]);
+      }
+    }
+    if (!ok) *abort_flag = 1;
+  } else {
+    // ------------------------------------------------ epilogue
+    const int qw = warp & 3;
+    const int r = 32 * qw + lane;
+    const uint32_t tlane = uint32_t(32 * qw) << 16;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      int4 d0, d1;
+      int4 dd0 = make_int4(0, 0, 0, 0), dd1 = dd0;
+      if (lane == 0 && !read_desc(it, dd0, dd1)) dd0.x = -2;
+      d0 = make_int4(__shfl_sync(0xffffffffu, dd0.x, 0), __shfl_sync(0xffffffffu, dd0.y, 0),
+                     __shfl_sync(0xffffffffu, dd0.z, 0), __shfl_sync(0xffffffffu, dd0.w, 0));
+      d1 = make_int4(__shfl_sync(0xffffffffu, dd1.x, 0), __shfl_sync(0xffffffffu, dd1.y, 0),
+                     __shfl_sync(0xffffffffu, dd1.z, 0), __shfl_sync(0xffffffffu, dd1.w, 0));
+      if (d0.x < 0) break;
+      const int sh = d0.x & 1, two = (d0.x >> 1) & 1;
+      const int fb = sh ? 2 : 0;
+      const int ntok = d0.w, N = d1.y, obase = d1.z;
+      const int buf = it & 1;
+      if (!mbar_wait(&acc_full[buf], uint32_t(it / 2) & 1u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + tlane + uint32_t(kTcAccCol + buf * 128);
+      if (P.phase == 0) {
+        const TcFam& G = P.fam[fb];
+        const TcFam& U = P.fam[fb + 1];
+        const int row = d0.z + r;
+        const bool on = row < G.rows;
+        float sg = 1.f, su = 1.f;
+        if (on && G.fmt == BQG_I4_ROW) {
+          sg = __ldg(reinterpret_cast<const float*>(G.base + (sh ? 0 : size_t(d0.y) * G.stride) + G.scale_off) + row);
+          su = __ldg(reinterpret_cast<const float*>(U.base + (sh ? 0 : size_t(d0.y) * U.stride) + U.scale_off) + row);
+        }
+        __half* hrow = P.hout[sh] + tc_kpos(row, P.hperm[sh]);
+        const int hs = P.hstride[sh];
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          uint32_t gv[16], uv[16];
+          tmem_ld16_nowait(acc + uint32_t(c0), gv);
+          tmem_ld16_nowait(acc + uint32_t(64 + c0), uv);
+          tmem_wait_ld();
+          if (on) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int n = c0 + i;
+              if (n < ntok) {
+                const float hv = act_fn(P.act, __uint_as_float(gv[i]) * sg) * (__uint_as_float(uv[i]) * su);
+                hrow[size_t(obase + n) * hs] = __float2half_rn(hv);
+              }
+            }
+          }
+        }
+      } else {
+        for (int f = 0; f <= two; ++f) {
+          const TcFam& D = P.fam[fb + f];
+          const int row = d0.z + D.m_off + r;
+          const bool on = row < D.rows;
+          float sd = 1.f;
+          if (on && D.fmt == BQG_I4_ROW)
+            sd = __ldg(reinterpret_cast<const float*>(D.base + (sh ? 0 : size_t(d0.y) * D.stride) + D.scale_off) + row);
+          for (int c0 = 0; c0 < N; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16_nowait(acc + uint32_t(f * 64 + c0), v);
+            tmem_wait_ld();
+            if (on) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int n = c0 + i;
+                if (n < ntok) {
+                  const int orow = sh ? obase + n : __ldg(P.perm + obase + n);
+                  P.yout[sh][size_t(orow) * P.ystride + row] = __uint_as_float(v[i]) * sd;
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kTcWarpMma) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// ---------------------------------------------------------------- activation rows in fp16
+// Routed rows in expert-grouped order (row i = x of token perm[i] / top_k) and, with a shared
+// expert, its rows in token order; each group of 8 values in the order of the family's format.
+__global__ void __launch_bounds__(256) k_moe_xprep(const float* __restrict__ x, const int32_t* __restrict__ perm,
+                                                 const int32_t* __restrict__ offsets, int n_experts, int top_k,
+                                                 int tokens, int hidden, __half* __restrict__ xg, int nib_r,
+                                                 __half* __restrict__ xs, int nib_s) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int routed_rows = offsets[n_experts];  // pairs with a valid expert id
+  const int groups = hidden / 8;
+  const long long total = (long long)(routed_rows + (xs != nullptr ? tokens : 0)) * groups;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int row = int(i / groups), m = int(i - (long long)row * groups);
+    int src;
+    __half* dst;
+    int nib;
+    if (row < routed_rows) {
+      src = __ldg(perm + row) / top_k;
+      dst = xg + size_t(row) * hidden + 8 * m;
+      nib = nib_r;
+    } else {
+      src = row - routed_rows;
+      dst = xs + size_t(src) * hidden + 8 * m;
+      nib = nib_s;
+    }
+    const float4 a = __ldg(reinterpret_cast<const float4*>(x + size_t(src) * hidden + 8 * m));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(x + size_t(src) * hidden + 8 * m) + 1);
+    uint4 o;
+    if (nib) {  // order 0,4,1,5,2,6,3,7
+      o.x = h2_bits(__floats2half2_rn(a.x, b.x));
+      o.y = h2_bits(__floats2half2_rn(a.y, b.y));
+      o.z = h2_bits(__floats2half2_rn(a.z, b.z));
+      o.w = h2_bits(__floats2half2_rn(a.w, b.w));
+    } else {
+      o.x = h2_bits(__floats2half2_rn(a.x, a.y));
+      o.y = h2_bits(__floats2half2_rn(a.z, a.w));
+      o.z = h2_bits(__floats2half2_rn(b.x, b.y));
+      o.w = h2_bits(__floats2half2_rn(b.z, b.w));
+    }
+    *reinterpret_cast<uint4*>(dst) = o;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+inline int tc_row_bytes(int fmt, int cols) {
+  return fmt == BQG_Q8_0 ? cols / 32 * 34 : fmt == BQG_Q4_0 ? cols / 32 * 18 : cols / 2;
+}
+
+// Geometry of one family on the tensor-core path; false when the shape is not supported there
+// (k not a multiple of 64, or rows not a whole number of super-rows).
+inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols, int m_off, TcFam* out) {
+  if (cols % 64 != 0 || rows % 32 != 0) return false;
+  TcFam F{};
+  F.base = static_cast<const uint8_t*>(base);
+  F.stride = (long long)stride;
+  F.fmt = fmt;
+  F.rows = rows;
+  F.cols = cols;
+  F.row_bytes = tc_row_bytes(fmt, cols);
+  F.g = (F.row_bytes % 16 == 0) ? 1 : (F.row_bytes % 8 == 0) ? 2 : (F.row_bytes % 4 == 0) ? 4 : 0;
+  if (F.g == 0 || rows % F.g != 0) return false;
+  if (fmt == BQG_I4_ROW) {
+    F.raw_k = 128;
+    F.cb = 64;
+    F.win = 64;  // rows are multiples of 32 bytes: every chunk starts 16-byte aligned
+    F.scale_off = int((size_t(rows) * F.row_bytes + 15) / 16 * 16);
+  } else {
+    F.raw_k = fmt == BQG_Q8_0 ? 64 : 128;
+    F.cb = F.raw_k / 32 * (fmt == BQG_Q8_0 ? 34 : 18);
+    F.win = 96;  // chunk (72 or 68 bytes) + up to 12 bytes of misalignment, rounded to 16
+  }
+  F.m_off = m_off;
+  *out = F;
+  return true;
+}
+
+// [expert][super-row][bytes] view of a family, 8-byte elements, boxes of one window x 128/g
+// super-rows of one expert.
+inline int tc_encode_amap(CUtensorMap* map, const TcFam& F, int n_experts) {
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (encode == nullptr) return BQG_ERR_CUDA;
+  const cuuint64_t srow = cuuint64_t(F.g) * F.row_bytes;
+  const cuuint64_t mat = (cuuint64_t(F.rows) * F.row_bytes + 15) / 16 * 16;
+  const cuuint64_t estride = n_experts > 1 ? cuuint64_t(F.stride) : mat;
+  const cuuint64_t dims[3] = {srow / 8, cuuint64_t(F.rows / F.g), cuuint64_t(n_experts)};
+  const cuuint64_t strides[2] = {srow, estride};
+  const cuuint32_t box[3] = {cuuint32_t(F.win / 8), cuuint32_t(128 / F.g), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  if (encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<uint8_t*>(F.base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return BQG_ERR_CUDA;
+  return BQG_OK;
+}
+
+// fp16 [rows x cols] activation rows, boxes of 64 k x 16 rows with 128-byte swizzle.
+inline int tc_encode_bmap(CUtensorMap* map, const __half* base, int rows, int cols) {
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (encode == nullptr) return BQG_ERR_CUDA;
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows < 1 ? 1 : rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return BQG_ERR_CUDA;
+  return BQG_OK;
+}
+
+inline size_t tc_smem_bytes(int raw_stages, int raw_stage_bytes) {
+  return kTcFixedSmem + size_t(raw_stages) * raw_stage_bytes;
+}
+
+// Ring depth for a window size: as many raw stages as fit the shared memory.
+inline void tc_raw_ring(int win, int* stages, int* stage_bytes) {
+  *stage_bytes = 2 * 128 * win;
+  int n = int((kTcMaxSmem - kTcFixedSmem) / size_t(*stage_bytes));
+  *stages = n > kTcRawMax ? kTcRawMax : n;
+}
+
+inline SmemAttrOnce g_tc_attr;
+
+}  // namespace bqg

@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "host_common.h"
+#include "tcgen05.cuh"
 
 namespace bqg {
 
@@ -53,103 +54,6 @@ struct PfParams {
   int ksplit;        // CTAs (cluster size) sharing one output tile
   int kchunks;       // k / kPfRawK; split s owns chunks [s*kchunks/ksplit, (s+1)*kchunks/ksplit)
 };
-
-// ---------------------------------------------------------------- tcgen05 / TMA helpers
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-  // K-major operand, 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFF);       // start address
-  d |= uint64_t(1) << 16;                     // leading byte offset (unused for swizzled K-major)
-  d |= uint64_t(1024 >> 4) << 32;             // stride byte offset: 8 rows x 128 bytes
-  d |= uint64_t(1) << 46;                     // descriptor version (sm_100)
-  d |= uint64_t(2) << 61;                     // swizzle: 128 bytes
-  return d;
-}
-
-// kind::f16 instruction descriptor: D fp32, A and B fp16, both K-major, M x N.
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int m, int n) {
-  return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
-      "[%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-
-// Eight Q4_0 weights of one qs word (element 2m = low nibble of byte m) as fp16 (q-8)*d,
-// returned as 4 half2 in element order (e0,e1) (e2,e3) (e4,e5) (e6,e7).
-__device__ __forceinline__ void q4_word_to_f16(uint32_t w, __half2 d2, uint32_t (&o)[4]) {
-  const __half2 bias = __half2half2(__ushort_as_half(0x6408));  // 1032
-  // 1024 + q as fp16: (e0,e4) (e1,e5) (e2,e6) (e3,e7)
-  uint32_t p04 = (w & 0x000F000Fu) | 0x64006400u;
-  uint32_t p15 = ((w >> 4) & 0x000F000Fu) | 0x64006400u;
-  uint32_t p26 = ((w >> 8) & 0x000F000Fu) | 0x64006400u;
-  uint32_t p37 = ((w >> 12) & 0x000F000Fu) | 0x64006400u;
-  // (1024 + q) - 1032 = q - 8 exactly; times d rounds once
-  p04 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p04), bias), d2));
-  p15 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p15), bias), d2));
-  p26 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p26), bias), d2));
-  p37 = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p37), bias), d2));
-  o[0] = __byte_perm(p04, p15, 0x5410);  // (e0, e1)
-  o[1] = __byte_perm(p26, p37, 0x5410);  // (e2, e3)
-  o[2] = __byte_perm(p04, p15, 0x7632);  // (e4, e5)
-  o[3] = __byte_perm(p26, p37, 0x7632);  // (e6, e7)
-}
-
-__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// 16 bytes at the same shared-memory offset in cluster rank `rank` (its own rank included).
-__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_saddr, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(rank));
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(remote)
-               : "memory");
-  return v;
-}
 
 // ---------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -404,25 +308,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline EncodeTiledFn encode_tiled_fn() {
-  static std::atomic<EncodeTiledFn> fn{nullptr};
-  EncodeTiledFn f = fn.load(std::memory_order_acquire);
-  if (f == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || p == nullptr)
-      return nullptr;
-    f = reinterpret_cast<EncodeTiledFn>(p);
-    fn.store(f, std::memory_order_release);
-  }
-  return f;
-}
-
 inline SmemAttrOnce g_prefill_attr;
 
 }  // namespace bqg

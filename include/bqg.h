@@ -70,6 +70,20 @@ enum bqg_status {
 enum bqg_fmt { BQG_Q8_0 = 1, BQG_Q4_0 = 2, BQG_I4_ROW = 3 };
 enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 
+/* How moe_forward runs the experts (bqg_moe_layer.path).  Both compute the same layer.
+ *   BQG_MOE_PATH_AUTO          the tensor cores from BQG_MOE_TC_MIN_TOKENS tokens on (when the
+ *                              shapes allow it), the CUDA cores below.
+ *   BQG_MOE_PATH_CUDA_CORES    grouped GEMV with integer dot products: every expert item is applied
+ *                              to its tokens one at a time (best for 1..8 tokens).
+ *   BQG_MOE_PATH_TENSOR_CORES  grouped expert GEMM on tcgen05: weights dequantized once into tensor
+ *                              memory and multiplied by all the expert's tokens at once (prefill
+ *                              chunks, large decode batches).  Needs hidden, inter and shared_inter
+ *                              multiples of 64, and activations (x and the gated hidden values)
+ *                              within the fp16 range; returns BQG_ERR_SHAPE when the shapes do not
+ *                              allow it. */
+enum bqg_moe_path { BQG_MOE_PATH_AUTO = 0, BQG_MOE_PATH_CUDA_CORES = 1, BQG_MOE_PATH_TENSOR_CORES = 2 };
+#define BQG_MOE_TC_MIN_TOKENS 16
+
 #define BQG_MAX_COLS 15360       /* largest cols (K) of the GEMV, router and prefill calls  */
 #define BQG_MAX_BATCH 256        /* largest descriptor count of one qgemv_batched call     */
 #define BQG_MAX_EXPERTS 256      /* largest n_experts of the router / MoE calls            */
@@ -188,6 +202,7 @@ typedef struct {
   const void* s_gate; /* NULL: no shared expert */
   const void* s_up;
   const void* s_down;
+  int path;          /* BQG_MOE_PATH_*: which kernels run the experts (0 = choose by token count) */
 } bqg_moe_layer;
 
 /* Bytes of device workspace moe_forward needs for `tokens` tokens (0 on invalid arguments).
@@ -225,13 +240,17 @@ BQG_API int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* i
  * held by every GPU that loads the library until the process exits; the call allocates and
  * frees nothing.  Arguments are those of moe_forward without the workspace.
  *   - Returns BQG_ERR_LIMIT when moe_workspace_size(L, tokens) exceeds BQG_NOALLOC_SCRATCH_BYTES.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress);
- *     make that first call before any stream capture that includes it.
+ *     32 MiB covers the Gemma-4-26B-A4B-like layer (hidden 2816, 128 experts, shared expert) up
+ *     to 128 tokens (21.4 MB) and the GLM-like layer (hidden 6144, 256 int4 experts of 2048) up to
+ *     64 tokens (21.0 MB); a GLM-like 128-token chunk (42 MB) does not fit.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current, and again after the device's context was destroyed and re-created
+ *     (cudaDeviceReset); make that first call before any stream capture that includes it.
  *   - All calls on a device share the one array: calls that may overlap on the GPU (different
  *     streams without ordering between them) race and must not be issued.  Calls ordered on one
  *     stream are fine; the array keeps the last call's contents, and every region the kernels read
  *     is written first by the same call, so nothing needs clearing. */
-#define BQG_NOALLOC_SCRATCH_BYTES (24u << 20)
+#define BQG_NOALLOC_SCRATCH_BYTES (32u << 20)
 BQG_API int moe_forward_noalloc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
                                 float* y, int tokens, void* stream);
 

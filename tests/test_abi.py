@@ -177,3 +177,59 @@ def test_moe_layer_binding_rejects_short_tensors():
     with pytest.raises(ValueError):
         bqg.MoELayer(4, 2, 64, 32, bqg.Q4_0, 1, T.gate, T.up, T.down, T.gate_stride, T.up_stride, T.down_stride,
                      short_shared)
+
+
+def _layer_c(spec, path=0):
+    import block_quant_gemv_b200 as bqg
+    c = bqg.MoELayerC()
+    c.n_experts, c.top_k, c.hidden, c.inter, c.expert_fmt, c.act = (spec.n_experts, spec.top_k, spec.hidden,
+                                                                     spec.inter, spec.expert_fmt, spec.act)
+    c.gate = c.up = c.down = 0x10000
+    c.gate_stride = c.up_stride = (synth.weight_bytes(spec.expert_fmt, spec.inter, spec.hidden) + 15) // 16 * 16
+    c.down_stride = (synth.weight_bytes(spec.expert_fmt, spec.hidden, spec.inter) + 15) // 16 * 16
+    if spec.shared_inter:
+        c.shared_inter, c.shared_fmt = spec.shared_inter, spec.shared_fmt
+        c.s_gate = c.s_up = c.s_down = 0x20000
+    c.path = path
+    return c
+
+
+def test_noalloc_scratch_covers_the_listed_configs(L):
+    """moe_forward_noalloc's fixed scratch holds the workspace of every listed MoE configuration:
+    the Gemma-like layer at 1, 16 and 128 tokens and the GLM-like layer at 1, 8 and 64 tokens."""
+    import re
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    m = re.search(r"#define BQG_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", open(HEADER).read())
+    limit = int(m.group(1)) << int(m.group(2))
+    assert limit == bqg.NOALLOC_SCRATCH_BYTES
+    for spec, Ts in ((wl.GEMMA_MOE, (1, 16, 128)), (wl.GLM_MOE, (1, 8, 64))):
+        for T in Ts:
+            for path in (0, 1, 2):
+                need = L.lib().moe_workspace_size(ctypes.byref(_layer_c(spec, path)), T)
+                assert 0 < need <= limit, (spec.name, T, path, need)
+
+
+def test_moe_workspace_covers_fewer_tokens(L):
+    """A workspace sized for T tokens serves every call with fewer tokens, whichever path the
+    automatic choice takes for them."""
+    from synth import workloads as wl
+    for spec in (wl.GEMMA_MOE, wl.GLM_MOE):
+        c = _layer_c(spec)
+        sizes = [L.lib().moe_workspace_size(ctypes.byref(c), T) for T in range(1, 70)]
+        assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+
+
+def test_moe_path_argument_errors(L):
+    """An unknown path value is refused; forcing the tensor cores on shapes they cannot take
+    (inter not a multiple of 64) gives BQG_ERR_SHAPE before any launch."""
+    from synth import workloads as wl
+    A = 0x10000
+    c = _layer_c(wl.GEMMA_MOE, 7)
+    assert L.lib().moe_workspace_size(ctypes.byref(c), 16) == 0
+    assert L.lib().moe_forward(ctypes.byref(c), A, A, A, A, 16, A, 1 << 30, None) == -1
+    spec = wl.MoESpec("odd", 8, 2, 128, 96, 2, 1, 0, 0, False)
+    c = _layer_c(spec, 2)
+    assert L.lib().moe_forward(ctypes.byref(c), A, A, A, A, 16, A, 1 << 30, None) == -3
+    c.path = 0
+    assert L.lib().moe_workspace_size(ctypes.byref(c), 16) > 0

@@ -53,7 +53,7 @@ def test_noalloc_rejects_sizes_beyond_the_scratch():
     spec = wl.MoESpec("na_limit", 4, 2, 2048, 2048, bqg.Q4_0, bqg.ACT_SILU, 0, 0, False)
     L = wl.build_moe_layer(spec, 0, 0, device="cuda")
     lay = device_layer(L)
-    tokens = 1024  # 2048 pairs x (2048 + 2048) floats > 24 MiB of scratch
+    tokens = 4096  # 8192 pairs of per-pair rows of 2048 values: far beyond the fixed scratch
     assert bqg.moe_workspace_size(lay, tokens) > bqg.NOALLOC_SCRATCH_BYTES
     x = torch.zeros(tokens, spec.hidden, device="cuda")
     idx = torch.zeros(tokens, 2, dtype=torch.int32, device="cuda")
