@@ -2,7 +2,7 @@
 
     python -m block_quant_gemv_b200.cases decode  [--layers 22] [--iters 5]
     python -m block_quant_gemv_b200.cases prefill [--tokens 128] [--n 14336] [--k 4096] [--iters 5]
-    python -m block_quant_gemv_b200.cases moe gemma|glm [--tokens 1] [--iters 5]
+    python -m block_quant_gemv_b200.cases moe gemma|glm [--tokens 1] [--experts E] [--path P] [--iters 5]
 
 decode:  one TinyLlama-shape decode step (7 Q4_0 projections per layer + the Q8_0 LM head),
          all matrices in one qgemv_batched launch per call.
@@ -15,6 +15,7 @@ call (CUDA events, after two warm-up calls) and the device error bits.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import os
 import sys
 
@@ -60,10 +61,12 @@ def prefill(args) -> str:
 
 def moe(args) -> str:
     spec = wl.GEMMA_MOE if args.layer == "gemma" else wl.GLM_MOE
+    if args.experts:  # the same layer geometry with fewer routed experts (a smaller footprint)
+        spec = dataclasses.replace(spec, n_experts=args.experts)
     T = wl.build_moe_layer(spec, 0, layer=0, device="cuda")
     shared = None if T.shared is None else (spec.shared_fmt, spec.shared_inter) + tuple(T.shared)
     L = bqg.MoELayer(spec.n_experts, spec.top_k, spec.hidden, spec.inter, spec.expert_fmt, spec.act, T.gate, T.up,
-                     T.down, T.gate_stride, T.up_stride, T.down_stride, shared)
+                     T.down, T.gate_stride, T.up_stride, T.down_stride, shared, path=args.path)
     tok = args.tokens
     x = wl.moe_tokens(spec, 0, tok).cuda()
     logits = (torch.empty(tok, spec.n_experts, device="cuda") if spec.router
@@ -94,6 +97,8 @@ def main(argv=None):
     m = sub.add_parser("moe")
     m.add_argument("layer", choices=["gemma", "glm"])
     m.add_argument("--tokens", type=int, default=1)
+    m.add_argument("--experts", type=int, default=0, help="routed experts (default: the layer's own count)")
+    m.add_argument("--path", type=int, default=0, help="0 automatic, 1 CUDA cores, 2 tensor cores")
     for s in (d, p, m):
         s.add_argument("--iters", type=int, default=5)
     args = ap.parse_args(argv)

@@ -162,12 +162,24 @@ inline bool tc_layer(const bqg_moe_layer* L, TcLayer* T) {
   return true;
 }
 
+// The automatic choice.  A tensor-core MMA instruction (M = 128 weight rows, K = 16) costs about
+// the same whatever the number of tokens on its N side, so that path pays per weight read,
+// while the CUDA-core path pays per (weight, token).  Measured crossovers on B200: with a
+// shared expert (its N is every token) from 16 tokens on; without one, once the routed experts
+// average 4 tokens each (GLM-like layer: T = 64 takes 2.06 ms on CUDA cores against 2.49 ms,
+// T = 128 3.96 ms against 2.88 ms).
+inline bool moe_tc_preferred(const bqg_moe_layer* L, int tokens) {
+  if (L->s_gate != nullptr && tokens >= BQG_MOE_TC_MIN_TOKENS) return true;
+  return (long long)tokens * L->top_k >= (long long)BQG_MOE_TC_MIN_PER_EXPERT * L->n_experts &&
+         tokens >= BQG_MOE_TC_MIN_TOKENS;
+}
+
 // Path for `tokens` tokens: BQG_MOE_PATH_CUDA_CORES or BQG_MOE_PATH_TENSOR_CORES (negative: error).
 inline int moe_path(const bqg_moe_layer* L, int tokens) {
   if (L->path == BQG_MOE_PATH_CUDA_CORES) return BQG_MOE_PATH_CUDA_CORES;
   const bool tc = tc_layer(L, nullptr);
   if (L->path == BQG_MOE_PATH_TENSOR_CORES) return tc ? int(BQG_MOE_PATH_TENSOR_CORES) : int(BQG_ERR_SHAPE);
-  return (tc && tokens >= BQG_MOE_TC_MIN_TOKENS) ? BQG_MOE_PATH_TENSOR_CORES : BQG_MOE_PATH_CUDA_CORES;
+  return (tc && moe_tc_preferred(L, tokens)) ? BQG_MOE_PATH_TENSOR_CORES : BQG_MOE_PATH_CUDA_CORES;
 }
 
 // Workspace for every call of up to `tokens` tokens (each path's layout grows with the tokens;
@@ -178,7 +190,9 @@ inline size_t moe_ws_total(const bqg_moe_layer* L, int tokens) {
   if (path == BQG_MOE_PATH_CUDA_CORES) return moe_ws_layout(L, tokens).total;
   size_t need = moe_ws_layout_tc(L, tokens).total;
   if (L->path == BQG_MOE_PATH_AUTO) {
-    const int below = tokens < BQG_MOE_TC_MIN_TOKENS ? tokens : BQG_MOE_TC_MIN_TOKENS - 1;
+    // the largest token count below `tokens` that the automatic choice sends to the CUDA cores
+    int below = tokens - 1;
+    while (below >= 1 && moe_tc_preferred(L, below)) --below;
     if (below >= 1) {
       const size_t cc = moe_ws_layout(L, below).total;
       if (cc > need) need = cc;

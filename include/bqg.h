@@ -71,8 +71,10 @@ enum bqg_fmt { BQG_Q8_0 = 1, BQG_Q4_0 = 2, BQG_I4_ROW = 3 };
 enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 
 /* How moe_forward runs the experts (bqg_moe_layer.path).  Both compute the same layer.
- *   BQG_MOE_PATH_AUTO          the tensor cores from BQG_MOE_TC_MIN_TOKENS tokens on (when the
- *                              shapes allow it), the CUDA cores below.
+ *   BQG_MOE_PATH_AUTO          the tensor cores (when the shapes allow it) from
+ *                              BQG_MOE_TC_MIN_TOKENS tokens on if the layer has a shared expert,
+ *                              else once tokens * top_k >= BQG_MOE_TC_MIN_PER_EXPERT * n_experts
+ *                              (and tokens >= BQG_MOE_TC_MIN_TOKENS); the CUDA cores otherwise.
  *   BQG_MOE_PATH_CUDA_CORES    grouped GEMV with integer dot products: every expert item is applied
  *                              to its tokens one at a time (best for 1..8 tokens).
  *   BQG_MOE_PATH_TENSOR_CORES  grouped expert GEMM on tcgen05: weights dequantized once into tensor
@@ -83,6 +85,7 @@ enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
  *                              allow it. */
 enum bqg_moe_path { BQG_MOE_PATH_AUTO = 0, BQG_MOE_PATH_CUDA_CORES = 1, BQG_MOE_PATH_TENSOR_CORES = 2 };
 #define BQG_MOE_TC_MIN_TOKENS 16
+#define BQG_MOE_TC_MIN_PER_EXPERT 4
 
 #define BQG_MAX_COLS 15360       /* largest cols (K) of the GEMV, router and prefill calls  */
 #define BQG_MAX_BATCH 256        /* largest descriptor count of one qgemv_batched call     */

@@ -37,3 +37,15 @@ def oracle_router_logits(spec: wl.MoESpec, seed: int, layer: int, x: np.ndarray)
     R = wl.normal_f32(seed, wl.stream_id(f"{spec.name}/L{layer}/router"), spec.n_experts * spec.hidden,
                       std=0.02).view(spec.n_experts, spec.hidden).numpy()
     return om.router_logits(R, x)
+
+
+def expected_path(spec: wl.MoESpec, tokens: int) -> int:
+    """The path the library's automatic choice takes for this layer (mirrors include/bqg.h):
+    tensor cores from 16 tokens on with a shared expert, else once the routed experts average 4
+    tokens each; only shapes that are multiples of 64 can take them."""
+    dims = [spec.hidden, spec.inter] + ([spec.shared_inter] if spec.shared_inter else [])
+    if any(d % 64 for d in dims) or tokens < bqg.MOE_TC_MIN_TOKENS:
+        return bqg.MOE_PATH_CUDA_CORES
+    if spec.shared_inter or tokens * spec.top_k >= bqg.MOE_TC_MIN_PER_EXPERT * spec.n_experts:
+        return bqg.MOE_PATH_TENSOR_CORES
+    return bqg.MOE_PATH_CUDA_CORES

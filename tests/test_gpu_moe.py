@@ -8,7 +8,7 @@ import block_quant_gemv_b200 as bqg
 import synth
 from synth import workloads as wl
 from oracle import moe as om
-from tests.moe_util import device_layer, oracle_layer, oracle_router_logits
+from tests.moe_util import device_layer, expected_path, oracle_layer, oracle_router_logits
 from tests.util import assert_close, need_gpu
 
 pytestmark = pytest.mark.gpu
@@ -143,9 +143,8 @@ def _glm_layer_check(L, spec, layer, tokens, sample=None):
     sel = np.arange(tokens) if sample is None else np.asarray(sample)
     ref = om.moe_layer(oracle_layer(spec, 0, layer), x.numpy()[sel], ridx[sel], rw[sel])
     assert_close(y.cpu().numpy()[sel], ref, what=f"glm-like layer {layer} T={tokens}")
-    # the automatic path: CUDA cores (x in 16-bit fixed point) below 16 tokens, tensor cores
-    # (fp16 operands) from 16 on
-    strict = 1e-4 if tokens < bqg.MOE_TC_MIN_TOKENS else 1e-3
+    # the automatic path: CUDA cores (x in 16-bit fixed point) or tensor cores (fp16 operands)
+    strict = 1e-4 if expected_path(spec, tokens) == bqg.MOE_PATH_CUDA_CORES else 1e-3
     assert_close(y.cpu().numpy()[sel], ref, tol=strict, what=f"glm-like layer {layer} T={tokens} (strict)")
 
 
