@@ -11,6 +11,8 @@ Modules
 * ``oracle.moe``     — router logits, top-k with renormalised weights, GeGLU/SwiGLU
                        expert FFN, routed + shared MoE layer, chained layer stack.
 * ``oracle.prefill`` — Y = X W^T for the 128-token prefill chunk, rounded to fp16.
+* ``oracle.argmax``  — greedy token selection (argmax, ties to the lower index) after the
+                       quantized LM head.
 
 Every function is pinned by tests under ``tests/test_oracle_*.py`` against values
 fixed by the pages' definitions and by mathematics (hand-worked blocks under
@@ -19,4 +21,4 @@ invariants).  The pages print no kernel outputs or worked examples, so no pin is
 page-printed value; each function is pinned by the closed forms, hand-worked blocks,
 brute force and invariants listed in those tests.
 """
-from . import moe, prefill, qgemv  # noqa: F401
+from . import argmax, moe, prefill, qgemv  # noqa: F401
