@@ -5,7 +5,8 @@ kernels.  PyTorch provides device memory and the current stream.  There is no CP
 fallback: if the library is not built, every call raises.
 
 The functions mirror the C ABI in include/bqg.h (same names):
-    qgemv, qgemv_batched, qgemm_prefill, moe_router_logits, moe_router_topk,
+    qgemv, qgemv_batched, qgemv_argmax, qgemv_batched_argmax (GemvBatch.run(argmax=...)),
+    qgemm_prefill, moe_router_logits, moe_router_topk,
     moe_workspace_size, moe_forward, moe_forward_noalloc, bqg_status_string, bqg_weight_bytes,
     bqg_device_errors, bqg_selftest_wait_timeout
 """
@@ -22,7 +23,7 @@ __all__ = [
     "MOE_PATH_AUTO", "MOE_PATH_CUDA_CORES", "MOE_PATH_TENSOR_CORES",
     "lib", "library_path", "bqg_status_string", "bqg_weight_bytes", "bqg_device_errors",
     "bqg_selftest_wait_timeout",
-    "qgemv", "qgemv_batched", "GemvBatch", "qgemm_prefill", "moe_router_logits",
+    "qgemv", "qgemv_batched", "GemvBatch", "qgemv_argmax", "ArgmaxState", "qgemm_prefill", "moe_router_logits",
     "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward", "moe_forward_noalloc",
 ]
 
@@ -67,6 +68,8 @@ _SIGNATURES = {
     "bqg_device_errors": (_i, [ctypes.POINTER(_i)]),
     "qgemv": (_i, [_i, _vp, _vp, _vp, _i, _i, _vp]),
     "qgemv_batched": (_i, [ctypes.POINTER(GemvDesc), _i, _vp]),
+    "qgemv_argmax": (_i, [_i, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
+    "qgemv_batched_argmax": (_i, [ctypes.POINTER(GemvDesc), _i, _i, _vp, _vp, _vp, _vp]),
     "qgemm_prefill": (_i, [_i, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "moe_router_logits": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "moe_router_topk": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
@@ -158,6 +161,35 @@ def qgemv(fmt: int, W: torch.Tensor, x: torch.Tensor, rows: int, cols: int,
     return y
 
 
+class ArgmaxState:
+    """Device outputs and working state of the fused greedy argmax: token (int32), its logit
+    (fp32) and the 16-byte state the kernel leaves zeroed after every call."""
+
+    def __init__(self, device):
+        self.token = torch.zeros(1, dtype=torch.int32, device=device)
+        self.value = torch.zeros(1, dtype=torch.float32, device=device)
+        self.state = torch.zeros(2, dtype=torch.int64, device=device)
+
+    def ptrs(self):
+        return _ptr(self.token), _ptr(self.value), _ptr(self.state)
+
+
+def qgemv_argmax(fmt: int, W: torch.Tensor, x: torch.Tensor, rows: int, cols: int,
+                 y: Optional[torch.Tensor] = None, out: Optional[ArgmaxState] = None):
+    """y = W x and the greedy token argmax(y) (ties to the lower index) in one launch.
+    Returns (y, ArgmaxState); read .token / .value on the device."""
+    _need_cuda("W", W, torch.uint8)
+    _need_cuda("x", x, torch.float32)
+    if y is None:
+        y = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _need_cuda("y", y, torch.float32)
+    if W.numel() < bqg_weight_bytes(fmt, rows, cols) or x.numel() < cols or y.numel() < rows:
+        raise ValueError("tensor smaller than the shape requires")
+    out = out if out is not None else ArgmaxState(x.device)
+    _check(lib().qgemv_argmax(fmt, _ptr(W), _ptr(x), _ptr(y), rows, cols, *out.ptrs(), _stream(x)), "qgemv_argmax")
+    return y, out
+
+
 class GemvBatch:
     """A prepared list of independent GEMVs (fmt, W, x, y, rows, cols) launched as one
     qgemv_batched call.  Keeps the tensors alive and the descriptor array ready."""
@@ -177,9 +209,16 @@ class GemvBatch:
             d.W, d.x, d.y = W.data_ptr(), x.data_ptr(), y.data_ptr()
         self.device = self.items[0][2].device
 
-    def run(self, stream: Optional[torch.cuda.Stream] = None):
+    def run(self, stream: Optional[torch.cuda.Stream] = None, argmax: Optional[tuple] = None):
+        """One launch over every descriptor; with argmax = (index, ArgmaxState) also the greedy
+        token of descriptor `index`'s y."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        _check(lib().qgemv_batched(self.descs, len(self.descs), _vp(s.cuda_stream)), "qgemv_batched")
+        if argmax is None:
+            _check(lib().qgemv_batched(self.descs, len(self.descs), _vp(s.cuda_stream)), "qgemv_batched")
+        else:
+            index, out = argmax
+            _check(lib().qgemv_batched_argmax(self.descs, len(self.descs), index, *out.ptrs(), _vp(s.cuda_stream)),
+                   "qgemv_batched_argmax")
 
 
 def qgemv_batched(items: Sequence[tuple]) -> None:

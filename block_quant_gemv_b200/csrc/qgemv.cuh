@@ -84,11 +84,37 @@ struct CtaRange {
 template <int MAXP>
 struct GemvParams {
   int n;
-  int pad;
+  int am_p;                    // problem whose y is reduced to its argmax (greedy token), or -1
   long long total_bytes;
+  int32_t* am_token;           // argmax index of y[am_p] (ties: the lower index)
+  float* am_value;             // its value (may be null)
+  unsigned long long* am_state;  // [2]: packed running maximum, CTA completion count (zero between calls)
   GemvProb p[MAXP];
   CtaRange cta[kGemvMaxGrid];
 };
+
+// ---------------------------------------------------------------- greedy argmax of one output
+// A running (value, row) maximum: equal values keep the lower row.
+__device__ __forceinline__ void am_take(float& bv, int& bi, float v, int i) {
+  if (v > bv || (v == bv && i < bi)) {
+    bv = v;
+    bi = i;
+  }
+}
+// 64-bit key whose unsigned order is (value, then lower row first): the value's bits made
+// order-preserving (sign flipped for positives, all bits for negatives; -0.0 taken as +0.0) in
+// the high word, the complemented row in the low word.
+__device__ __forceinline__ unsigned long long am_pack(float v, int i) {
+  if (v == 0.f) v = 0.f;
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<unsigned long long>(u) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(i));
+}
+__device__ __forceinline__ void am_unpack(unsigned long long key, float& v, int& i) {
+  const uint32_t u = static_cast<uint32_t>(key >> 32);
+  v = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+  i = static_cast<int>(~static_cast<uint32_t>(key & 0xffffffffu));
+}
 
 __host__ __device__ constexpr int unit_bytes(int kind) {
   return kind == kQ8Pair ? 68 : kind == kQ8One ? 34 : kind == kQ4Pair ? 36 : kind == kQ4One ? 18 : kind == kI4x64 ? 32 : 16;
@@ -369,8 +395,9 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 template <int KIND, int MAXP>
 __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi, int ra, int rbnd, uint8_t* ring,
                                             float* xs, float* red, uint64_t* full, uint64_t* xfull, uint64_t* xfree,
-                                            uint64_t* empty, int& s, int& xs_n, XUnit& X) {
+                                            uint64_t* empty, int& s, int& xs_n, XUnit& X, float& am_v, int& am_i) {
   const GemvProb& P = prm.p[pi];
+  const bool track = pi == prm.am_p;  // this matrix's rows also feed the greedy argmax
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = P.units, row_bytes = P.row_bytes;
   const int gw = gemv_group_warps(units);
@@ -424,9 +451,11 @@ __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi,
           if (gw == 1) {
             if (is_i4(KIND)) v[0] *= __ldg(scales + i);
             P.y[r0 + i] = v[0];
+            if (track) am_take(am_v, am_i, v[0], r0 + i);
             if (two) {
               if (is_i4(KIND)) v[1] *= __ldg(scales + i + groups);
               P.y[r0 + i + groups] = v[1];
+              if (track) am_take(am_v, am_i, v[1], r0 + i + groups);
             }
           } else {
             red[(par * kGemvConsumerWarps + warp) * kGemvRedRows + nmine] = v[0];
@@ -447,6 +476,7 @@ __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi,
         const int row = r0 + g + lane * groups;
         if (is_i4(KIND)) v *= __ldg(reinterpret_cast<const float*>(P.W + P.scale_off) + row);
         P.y[row] = v;
+        if (track) am_take(am_v, am_i, v, row);
       }
     }
   }
@@ -546,6 +576,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
   int s = 0;     // stage counter (same sequence as the producer's, and in every consumer warp)
   int xs_n = 0;  // problems whose x has been read
   XUnit X;
+  float am_v = -INFINITY;  // greedy argmax: the best (value, row) this thread has written
+  int am_i = 0x7fffffff;
   for (int pi = cr.p0; pi <= p_last; ++pi) {
     const GemvProb& P = prm.p[pi];
     int ra, rbnd;
@@ -556,14 +588,47 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
     named_bar_sync(1, kGemvCompute);
     bool ok;
     switch (P.kind) {
-      case kQ4Pair: ok = gemv_matrix<kQ4Pair, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
-      case kQ8Pair: ok = gemv_matrix<kQ8Pair, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
-      case kI4x64: ok = gemv_matrix<kI4x64, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
-      case kQ4One: ok = gemv_matrix<kQ4One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
-      case kQ8One: ok = gemv_matrix<kQ8One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
-      default: ok = gemv_matrix<kI4x32, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X); break;
+      case kQ4Pair: ok = gemv_matrix<kQ4Pair, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
+      case kQ8Pair: ok = gemv_matrix<kQ8Pair, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
+      case kI4x64: ok = gemv_matrix<kI4x64, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
+      case kQ4One: ok = gemv_matrix<kQ4One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
+      case kQ8One: ok = gemv_matrix<kQ8One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
+      default: ok = gemv_matrix<kI4x32, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
     }
-    if (!ok) return;
+    if (!ok) break;  // still takes part in the argmax completion below, so its count stays whole
+  }
+  if (prm.am_p < 0) return;
+  // Greedy argmax of y[am_p]: warp, then CTA maximum; one 64-bit atomicMax per CTA on the
+  // packed key; the last CTA to finish decodes it into the token and clears the state.
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, am_v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, am_i, o);
+    am_take(am_v, am_i, ov, oi);
+  }
+  __shared__ float am_wv[kGemvConsumerWarps];
+  __shared__ int am_wi[kGemvConsumerWarps];
+  if (lane == 0) {
+    am_wv[warp] = am_v;
+    am_wi[warp] = am_i;
+  }
+  named_bar_sync(1, kGemvCompute);
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kGemvConsumerWarps; ++w) am_take(am_v, am_i, am_wv[w], am_wi[w]);
+    if (am_i != 0x7fffffff) atomicMax(prm.am_state, am_pack(am_v, am_i));
+    __threadfence();
+    unsigned int* count = reinterpret_cast<unsigned int*>(prm.am_state + 1);
+    if (atomicAdd(count, 1u) == gridDim.x - 1) {
+      __threadfence();
+      const unsigned long long key = atomicAdd(prm.am_state, 0ull);
+      float v;
+      int i;
+      am_unpack(key, v, i);
+      *prm.am_token = i;
+      if (prm.am_value != nullptr) *prm.am_value = v;
+      prm.am_state[0] = 0ull;  // ready for the next call on this stream
+      *count = 0u;
+    }
   }
 }
 

@@ -123,27 +123,68 @@ inline int launch_gemv(GemvParams<MAXP>& prm, long long total_rows, cudaStream_t
 
 extern "C" size_t bqg_weight_bytes(int fmt, int rows, int cols) { return bqg::weight_bytes(fmt, rows, cols); }
 
-extern "C" int qgemv(int fmt, const void* W, const float* x, float* y, int rows, int cols, void* stream) {
-  bqg::GemvParams<1> prm{};
-  int st = bqg::make_gemv_prob(fmt, W, x, y, rows, cols, &prm.p[0]);
-  if (st != BQG_OK) return st;
-  prm.n = 1;
-  return bqg::launch_gemv<1>(prm, rows, static_cast<cudaStream_t>(stream));
+namespace bqg {
+// The greedy-argmax outputs of a GEMV launch (none when token is null).
+template <int MAXP>
+inline int set_argmax(GemvParams<MAXP>& prm, int index, int32_t* token, float* value, unsigned long long* state) {
+  prm.am_p = -1;
+  if (token == nullptr && state == nullptr && value == nullptr) return BQG_OK;
+  if (token == nullptr || state == nullptr || index < 0 || index >= prm.n) return BQG_ERR_ARG;
+  if (!aligned(token, 4) || !aligned(state, 8) || (value != nullptr && !aligned(value, 4))) return BQG_ERR_ALIGN;
+  prm.am_p = index;
+  prm.am_token = token;
+  prm.am_value = value;
+  prm.am_state = state;
+  return BQG_OK;
 }
 
-extern "C" int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream) {
+inline int qgemv_impl(int fmt, const void* W, const float* x, float* y, int rows, int cols, int32_t* token,
+                      float* value, unsigned long long* state, void* stream) {
+  GemvParams<1> prm{};
+  int st = make_gemv_prob(fmt, W, x, y, rows, cols, &prm.p[0]);
+  if (st != BQG_OK) return st;
+  prm.n = 1;
+  if ((st = set_argmax(prm, 0, token, value, state)) != BQG_OK) return st;
+  return launch_gemv<1>(prm, rows, static_cast<cudaStream_t>(stream));
+}
+
+inline int qgemv_batched_impl(const bqg_gemv_desc* descs, int n, int am_index, int32_t* token, float* value,
+                              unsigned long long* state, void* stream) {
   if (descs == nullptr || n < 1) return BQG_ERR_ARG;
   if (n > BQG_MAX_BATCH) return BQG_ERR_LIMIT;
-  static_assert(sizeof(bqg::GemvParams<BQG_MAX_BATCH>) < 32000, "kernel parameter block too large");
-  bqg::GemvParams<BQG_MAX_BATCH> prm{};
+  static_assert(sizeof(GemvParams<BQG_MAX_BATCH>) < 32000, "kernel parameter block too large");
+  GemvParams<BQG_MAX_BATCH> prm{};
   long long total_rows = 0;
   for (int i = 0; i < n; ++i) {
     const bqg_gemv_desc& d = descs[i];
     if (d.reserved != 0) return BQG_ERR_ARG;
-    int st = bqg::make_gemv_prob(d.fmt, d.W, d.x, d.y, d.rows, d.cols, &prm.p[i]);
+    int st = make_gemv_prob(d.fmt, d.W, d.x, d.y, d.rows, d.cols, &prm.p[i]);
     if (st != BQG_OK) return st;
     total_rows += d.rows;
   }
   prm.n = n;
-  return bqg::launch_gemv<BQG_MAX_BATCH>(prm, total_rows, static_cast<cudaStream_t>(stream));
+  const int st = set_argmax(prm, am_index, token, value, state);
+  if (st != BQG_OK) return st;
+  return launch_gemv<BQG_MAX_BATCH>(prm, total_rows, static_cast<cudaStream_t>(stream));
+}
+}  // namespace bqg
+
+extern "C" int qgemv(int fmt, const void* W, const float* x, float* y, int rows, int cols, void* stream) {
+  return bqg::qgemv_impl(fmt, W, x, y, rows, cols, nullptr, nullptr, nullptr, stream);
+}
+
+extern "C" int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream) {
+  return bqg::qgemv_batched_impl(descs, n, -1, nullptr, nullptr, nullptr, stream);
+}
+
+extern "C" int qgemv_argmax(int fmt, const void* W, const float* x, float* y, int rows, int cols, int32_t* token,
+                            float* max_value, unsigned long long* state, void* stream) {
+  if (token == nullptr || state == nullptr) return BQG_ERR_ARG;
+  return bqg::qgemv_impl(fmt, W, x, y, rows, cols, token, max_value, state, stream);
+}
+
+extern "C" int qgemv_batched_argmax(const bqg_gemv_desc* descs, int n, int argmax_index, int32_t* token,
+                                    float* max_value, unsigned long long* state, void* stream) {
+  if (token == nullptr || state == nullptr) return BQG_ERR_ARG;
+  return bqg::qgemv_batched_impl(descs, n, argmax_index, token, max_value, state, stream);
 }

@@ -144,6 +144,27 @@ typedef struct {
 
 BQG_API int qgemv_batched(const bqg_gemv_desc* descs, int n, void* stream);
 
+/* ---------------------------------------------------------------- LM head with the greedy token
+ * qgemv_argmax, qgemv_batched_argmax: the same GEMVs as qgemv / qgemv_batched, and in the same
+ * launch the greedy token of one output vector: *token = the index of the largest value of y
+ * (of descriptor argmax_index), values compared as IEEE floats (-0.0 == +0.0), an exact tie
+ * going to the lower index; *max_value (optional) = that value.  The token is the argmax of the
+ * fp32 y the call writes, bit for bit.
+ *   Source: Camelid README, "At a glance" (the Apple Silicon path: GPU decode with on-GPU greedy
+ *   sampling) and "Supported models" (the first token is the argmax of the head's logits).
+ *   token      device int32 [1].   max_value  device fp32 [1], or NULL.
+ *   state      device, 2 x uint64 (16 bytes, 8-byte aligned) of working state: zero it once
+ *              before the first call (cudaMemset); every call that completes leaves it zero again.
+ *              Calls sharing a state must be ordered (one stream); after a device error
+ *              (bqg_device_errors) zero it again.
+ *   Each CTA reduces the rows it wrote, then one 64-bit atomicMax per CTA merges them and the
+ *   last CTA to finish writes the token: no extra launch, no extra pass over y.
+ *   Finite y values are a precondition. */
+BQG_API int qgemv_argmax(int fmt, const void* W, const float* x, float* y, int rows, int cols, int32_t* token,
+                         float* max_value, unsigned long long* state, void* stream);
+BQG_API int qgemv_batched_argmax(const bqg_gemv_desc* descs, int n, int argmax_index, int32_t* token,
+                                 float* max_value, unsigned long long* state, void* stream);
+
 /* ---------------------------------------------------------------- a11: prefill-chunk GEMM
  * qgemm_prefill: Y = X W^T with fp16 activations and Q4_0 weights on the tcgen05 tensor
  * cores (fp16 operands, fp32 accumulation in tensor memory, fp16 output, round to nearest).

@@ -5,7 +5,7 @@ Sources (page, section):
   rows quantized Q8_0; Camelid README, "Gemma 4" (Q8_0 projection GEMVs).
 * Q4_0 — Camelid README, "Gemma 4" (Q4_0 projections decoded on the GPU by
   parity-gated GEMVs) and "Experimental lanes" (per-kernel q4_0 GEMV unit tests).
-* packed int4 with a per-row scale — colibri wiki summary, "구현 범위"
+* packed int4 and packed int2 with a per-row scale — colibri wiki summary, "구현 범위"
   (int8 / packed int4 / packed int2 quantization with per-row scale).
 
 The pages name the formats but print no byte layout.  Readings taken (each pinned
@@ -16,6 +16,9 @@ by a test under tests/):
 * i4_row: row r is cols/2 bytes, element 2j in the low nibble of byte j, nibbles are
   two's complement (-8..7); after all rows, zero padding to a 16-byte boundary, then
   one little-endian fp32 scale per row; y_r = s_r * sum_i q_ri x_i.
+* i2_row: row r is cols/4 bytes, element 4j+k in bits 2k..2k+1 of byte j (lowest bits first),
+  two's complement (0b00 = 0, 0b01 = 1, 0b10 = -2, 0b11 = -1); after all rows, zero padding to a
+  16-byte boundary, then one little-endian fp32 scale per row; y_r = s_r * sum_i q_ri x_i.
 * Rows are stored one after another; row r holds its cols/32 blocks in order.
 
 This module is test infrastructure: only tests, the smoke check and the
@@ -25,7 +28,7 @@ from __future__ import annotations
 
 import numpy as np
 
-FMT_Q8_0, FMT_Q4_0, FMT_I4_ROW = 1, 2, 3
+FMT_Q8_0, FMT_Q4_0, FMT_I4_ROW, FMT_I2_ROW = 1, 2, 3, 4
 QK = 32  # weights per block
 
 
@@ -75,6 +78,23 @@ def i4_row_decode(W: np.ndarray, rows: int, cols: int):
     return q, s
 
 
+def i2_row_scale_offset(rows: int, cols: int) -> int:
+    return (rows * (cols // 4) + 15) // 16 * 16
+
+
+def i2_row_decode(W: np.ndarray, rows: int, cols: int):
+    """Split an i2_row matrix into signed 2-bit values q[rows, cols] in -2..1 and fp32 scales s[rows]."""
+    W = np.asarray(W, dtype=np.uint8)
+    packed = W[: rows * (cols // 4)].reshape(rows, cols // 4).astype(np.int64)
+    u = np.empty((rows, cols), dtype=np.int64)
+    for k in range(4):                            # element 4j+k: bits 2k..2k+1 of byte j
+        u[:, k::4] = (packed >> (2 * k)) & 0x3
+    q = np.where(u >= 2, u - 4, u)                # two's complement
+    off = i2_row_scale_offset(rows, cols)
+    s = W[off: off + 4 * rows].view("<f4").astype(np.float64)
+    return q, s
+
+
 def dequantize(fmt: int, W: np.ndarray, rows: int, cols: int) -> np.ndarray:
     """Every weight as a float64 value (exact: an fp16 or fp32 scale times a small integer)."""
     if fmt == FMT_Q8_0:
@@ -86,6 +106,9 @@ def dequantize(fmt: int, W: np.ndarray, rows: int, cols: int) -> np.ndarray:
     if fmt == FMT_I4_ROW:
         q, s = i4_row_decode(W, rows, cols)
         return s[:, None] * q
+    if fmt == FMT_I2_ROW:
+        q, s = i2_row_decode(W, rows, cols)
+        return s[:, None] * q
     raise ValueError(f"unknown format {fmt}")
 
 
@@ -94,7 +117,7 @@ def qgemv(fmt: int, W: np.ndarray, x: np.ndarray, rows: int, cols: int) -> np.nd
 
     Q8_0:  y_r = sum_b d_rb * sum_i q_rbi * x_{32b+i}
     Q4_0:  y_r = sum_b d_rb * sum_i (q_rbi - 8) * x_{32b+i}
-    i4_row: y_r = s_r * sum_i q_ri * x_i
+    i4_row, i2_row: y_r = s_r * sum_i q_ri * x_i
     """
     x = np.asarray(x, dtype=np.float64).reshape(cols)
     if fmt in (FMT_Q8_0, FMT_Q4_0):
@@ -109,6 +132,9 @@ def qgemv(fmt: int, W: np.ndarray, x: np.ndarray, rows: int, cols: int) -> np.nd
         return (d * inner).sum(axis=1)
     if fmt == FMT_I4_ROW:
         q, s = i4_row_decode(W, rows, cols)
+        return s * (q.astype(np.float64) @ x)
+    if fmt == FMT_I2_ROW:
+        q, s = i2_row_decode(W, rows, cols)
         return s * (q.astype(np.float64) @ x)
     raise ValueError(f"unknown format {fmt}")
 
@@ -126,12 +152,13 @@ def qgemv_rows(fmt: int, W: np.ndarray, x: np.ndarray, rows: int, cols: int, sel
         elif fmt == FMT_Q4_0:
             rb = (cols // QK) * 18
             out.append(qgemv(fmt, W[r * rb:(r + 1) * rb], x, 1, cols)[0])
-        elif fmt == FMT_I4_ROW:
-            rb = cols // 2
-            off = i4_row_scale_offset(rows, cols)
-            one = np.zeros(i4_row_scale_offset(1, cols) + 4, dtype=np.uint8)
+        elif fmt in (FMT_I4_ROW, FMT_I2_ROW):
+            rb = cols // 2 if fmt == FMT_I4_ROW else cols // 4
+            sofs = i4_row_scale_offset if fmt == FMT_I4_ROW else i2_row_scale_offset
+            off = sofs(rows, cols)
+            one = np.zeros(sofs(1, cols) + 4, dtype=np.uint8)
             one[:rb] = W[r * rb:(r + 1) * rb]
-            soff = i4_row_scale_offset(1, cols)
+            soff = sofs(1, cols)
             one[soff:soff + 4] = W[off + 4 * r: off + 4 * r + 4]
             out.append(qgemv(fmt, one, x, 1, cols)[0])
         else:

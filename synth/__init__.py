@@ -8,6 +8,8 @@ byte formats the method consumes:
 * ``q4_0``  : rows x (cols/32) blocks of 18 bytes ``{fp16 d; uint8 qs[16]}``
 * ``i4_row``: rows x (cols/2) packed bytes, zero padding to a 16-byte boundary,
   then ``rows`` little-endian fp32 scales.
+* ``i2_row``: rows x (cols/4) packed bytes (four 2-bit values per byte), zero padding to a
+  16-byte boundary, then ``rows`` little-endian fp32 scales.
 
 Randomness comes from a counter-based generator: every 32-bit word is a pure
 function of ``(seed, stream, index)``, so any tensor (or any single expert of a
@@ -133,7 +135,7 @@ def normal_f16(seed: int, stream: int, n: int, std: float = 1.0) -> torch.Tensor
 # ---------------------------------------------------------------- block layouts
 Q8_0_BLOCK = 34
 Q4_0_BLOCK = 18
-FMT_Q8_0, FMT_Q4_0, FMT_I4_ROW = 1, 2, 3
+FMT_Q8_0, FMT_Q4_0, FMT_I4_ROW, FMT_I2_ROW = 1, 2, 3, 4
 
 
 def weight_bytes(fmt: int, rows: int, cols: int) -> int:
@@ -144,12 +146,20 @@ def weight_bytes(fmt: int, rows: int, cols: int) -> int:
         return rows * (cols // 32) * Q4_0_BLOCK
     if fmt == FMT_I4_ROW:
         return i4_row_scale_offset(rows, cols) + 4 * rows
+    if fmt == FMT_I2_ROW:
+        return i2_row_scale_offset(rows, cols) + 4 * rows
     raise ValueError(f"unknown format {fmt}")
 
 
 def i4_row_scale_offset(rows: int, cols: int) -> int:
     """Byte offset of the fp32 row scales inside an i4_row matrix (packed data padded to 16 B)."""
     packed = rows * (cols // 2)
+    return (packed + 15) // 16 * 16
+
+
+def i2_row_scale_offset(rows: int, cols: int) -> int:
+    """Byte offset of the fp32 row scales inside an i2_row matrix (packed data padded to 16 B)."""
+    packed = rows * (cols // 4)
     return (packed + 15) // 16 * 16
 
 
@@ -201,6 +211,24 @@ def i4_row_matrix(rows: int, cols: int, seed: int, name: str, device="cpu",
     return out
 
 
+def i2_row_matrix(rows: int, cols: int, seed: int, name: str, device="cpu",
+                  s_range=(1e-3, 1e-2), r0: int = 0, r1: Optional[int] = None) -> torch.Tensor:
+    """i2_row matrix bytes: uniformly random bytes (four independent 2-bit values each),
+    zero padding to 16 B, then fp32 row scales ~ U[s_range].
+    With r0/r1, only rows r0..r1-1 of the same matrix (as a standalone matrix)."""
+    assert cols % 4 == 0
+    r1 = rows if r1 is None else r1
+    n = r1 - r0
+    s = stream_id(name)
+    rb = cols // 4
+    packed = n * rb
+    off = i2_row_scale_offset(n, cols)
+    out = torch.zeros(off + 4 * n, dtype=torch.uint8, device=device)
+    out[:packed] = random_bytes(seed, s ^ 0x2, packed, device=device, start=r0 * rb)
+    out[off:] = uniform_f32(seed, s ^ 0x1, n, *s_range, device=device, start=r0).view(torch.uint8)
+    return out
+
+
 def matrix(fmt: int, rows: int, cols: int, seed: int, name: str, device="cpu",
            r0: int = 0, r1: Optional[int] = None) -> torch.Tensor:
     if fmt == FMT_Q8_0:
@@ -209,4 +237,6 @@ def matrix(fmt: int, rows: int, cols: int, seed: int, name: str, device="cpu",
         return q4_0_matrix(rows, cols, seed, name, device, r0=r0, r1=r1)
     if fmt == FMT_I4_ROW:
         return i4_row_matrix(rows, cols, seed, name, device, r0=r0, r1=r1)
+    if fmt == FMT_I2_ROW:
+        return i2_row_matrix(rows, cols, seed, name, device, r0=r0, r1=r1)
     raise ValueError(f"unknown format {fmt}")

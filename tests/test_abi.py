@@ -32,7 +32,8 @@ def test_header_declares_the_api():
     names = declared_functions()
     for want in ["qgemv", "qgemv_batched", "qgemm_prefill", "moe_router_logits", "moe_router_topk",
                  "moe_workspace_size", "moe_forward", "moe_forward_noalloc", "bqg_status_string", "bqg_weight_bytes",
-                 "bqg_device_errors", "bqg_version", "bqg_selftest_wait_timeout"]:
+                 "bqg_device_errors", "bqg_version", "bqg_selftest_wait_timeout", "qgemv_argmax",
+                 "qgemv_batched_argmax"]:
         assert want in names
 
 
@@ -233,3 +234,18 @@ def test_moe_path_argument_errors(L):
     assert L.lib().moe_forward(ctypes.byref(c), A, A, A, A, 16, A, 1 << 30, None) == -3
     c.path = 0
     assert L.lib().moe_workspace_size(ctypes.byref(c), 16) > 0
+
+
+def test_argmax_argument_errors(L):
+    f = L.lib().qgemv_argmax
+    A = 0x10000
+    assert f(2, A, A, A, 4, 32, None, None, A, None) == -1          # no token pointer
+    assert f(2, A, A, A, 4, 32, A, None, None, None) == -1          # no state
+    assert f(2, A, A, A, 4, 32, A, None, A + 4, None) == -4         # state not 8-byte aligned
+    assert f(2, A, A, A, 4, 32, A + 2, None, A, None) == -4         # token not 4-byte aligned
+    g = L.lib().qgemv_batched_argmax
+    D = (L.GemvDesc * 3)()
+    for d in D:
+        d.fmt, d.rows, d.cols, d.W, d.x, d.y = 2, 4, 32, A, A, A
+    assert g(D, 3, 3, A, None, A, None) == -1                       # index outside the batch
+    assert g(D, 3, -1, A, None, A, None) == -1

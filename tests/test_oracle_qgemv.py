@@ -253,3 +253,92 @@ def test_i4_row_scale_factors_out():
     W2[off:off + 4 * rows] = np.ones(rows, dtype="<f4").view(np.uint8)
     y_int = oq.qgemv(oq.FMT_I4_ROW, W2, x, rows, cols)
     np.testing.assert_allclose(y, s.astype(np.float64) * y_int, rtol=1e-14)
+
+
+# ---------------------------------------------------------------- packed int2 with a per-row scale
+def _i2_pack_row(vals):
+    """Bytes of one row of 2-bit two's-complement values, element 4j+k in bits 2k..2k+1 of byte j
+    (written out by shifting each value into place, independently of the oracle's decoder)."""
+    out = bytearray()
+    for j in range(len(vals) // 4):
+        b = 0
+        for k in range(4):
+            b |= (int(vals[4 * j + k]) & 0x3) << (2 * k)
+        out.append(b)
+    return bytes(out)
+
+
+def test_i2_row_golden_probes(golden_dir):
+    g = _load(golden_dir, "i2_row_hand.json")
+    for p in g["probes"]:
+        raw = bytes([p["byte"]]) + bytes(15) + struct.pack("<f", 1.0)
+        W = np.frombuffer(raw, dtype=np.uint8)
+        for j, want in enumerate(p["values"]):
+            x = np.zeros(4)
+            x[j] = 1.0
+            assert oq.qgemv(oq.FMT_I2_ROW, W, x, 1, 4)[0] == want, (p, j)
+    h = g["hand_row"]
+    raw = bytes(h["bytes"]) + bytes(12) + struct.pack("<f", h["scale"])
+    y = oq.qgemv(oq.FMT_I2_ROW, np.frombuffer(raw, dtype=np.uint8), np.ones(16), 1, 16)
+    assert y[0] == h["y"]
+
+
+def test_i2_row_random_tiny_matches_exact_rational():
+    rng = np.random.default_rng(21)
+    rows, cols = 6, 16
+    vals = rng.integers(-2, 2, (rows, cols))
+    s = rng.uniform(-1, 1, rows).astype(np.float32)
+    packed = b"".join(_i2_pack_row(vals[r]) for r in range(rows))
+    off = (len(packed) + 15) // 16 * 16
+    raw = packed + bytes(off - len(packed)) + s.astype("<f4").tobytes()
+    x = rng.standard_normal(cols).astype(np.float32)
+    got = oq.qgemv(oq.FMT_I2_ROW, np.frombuffer(raw, dtype=np.uint8), x, rows, cols)
+    for r in range(rows):
+        want = Fraction(float(s[r])) * sum(int(vals[r, i]) * Fraction(float(x[i])) for i in range(cols))
+        assert abs(Fraction(got[r]) - want) <= Fraction(1, 10 ** 9) * (1 + abs(want))
+
+
+def test_i2_row_unit_probes_pin_the_order():
+    """x = e_j returns s_r * q_rj for every j of a random row."""
+    rng = np.random.default_rng(23)
+    cols = 64
+    vals = rng.integers(-2, 2, cols)
+    raw = _i2_pack_row(vals) + bytes(0) + struct.pack("<f", 0.25)
+    for j in range(cols):
+        x = np.zeros(cols)
+        x[j] = 1.0
+        assert oq.qgemv(oq.FMT_I2_ROW, np.frombuffer(raw, dtype=np.uint8), x, 1, cols)[0] == 0.25 * vals[j]
+
+
+def test_i2_row_unit_scale_is_integer_matvec_and_scale_factors_out():
+    import synth
+    rows, cols = 9, 128
+    W = synth.i2_row_matrix(rows, cols, 4, "i2sc").numpy().copy()
+    x = synth.normal(4, 5, cols).numpy()
+    off = oq.i2_row_scale_offset(rows, cols)
+    s = W[off:off + 4 * rows].view("<f4").copy().astype(np.float64)
+    W1 = W.copy()
+    W1[off:off + 4 * rows] = np.ones(rows, dtype="<f4").view(np.uint8)
+    xi = np.arange(cols, dtype=np.float64) % 7 - 3
+    # naive integer matvec from the raw bytes by explicit bit extraction
+    rb = cols // 4
+    want = []
+    for r in range(rows):
+        acc = 0
+        for i in range(cols):
+            c = (int(W[r * rb + i // 4]) >> (2 * (i % 4))) & 3
+            acc += (c - 4 if c >= 2 else c) * int(xi[i])
+        want.append(acc)
+    assert oq.qgemv(oq.FMT_I2_ROW, W1, xi, rows, cols).tolist() == want
+    np.testing.assert_allclose(oq.qgemv(oq.FMT_I2_ROW, W, x, rows, cols),
+                               s * oq.qgemv(oq.FMT_I2_ROW, W1, x, rows, cols), rtol=1e-14)
+    np.testing.assert_allclose(oq.dequantize(oq.FMT_I2_ROW, W, rows, cols) @ x,
+                               oq.qgemv(oq.FMT_I2_ROW, W, x, rows, cols), rtol=1e-12, atol=1e-12)
+
+
+def test_i2_row_expert_size():
+    """A GLM-like expert (gate, up 2048 x 6144, down 6144 x 2048) in packed int2: a quarter byte per
+    weight plus fp32 row scales."""
+    import synth
+    b = 2 * synth.weight_bytes(oq.FMT_I2_ROW, 2048, 6144) + synth.weight_bytes(oq.FMT_I2_ROW, 6144, 2048)
+    assert b == 3 * 2048 * 6144 // 4 + 4 * (2048 + 2048 + 6144)
