@@ -3,9 +3,10 @@
 
 Headline workload (one "step"): one decode step's projections at TinyLlama-1.1B shape,
 batch 1 — 22 layers of Q4_0 q/o 2048x2048, k/v 256x2048, gate/up 5632x2048, down
-2048x5632 plus a Q8_0 LM head 32000x2048 (614,629,376 weight bytes), all streamed by ONE
-qgemv_batched launch.  Inputs are seeded synthetic tensors resident in HBM; the weights of
-a step (615 MB) are larger than L2 (126 MB), so no flush is needed between steps.
+2048x5632 plus a Q8_0 LM head 32000x2048 (614,629,376 weight bytes) and the greedy token
+(argmax of the head's logits), all in ONE qgemv_batched_argmax launch.  Inputs are seeded
+synthetic tensors resident in HBM; the weights of a step (615 MB) are larger than L2
+(126 MB), so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -80,22 +81,19 @@ def kernel_source_hash() -> str:
 
 
 def committed_traffic():
-    """Per-launch DRAM bytes of the headline kernel from the committed ncu summary, or None
-    when the summary is missing or was taken on a different kernel source."""
-    p = os.path.join(ROOT, "profiles", "k_qgemv_tinyllama_decode.md")
+    """Per-launch DRAM bytes of the headline kernel from the committed ncu record
+    (profiles/k_qgemv_tinyllama_decode.json), or None when it is missing or was taken on a
+    different kernel source."""
+    p = os.path.join(ROOT, "profiles", "k_qgemv_tinyllama_decode.json")
     if not os.path.exists(p):
         return None
-    vals = {}
     with open(p) as f:
-        for line in f:
-            if ":" in line and line.startswith("- "):
-                k, v = line[2:].split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_hash") != kernel_source_hash():
+        rec = json.load(f)
+    if rec.get("kernel_source_hash") != kernel_source_hash():
         return None
     try:
-        return int(vals["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return int(rec["traffic_bytes_per_launch"])
+    except (KeyError, ValueError, TypeError):
         return None
 
 
@@ -220,9 +218,9 @@ def max_over_ranks(v: float, world: int) -> float:
 
 
 # ---------------------------------------------------------------- CPU oracle leg
-def oracle_sample(seconds: float, seed: int):
-    """Time the float64 oracle (single thread) on whole matrices of the decode step, in
-    execution order, until the time budget is used.  Returns (bytes, seconds, n_matrices)."""
+def oracle_sample(seconds: float, seed: int, threads: int = 1):
+    """Time the float64 oracle (on `threads` BLAS threads) on whole matrices of the decode step,
+    in execution order, until the time budget is used.  Returns (bytes, seconds, n_matrices)."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
@@ -233,7 +231,7 @@ def oracle_sample(seconds: float, seed: int):
     specs = wl.decode_step_specs()
     done_bytes, t_total, n = 0, 0.0, 0
     xs = {}
-    with threadpool_limits(1):
+    with threadpool_limits(threads):
         for s in specs:
             if s.x_name not in xs:
                 xs[s.x_name] = wl.x_host(specs, s.x_name, seed).numpy().astype(np.float64)
@@ -295,19 +293,87 @@ def run_reference(args, world, rank):
         tot_t = sum(one_pass() for _ in range(args.steps))
     pass_bytes = sum(synth.weight_bytes(s.fmt, r1 - r0, s.cols) + 4 * (r1 - r0 + s.cols) for s, r0, r1, _ in sample)
     gbs = pass_bytes * args.steps / tot_t / 1e9
-    step_bytes = sum(synth_bytes(s) for s in specs)
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_bytes / (gbs * 1e9) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(),
         "cpu_baseline": {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"float64 oracle, single thread, the first {pass_bytes / 1e6:.2f} MB of the "
-                                   f"decode step's matrices in execution order ({len(sample)} row chunks) per "
-                                   f"step; ms_per_step extrapolates to the whole 614.6 MB step"},
+                         "sample": f"float64 oracle, single thread: each timed step is the first "
+                                   f"{pass_bytes / 1e6:.2f} MB of the decode step's matrices in execution order "
+                                   f"({len(sample)} row chunks); ms_per_step is the time of that sample"},
         "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def oracle_moe_sample(seed: int, threads: int):
+    """The float64 oracle on one Gemma-like MoE layer at one token (router, top-8, 8 routed
+    experts and the shared expert): seconds and algorithmic bytes of that layer."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import synth
+    from oracle import moe as om
+    from synth import workloads as wl
+    spec = wl.GEMMA_MOE
+    x = wl.moe_tokens(spec, seed, 1).numpy().astype(np.float64)
+    R = synth.normal_f32(seed, synth.stream_id(f"{spec.name}/L0/router"), spec.n_experts * spec.hidden,
+                         std=0.02).view(spec.n_experts, spec.hidden).numpy()
+    experts = {}
+
+    def expert(e):
+        if e not in experts:
+            experts[e] = om.Expert(spec.expert_fmt, *[wl.expert_matrix(spec, seed, 0, e, w).numpy()
+                                                      for w in ("gate", "up", "down")])
+        return experts[e]
+    shared = om.Expert(spec.shared_fmt, *[wl.shared_matrix(spec, seed, 0, w).numpy() for w in ("gate", "up", "down")])
+    layer = om.Layer(spec.n_experts, spec.top_k, spec.hidden, spec.inter, spec.act, expert, shared, spec.shared_inter)
+    idx, _ = om.router_topk(om.router_logits(R, x), spec.top_k)
+    for e in idx.reshape(-1):
+        expert(int(e))                          # generate the touched experts' bytes outside the timing
+    with threadpool_limits(threads):
+        t0 = time.perf_counter()
+        idx, w = om.router_topk(om.router_logits(R, x), spec.top_k)
+        om.moe_layer(layer, x, idx, w)
+        t = time.perf_counter() - t0
+    nbytes = 4 * spec.n_experts * spec.hidden + sum(spec.shared_bytes(m) for m in ("gate", "up", "down")) + \
+        8 * sum(spec.mat_bytes(m) for m in ("gate", "up", "down"))
+    return t, nbytes
+
+
+def oracle_prefill_sample(seed: int, threads: int):
+    """The float64 oracle on the prefill chunk at N = 1024 (128 x 1024 x 4096): seconds, FLOPs."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import synth
+    from oracle import prefill as op
+    t, n, k = 128, 1024, 4096
+    W = synth.q4_0_matrix(n, k, seed, f"prefill/N{n}/copy0").numpy()
+    X = synth.normal_f16(seed, synth.stream_id("prefill/X"), t * k).view(t, k).numpy()
+    with threadpool_limits(threads):
+        t0 = time.perf_counter()
+        op.prefill(2, W, X, n, k)
+        dt = time.perf_counter() - t0
+    return dt, 2.0 * t * n * k
+
+
+def cpu_baselines(args):
+    """The oracle on one host core and on all of them (decode-step GB/s), plus one MoE layer and
+    the N = 1024 prefill chunk."""
+    cores = os.cpu_count() or 1
+    out = {}
+    for threads in (1, cores):
+        b, t, n = oracle_sample(args.cpu_seconds / 2, args.seed, threads)
+        out[threads] = {"value": b / t / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+                        "sample": f"float64 oracle on {threads} thread(s), the first {n} whole matrices of the "
+                                  f"decode step ({b / 1e6:.0f} MB in {t:.1f} s)"}
+    mt, mb = oracle_moe_sample(args.seed, cores)
+    pt, pf = oracle_prefill_sample(args.seed, cores)
+    extra = {"moe_gemma_T1": {"us_per_layer": mt * 1e6, "GB/s": mb / mt / 1e9, "cores": cores},
+             "prefill_N1024": {"us_per_call": pt * 1e6, "GFLOP/s": pf / pt / 1e9, "cores": cores}}
+    return out[1], out[cores], extra
 
 
 def synth_bytes(s):
@@ -317,8 +383,9 @@ def synth_bytes(s):
 
 def workload_config():
     return {"workload": "tinyllama_decode: 22 layers x Q4_0 (q,o 2048x2048; k,v 256x2048; gate,up 5632x2048; "
-                        "down 2048x5632) + Q8_0 LM head 32000x2048, batch 1, x ~ N(0,1)",
-            "weight_bytes_per_step": 614629376, "launch": "one qgemv_batched launch per step",
+                        "down 2048x5632) + Q8_0 LM head 32000x2048 + greedy token (argmax of the head), batch 1, "
+                        "x ~ N(0,1)",
+            "weight_bytes_per_step": 614629376, "launch": "one qgemv_batched_argmax launch per step",
             "l2": "inputs larger than L2 (615 MB of weights per step vs 126 MB L2); no flush",
             "parallelism": "replicas"}
 
@@ -333,12 +400,17 @@ def time_decode_step(args, world, dev):
     specs = wl.decode_step_specs()
     W = wl.build_gemv_workload(specs, seed=args.seed, device=dev)
     batch = bqg.GemvBatch(W.items())
+    greedy = bqg.ArgmaxState(dev)
+    head = len(specs) - 1
+
+    def step():
+        batch.run(argmax=(head, greedy))
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(physical_gpu(torch.cuda.current_device()))
     clocks.start()
     clocks.wait_first()
     for _ in range(max(3, args.warmup)):
-        batch.run()
+        step()
     torch.cuda.synchronize()
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -351,7 +423,7 @@ def time_decode_step(args, world, dev):
     t_begin.record(stream)
     for i in range(args.steps):
         starts[i].record(stream)
-        batch.run()
+        step()
         ends[i].record(stream)
     t_end.record(stream)
     torch.cuda.nvtx.range_pop()
@@ -362,30 +434,52 @@ def time_decode_step(args, world, dev):
     launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     total_ms = max_over_ranks(total_ms, world)
 
-    # end to end through the public API: pinned host x -> device, step, device y -> pinned host
+    # the same step without the greedy token (the cost of the fused argmax)
+    n_plain = max(20, min(args.steps, 500))
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(n_plain):
+        batch.run()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    plain_ms = p0.elapsed_time(p1) / n_plain
+
+    # end to end through the public API: pinned host x -> device, step, greedy token (and its
+    # logit) -> pinned host; the H2D and D2H legs are also timed on their own
     x_host = torch.empty(W.x_all.shape, dtype=torch.float32, pin_memory=True)
     x_host.copy_(W.x_all.cpu())
-    y_host = torch.empty(W.y_all.shape, dtype=torch.float32, pin_memory=True)
+    tok_host = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    val_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        W.x_all.copy_(x_host, non_blocking=True)
+        step()
+        tok_host.copy_(greedy.token, non_blocking=True)
+        val_host.copy_(greedy.value, non_blocking=True)
     e_steps = max(10, min(args.steps, 500))
     for _ in range(3):
-        W.x_all.copy_(x_host, non_blocking=True)
-        batch.run()
-        y_host.copy_(W.y_all, non_blocking=True)
+        e2e_step()
     torch.cuda.synchronize()
     barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    ev[0].record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    ev[1].record(stream)
     for _ in range(e_steps):
         W.x_all.copy_(x_host, non_blocking=True)
-        batch.run()
-        y_host.copy_(W.y_all, non_blocking=True)
-    e1.record(stream)
+    ev[2].record(stream)
+    for _ in range(e_steps):
+        tok_host.copy_(greedy.token, non_blocking=True)
+        val_host.copy_(greedy.value, non_blocking=True)
+    ev[3].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e_steps
+    e2e_ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world) / e_steps
+    legs = {"h2d_us": ev[1].elapsed_time(ev[2]) * 1e3 / e_steps, "d2h_us": ev[2].elapsed_time(ev[3]) * 1e3 / e_steps}
+    assert int(tok_host.item()) == int(torch.argmax(W.y(head)).item())
     barrier(world)
-    return dict(W=W, total_ms=total_ms, launch_ms=launch_ms, clocks=clk, e2e_ms=e2e_ms,
-                h2d=x_host.numel() * 4, d2h=y_host.numel() * 4)
+    return dict(W=W, total_ms=total_ms, launch_ms=launch_ms, clocks=clk, e2e_ms=e2e_ms, plain_ms=plain_ms,
+                legs=legs, h2d=x_host.numel() * 4, d2h=4 + 4)
 
 
 def time_single_q8_0(dev, seed):
@@ -562,6 +656,44 @@ def time_moe_glm(dev, seed, peak):
     return out
 
 
+def time_moe_glm_i2(dev, seed, peak, layers=8):
+    """The GLM-like stack with packed int2 experts (a quarter byte per weight): 8 resident layers
+    of 256 experts (19.3 GB), given N(0,1) logits, top-8, run back to back; T = 1, 8, 64."""
+    import dataclasses
+
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    spec = dataclasses.replace(wl.GLM_MOE, name="glm_i2", expert_fmt=bqg.I2_ROW)
+    Ts = [wl.build_moe_layer(spec, seed, layer=l, device=dev) for l in range(layers)]
+    Ls = [moe_device_layer(T) for T in Ts]
+    expert_bytes = sum(spec.mat_bytes(w) for w in ("gate", "up", "down"))
+    resident = sum(T.gate.numel() + T.up.numel() + T.down.numel() for T in Ts)
+    out = {"workload": f"glm_moe_i2: {layers} layers x 256 packed-int2 experts (hidden 6144, SwiGLU 2048), "
+                       f"top-8 of given N(0,1) logits, layers back to back; {resident / 1e9:.1f} GB resident"}
+    for T in (1, 8, 64):
+        logits = [wl.moe_logits(spec, seed, l, T).to(dev) for l in range(len(Ls))]
+        idx = [torch.empty(T, spec.top_k, dtype=torch.int32, device=dev) for _ in Ls]
+        w = [torch.empty(T, spec.top_k, device=dev) for _ in Ls]
+        xs = [wl.moe_tokens(spec, seed, T, layer=l).to(dev) for l in range(len(Ls))]
+        ys = [torch.empty(T, spec.hidden, device=dev) for _ in Ls]
+        ws = torch.empty(bqg.moe_workspace_size(Ls[0], T), dtype=torch.uint8, device=dev)
+
+        def fn():
+            for l in range(len(Ls)):
+                bqg.moe_router_topk(logits[l], spec.top_k, idx[l], w[l])
+                bqg.moe_forward(Ls[l], xs[l], idx[l], w[l], ys[l], ws)
+        us = graph_us(fn, reps=5) / len(Ls)
+        distinct = sum(int(torch.unique(i).numel()) for i in idx) / len(Ls)
+        nbytes = distinct * expert_bytes + 8 * T * spec.hidden + 4 * T * spec.n_experts
+        out[f"T{T}"] = {"us_per_layer": us, "distinct_experts": distinct, "bytes_per_layer": nbytes,
+                        "GB/s": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak}
+    del Ts, Ls
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
     assert torch.cuda.is_available(), "bench.py --impl ours needs a CUDA device"
@@ -585,19 +717,24 @@ def run_ours(args, world, rank, local):
         extras["moe_gemma"] = time_moe_gemma(dev, args.seed, peak)
         if not args.no_glm:
             extras["moe_glm"] = time_moe_glm(dev, args.seed, peak)
+            extras["moe_glm_i2"] = time_moe_glm_i2(dev, args.seed, peak)
+    extras["decode_step_without_greedy_token"] = {
+        "ms_per_step": r["plain_ms"], "GB/s": step_bytes / (r["plain_ms"] * 1e-3) / 1e9,
+        "argmax_cost_frac": r["launch_ms"] / r["plain_ms"] - 1.0}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        b, t, n = oracle_sample(args.cpu_seconds, args.seed)
-        cpu = {"value": b / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"float64 oracle, single thread, the first {n} whole matrices of the decode step "
-                         f"({b / 1e6:.0f} MB in {t:.1f} s)"}
+        cpu, cpu_all, cpu_extra = cpu_baselines(args)
+        cpu = dict(cpu, all_cores=cpu_all)
+        extras["cpu_oracle"] = cpu_extra
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "q4_0/q8_0 weights x fp32 activations, fp32 accumulate",
+            "vs_baseline": None,
+            "dtype": "q4_0/q8_0 weights x fp32 activations held as 16-bit fixed point per 32/64 values inside "
+                     "the kernel (exact int32 block sums), fp32 accumulate",
             "data": "synthetic", "config": workload_config(),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind, "traffic": committed_traffic(),
@@ -605,7 +742,8 @@ def run_ours(args, world, rank, local):
                          "algorithmic_bytes_per_launch": step_bytes},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_gbs, "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                    "ms_per_step": r["e2e_ms"]},
+                    "ms_per_step": r["e2e_ms"], "legs": r["legs"],
+                    "result": "greedy token and its logit (8 bytes) read back every step"},
             "gpu_launches": args.steps,
             "clocks": r["clocks"],
             "extras": extras,

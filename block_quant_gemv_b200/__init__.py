@@ -27,7 +27,7 @@ __all__ = [
     "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward", "moe_forward_noalloc",
 ]
 
-Q8_0, Q4_0, I4_ROW = 1, 2, 3
+Q8_0, Q4_0, I4_ROW, I2_ROW = 1, 2, 3, 4
 ACT_GELU_TANH, ACT_SILU = 1, 2
 MOE_PATH_AUTO, MOE_PATH_CUDA_CORES, MOE_PATH_TENSOR_CORES = 0, 1, 2
 MOE_TC_MIN_TOKENS, MOE_TC_MIN_PER_EXPERT = 16, 4

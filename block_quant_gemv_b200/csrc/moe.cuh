@@ -132,6 +132,36 @@ __device__ __forceinline__ void quant_seg(const QuantJob& J, long long gs, bool 
     xi[i] = __float2int_rn(xv[i] * inv);
     sum += xi[i];
   }
+  if constexpr (is_i2(KIND)) {
+    // int2 record: h/l word 4w + k holds elements 16w + k + 4b (b = 0..3), the order of the 2-bit
+    // values in bits 2k..2k+1 of weight word w.  Segment m = 2w + half holds b = 2 half, 2 half + 1
+    // of every plane: each lane builds its 16-bit halves, the pair exchanges them, the even lane
+    // stores the h words and the odd lane the l words.
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t hh = (uint32_t(xi[k] >> 8) & 0xFFu) | ((uint32_t(xi[4 + k] >> 8) & 0xFFu) << 8);
+      const uint32_t ll = (uint32_t(xi[k]) & 0xFFu) | ((uint32_t(xi[4 + k]) & 0xFFu) << 8);
+      const uint32_t ph = __shfl_xor_sync(0xffffffffu, hh, 1);
+      const uint32_t pl = __shfl_xor_sync(0xffffffffu, ll, 1);
+      hw[k] = (m & 1) ? (ph | (hh << 16)) : (hh | (ph << 16));
+      lw[k] = (m & 1) ? (pl | (ll << 16)) : (ll | (pl << 16));
+    }
+    int tot = sum;  // all 64 values of the unit: the t ^ 2 = t + 2 offset
+    tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+    tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+    tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+    if (valid) {
+      uint32_t* rec = reinterpret_cast<uint32_t*>(J.dst + unit * xrec_chunks(KIND));
+      const int w = m >> 1;
+      if ((m & 1) == 0) *reinterpret_cast<uint4*>(rec + 4 * w) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      else *reinterpret_cast<uint4*>(rec + NW + 4 * w) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      if (m == 0)
+        *reinterpret_cast<uint4*>(rec + 2 * NW) =
+            make_uint4(uint32_t(-2 * tot), 0u, __float_as_uint(amax * (1.f / 32767.f)), 0u);
+    }
+    return;
+  }
   uint32_t h0, h1, l0, l1;
   if constexpr (is_q8(KIND)) {  // words 2m, 2m+1 = elements 8m..8m+3, 8m+4..8m+7
     h0 = pack_byte(xi[0], xi[1], xi[2], xi[3], 1);
@@ -176,6 +206,7 @@ __device__ __forceinline__ void quant_jobs(const QuantJobs& Q, long long i0, lon
         case kQ8Pair: quant_seg<kQ8Pair>(J, i, valid); break;
         case kQ8One: quant_seg<kQ8One>(J, i, valid); break;
         case kI4x64: quant_seg<kI4x64>(J, i, valid); break;
+        case kI2x64: quant_seg<kI2x64>(J, i, valid); break;
         default: quant_seg<kI4x32>(J, i, valid); break;
       }
     }

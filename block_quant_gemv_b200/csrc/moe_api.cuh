@@ -20,6 +20,7 @@ inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 inline int moe_kind(int fmt, int cols) {
   if (fmt == BQG_Q8_0) return kQ8One;
   if (fmt == BQG_Q4_0) return kQ4One;
+  if (fmt == BQG_I2_ROW) return kI2x64;
   return cols % 64 == 0 ? kI4x64 : kI4x32;
 }
 
@@ -31,6 +32,7 @@ inline MgKernel mg_kernel_ks(int ks) {
     case kQ4One: return k_moe_gemv<KR, kQ4One>;
     case kQ8One: return k_moe_gemv<KR, kQ8One>;
     case kI4x64: return k_moe_gemv<KR, kI4x64>;
+    case kI2x64: return k_moe_gemv<KR, kI2x64>;
     default: return k_moe_gemv<KR, kI4x32>;
   }
 }
@@ -39,12 +41,13 @@ inline MgKernel mg_kernel(int kr, int ks) {
     case kQ4One: return mg_kernel_ks<kQ4One>(ks);
     case kQ8One: return mg_kernel_ks<kQ8One>(ks);
     case kI4x64: return mg_kernel_ks<kI4x64>(ks);
+    case kI2x64: return mg_kernel_ks<kI2x64>(ks);
     default: return mg_kernel_ks<kI4x32>(ks);
   }
 }
 
 inline int mg_row_bytes(int fmt, int cols) {
-  return fmt == BQG_Q8_0 ? cols / 32 * 34 : fmt == BQG_Q4_0 ? cols / 32 * 18 : cols / 2;
+  return fmt == BQG_Q8_0 ? cols / 32 * 34 : fmt == BQG_Q4_0 ? cols / 32 * 18 : fmt == BQG_I2_ROW ? cols / 4 : cols / 2;
 }
 
 // One family of stacked matrices [rows x cols] (expert e at base + e * stride).
@@ -57,7 +60,7 @@ inline MgMat mg_mat(int fmt, const void* base, size_t stride, int rows, int cols
   M.kind = moe_kind(fmt, cols);
   M.row_bytes = mg_row_bytes(fmt, cols);
   M.units = cols / unit_weights(M.kind);
-  M.scale_off = fmt == BQG_I4_ROW ? int((size_t(rows) * M.row_bytes + 15) / 16 * 16) : 0;
+  M.scale_off = (fmt == BQG_I4_ROW || fmt == BQG_I2_ROW) ? int((size_t(rows) * M.row_bytes + 15) / 16 * 16) : 0;
   M.stage_rows = mg_stage_rows(M.units, M.row_bytes);
   M.nstages = (rows + M.stage_rows - 1) / M.stage_rows;
   return M;
@@ -201,7 +204,7 @@ inline size_t moe_ws_total(const bqg_moe_layer* L, int tokens) {
   return need;
 }
 
-inline bool valid_fmt(int f) { return f == BQG_Q8_0 || f == BQG_Q4_0 || f == BQG_I4_ROW; }
+inline bool valid_fmt(int f) { return f == BQG_Q8_0 || f == BQG_Q4_0 || f == BQG_I4_ROW || f == BQG_I2_ROW; }
 
 inline int check_layer(const bqg_moe_layer* L) {
   if (L == nullptr) return BQG_ERR_ARG;
@@ -213,6 +216,7 @@ inline int check_layer(const bqg_moe_layer* L) {
   if (L->path != BQG_MOE_PATH_AUTO && L->path != BQG_MOE_PATH_CUDA_CORES && L->path != BQG_MOE_PATH_TENSOR_CORES)
     return BQG_ERR_ARG;
   if (L->hidden % 32 || L->inter % 32) return BQG_ERR_SHAPE;
+  if (L->expert_fmt == BQG_I2_ROW && (L->hidden % 64 || L->inter % 64)) return BQG_ERR_SHAPE;
   if (L->hidden > kMoeMaxCols || L->inter > kMoeMaxCols) return BQG_ERR_LIMIT;
   if (L->gate == nullptr || L->up == nullptr || L->down == nullptr) return BQG_ERR_ARG;
   if (!aligned(L->gate, 16) || !aligned(L->up, 16) || !aligned(L->down, 16)) return BQG_ERR_ALIGN;
@@ -227,15 +231,18 @@ inline int check_layer(const bqg_moe_layer* L) {
     if (L->s_up == nullptr || L->s_down == nullptr) return BQG_ERR_ARG;
     if (!valid_fmt(L->shared_fmt)) return BQG_ERR_FMT;
     if (L->shared_inter < 1 || L->shared_inter % 32) return BQG_ERR_SHAPE;
+    if (L->shared_fmt == BQG_I2_ROW && (L->hidden % 64 || L->shared_inter % 64)) return BQG_ERR_SHAPE;
     if (L->shared_inter > kMoeMaxCols) return BQG_ERR_LIMIT;
     if (!aligned(L->s_gate, 16) || !aligned(L->s_up, 16) || !aligned(L->s_down, 16)) return BQG_ERR_ALIGN;
   }
   return BQG_OK;
 }
 
-// one attribute cache per kernel instance (4 x 4)
-inline SmemAttrOnce g_moe_attr[16];
-inline int moe_kind_index(int kind) { return kind == kQ4One ? 0 : kind == kQ8One ? 1 : kind == kI4x64 ? 2 : 3; }
+// one attribute cache per kernel instance (5 x 5)
+inline SmemAttrOnce g_moe_attr[25];
+inline int moe_kind_index(int kind) {
+  return kind == kQ4One ? 0 : kind == kQ8One ? 1 : kind == kI4x64 ? 2 : kind == kI2x64 ? 4 : 3;
+}
 
 inline int quant_grid(long long threads, int cap) {
   long long g = (threads + 255) / 256;
@@ -448,7 +455,7 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   {
     const int kr = gate.kind, ks = sh ? s_gate.kind : gate.kind;
     const MgKernel k = mg_kernel(kr, ks);
-    if ((st = g_moe_attr[moe_kind_index(kr) * 4 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
+    if ((st = g_moe_attr[moe_kind_index(kr) * 5 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
       return st;
     if ((st = launch_pdl(k, dim3(info->sm_count), dim3(kGemvThreads), kMgSmemBytes, s, P)) != BQG_OK) return st;
   }
@@ -482,7 +489,7 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   {
     const int kr = down.kind, ks = sh ? s_down.kind : down.kind;
     const MgKernel k = mg_kernel(kr, ks);
-    if ((st = g_moe_attr[moe_kind_index(kr) * 4 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
+    if ((st = g_moe_attr[moe_kind_index(kr) * 5 + moe_kind_index(ks)].ensure(dev, k, kMgSmemBytes)) != BQG_OK)
       return st;
     if ((st = launch_pdl(k, dim3(info->sm_count), dim3(kGemvThreads), kMgSmemBytes, s, D)) != BQG_OK) return st;
   }

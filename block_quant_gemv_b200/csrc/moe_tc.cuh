@@ -628,6 +628,7 @@ inline int tc_row_bytes(int fmt, int cols) {
 // Geometry of one family on the tensor-core path; false when the shape is not supported there
 // (k not a multiple of 64, or rows not a whole number of super-rows).
 inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols, int m_off, TcFam* out) {
+  if (fmt == BQG_I2_ROW) return false;  // the tensor-core path dequantizes Q8_0, Q4_0 and int4 only
   if (cols % 64 != 0 || rows % 32 != 0) return false;
   TcFam F{};
   F.base = static_cast<const uint8_t*>(base);

@@ -57,7 +57,8 @@ enum UnitKind : int {
   kQ4Pair = 2,   // two Q4_0 blocks, 36 bytes, 64 weights
   kQ4One = 3,    // one Q4_0 block, 18 bytes, 32 weights
   kI4x64 = 4,    // 64 int4 weights, 32 bytes (cols % 64 == 0)
-  kI4x32 = 5     // 32 int4 weights, 16 bytes
+  kI4x32 = 5,    // 32 int4 weights, 16 bytes
+  kI2x64 = 6     // 64 int2 weights, 16 bytes (cols % 64 == 0)
 };
 
 struct GemvProb {
@@ -86,6 +87,8 @@ struct GemvParams {
   int n;
   int am_p;                    // problem whose y is reduced to its argmax (greedy token), or -1
   long long total_bytes;
+  int am_ctas;                 // CTAs that hold rows of problem am_p (they alone take part)
+  int am_pad;
   int32_t* am_token;           // argmax index of y[am_p] (ties: the lower index)
   float* am_value;             // its value (may be null)
   unsigned long long* am_state;  // [2]: packed running maximum, CTA completion count (zero between calls)
@@ -120,9 +123,11 @@ __host__ __device__ constexpr int unit_bytes(int kind) {
   return kind == kQ8Pair ? 68 : kind == kQ8One ? 34 : kind == kQ4Pair ? 36 : kind == kQ4One ? 18 : kind == kI4x64 ? 32 : 16;
 }
 __host__ __device__ constexpr int unit_weights(int kind) {
-  return (kind == kQ8Pair || kind == kQ4Pair || kind == kI4x64) ? 64 : 32;
+  return (kind == kQ8Pair || kind == kQ4Pair || kind == kI4x64 || kind == kI2x64) ? 64 : 32;
 }
-__host__ __device__ constexpr bool is_i4(int kind) { return kind == kI4x64 || kind == kI4x32; }
+__host__ __device__ constexpr bool is_i2(int kind) { return kind == kI2x64; }
+// Formats with one fp32 scale per row (int4 and int2): applied to the row's sum by the caller.
+__host__ __device__ constexpr bool is_i4(int kind) { return kind == kI4x64 || kind == kI4x32 || kind == kI2x64; }
 __host__ __device__ constexpr bool is_q8(int kind) { return kind == kQ8Pair || kind == kQ8One; }
 
 // Geometry shared by host and device: warps per row group, groups, rows per stage.
@@ -200,6 +205,21 @@ __device__ __forceinline__ void quantize_unit(const float (&xv)[unit_weights(KIN
       X.l[m] = pack_byte(xi[4 * m], xi[4 * m + 1], xi[4 * m + 2], xi[4 * m + 3], 0);
     }
     X.c0 = X.c1 = 0;
+  } else if constexpr (is_i2(KIND)) {
+    // word 4m + k: elements 16m + k, 16m + 4 + k, 16m + 8 + k, 16m + 12 + k (the 2-bit values in
+    // bits 2k..2k+1 of the four bytes of weight word m); the -2 offset of t ^ 2 = t + 2 goes to c0
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        X.h[4 * m + k] = pack_byte(xi[16 * m + k], xi[16 * m + 4 + k], xi[16 * m + 8 + k], xi[16 * m + 12 + k], 1);
+        X.l[4 * m + k] = pack_byte(xi[16 * m + k], xi[16 * m + 4 + k], xi[16 * m + 8 + k], xi[16 * m + 12 + k], 0);
+      }
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) sum += xi[i];
+    X.c0 = -2 * sum;
+    X.c1 = 0;
   } else {
 #pragma unroll
     for (int m = 0; m < UW / 8; ++m) {
@@ -348,6 +368,34 @@ __device__ __forceinline__ void units_dot(const uint32_t (&u)[NR], const XUnit& 
 #pragma unroll
     for (int n = 0; n < NR; ++n)
       out[n] = X.s * half_bits_to_float(__funnelshift_r(v[n][0], v[n][1], sh[n])) * float(h[n] * 256 + l[n]);
+  } else if constexpr (KIND == kI2x64) {  // int2 with per-row scale (applied by the caller): 4 words
+    uint32_t q[NR][4];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      const uint4 p0 = lds128(u[n]);  // 16-byte aligned
+      q[n][0] = p0.x; q[n][1] = p0.y; q[n][2] = p0.z; q[n][3] = p0.w;
+    }
+    int h[NR], l[NR];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+      h[n] = 0;
+      l[n] = X.c0;
+    }
+    // two's-complement 2-bit t: t ^ 2 = t + 2 in 0..3; plane k of a word = bits 2k..2k+1 of its bytes
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int n = 0; n < NR; ++n) {
+        const uint32_t w = q[n][m] ^ 0xAAAAAAAAu;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t c = (w >> (2 * k)) & 0x03030303u;
+          h[n] = dp4a_us(c, X.h[4 * m + k], h[n]);
+          l[n] = dp4a_uu(c, X.l[4 * m + k], l[n]);
+        }
+      }
+#pragma unroll
+    for (int n = 0; n < NR; ++n) out[n] = X.s * float(h[n] * 256 + l[n]);
   } else {  // int4 with per-row scale (applied by the caller): kI4x64 (8 words) or kI4x32 (4 words)
     constexpr int NW = (KIND == kI4x64) ? 8 : 4;
     uint32_t q[NR][8];
@@ -593,13 +641,20 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
       case kI4x64: ok = gemv_matrix<kI4x64, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
       case kQ4One: ok = gemv_matrix<kQ4One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
       case kQ8One: ok = gemv_matrix<kQ8One, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
+      case kI2x64: ok = gemv_matrix<kI2x64, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
       default: ok = gemv_matrix<kI4x32, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
     }
     if (!ok) break;  // still takes part in the argmax completion below, so its count stays whole
   }
   if (prm.am_p < 0) return;
-  // Greedy argmax of y[am_p]: warp, then CTA maximum; one 64-bit atomicMax per CTA on the
-  // packed key; the last CTA to finish decodes it into the token and clears the state.
+  {
+    int ra, rb;
+    cta_rows(cr, prm.p[prm.am_p], prm.am_p, ra, rb);
+    if (!(prm.am_p >= cr.p0 && prm.am_p <= p_last && ra < rb)) return;  // no rows of the argmax output
+  }
+  // Greedy argmax of y[am_p] over the CTAs that wrote its rows: warp, then CTA maximum; one
+  // 64-bit max reduction per CTA on the packed key, then a release/acquire count; the last of
+  // these CTAs decodes the key into the token and clears the state.
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, am_v, o);
@@ -615,12 +670,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
   named_bar_sync(1, kGemvCompute);
   if (threadIdx.x == 0) {
     for (int w = 1; w < kGemvConsumerWarps; ++w) am_take(am_v, am_i, am_wv[w], am_wi[w]);
-    if (am_i != 0x7fffffff) atomicMax(prm.am_state, am_pack(am_v, am_i));
-    __threadfence();
     unsigned int* count = reinterpret_cast<unsigned int*>(prm.am_state + 1);
-    if (atomicAdd(count, 1u) == gridDim.x - 1) {
-      __threadfence();
-      const unsigned long long key = atomicAdd(prm.am_state, 0ull);
+    if (am_i != 0x7fffffff)
+      asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(prm.am_state), "l"(am_pack(am_v, am_i))
+                   : "memory");
+    unsigned int prev;
+    // release: this CTA's maximum is visible before its count; acquire: the last CTA sees them all
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(count) : "memory");
+    if (prev == unsigned(prm.am_ctas) - 1u) {
+      unsigned long long key;
+      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(key) : "l"(prm.am_state) : "memory");
       float v;
       int i;
       am_unpack(key, v, i);

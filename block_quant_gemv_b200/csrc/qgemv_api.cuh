@@ -16,6 +16,11 @@ inline size_t weight_bytes(int fmt, int rows, int cols) {
       const size_t packed = size_t(rows) * size_t(cols / 2);
       return (packed + 15) / 16 * 16 + 4 * size_t(rows);
     }
+    case BQG_I2_ROW: {
+      if (cols % 64 != 0) return 0;
+      const size_t packed = size_t(rows) * size_t(cols / 4);
+      return (packed + 15) / 16 * 16 + 4 * size_t(rows);
+    }
     default: return 0;
   }
 }
@@ -23,8 +28,9 @@ inline size_t weight_bytes(int fmt, int rows, int cols) {
 // Fills a GemvProb from one (fmt, W, x, y, rows, cols) after checking it.
 inline int make_gemv_prob(int fmt, const void* W, const float* x, float* y, int rows, int cols, GemvProb* out) {
   if (W == nullptr || x == nullptr || y == nullptr || rows < 1 || cols < 1) return BQG_ERR_ARG;
-  if (fmt != BQG_Q8_0 && fmt != BQG_Q4_0 && fmt != BQG_I4_ROW) return BQG_ERR_FMT;
+  if (fmt != BQG_Q8_0 && fmt != BQG_Q4_0 && fmt != BQG_I4_ROW && fmt != BQG_I2_ROW) return BQG_ERR_FMT;
   if (cols % 32 != 0 || cols > BQG_MAX_COLS) return BQG_ERR_SHAPE;
+  if (fmt == BQG_I2_ROW && cols % 64 != 0) return BQG_ERR_SHAPE;
   if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 4)) return BQG_ERR_ALIGN;
   GemvProb P{};
   P.W = static_cast<const uint8_t*>(W);
@@ -39,6 +45,12 @@ inline int make_gemv_prob(int fmt, const void* W, const float* x, float* y, int 
   } else if (fmt == BQG_Q4_0) {
     P.kind = (nb % 2 == 0) ? kQ4Pair : kQ4One;
     P.row_bytes = nb * 18;
+  } else if (fmt == BQG_I2_ROW) {
+    P.kind = kI2x64;
+    P.row_bytes = cols / 4;
+    const long long packed = (long long)rows * P.row_bytes;
+    if ((packed + 15) / 16 * 16 > 0x7fffffffLL) return BQG_ERR_LIMIT;
+    P.scale_off = int((packed + 15) / 16 * 16);
   } else {
     P.kind = (cols % 64 == 0) ? kI4x64 : kI4x32;
     P.row_bytes = cols / 2;
@@ -114,6 +126,17 @@ inline int launch_gemv(GemvParams<MAXP>& prm, long long total_rows, cudaStream_t
       prm.cta[c - 1].r1 = cur.r0;
     }
     prev = cur;
+  }
+  if (prm.am_p >= 0) {  // the CTAs whose row range includes rows of the argmax output
+    prm.am_ctas = 0;
+    for (int c = 0; c < grid; ++c) {
+      const CtaRange& r = prm.cta[c];
+      const int q = prm.am_p;
+      const int ra = q == r.p0 ? r.r0 : 0;
+      const int rb = q < r.p1 ? prm.p[q].rows : (q == r.p1 ? r.r1 : 0);
+      if (q >= r.p0 && q <= r.p1 && q < prm.n && ra < rb) ++prm.am_ctas;
+    }
+    if (prm.am_ctas == 0) return BQG_ERR_ARG;
   }
   k_qgemv<MAXP><<<grid, kGemvThreads, kGemvSmemBytes, stream>>>(prm);
   return launch_status();

@@ -36,6 +36,10 @@
  *   BQG_I4_ROW row r = cols/2 bytes of two's-complement nibbles (weight 2j in the low nibble
  *              of byte j); after all rows, zero padding to a 16-byte boundary, then one
  *              little-endian fp32 scale per row; y_r = s_r * sum_i q_ri * x_i.
+ *   BQG_I2_ROW row r = cols/4 bytes of two's-complement 2-bit values (weight 4j+k in bits
+ *              2k..2k+1 of byte j: 0b00 = 0, 0b01 = 1, 0b10 = -2, 0b11 = -1); after all rows, zero
+ *              padding to a 16-byte boundary, then one fp32 scale per row; cols % 64 == 0.
+ *              Source: colibri wiki summary, "구현 범위" (packed int2 with a per-row scale).
  */
 #ifndef BQG_H
 #define BQG_H
@@ -67,7 +71,7 @@ enum bqg_status {
   BQG_ERR_LIMIT = -8      /* a documented maximum is exceeded (descriptor count, sizes)    */
 };
 
-enum bqg_fmt { BQG_Q8_0 = 1, BQG_Q4_0 = 2, BQG_I4_ROW = 3 };
+enum bqg_fmt { BQG_Q8_0 = 1, BQG_Q4_0 = 2, BQG_I4_ROW = 3, BQG_I2_ROW = 4 };
 enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 
 /* How moe_forward runs the experts (bqg_moe_layer.path).  Both compute the same layer.
@@ -117,7 +121,7 @@ BQG_API int bqg_device_errors(int* bits);
  * qgemv: y = W x for one quantized matrix.
  *   Source: Camelid README, "Engine status" (Q8_0) and "Gemma 4" (Q4_0 projection GEMVs);
  *   colibri wiki summary, "구현 범위" (packed int4 with per-row scale).
- *   fmt   BQG_Q8_0, BQG_Q4_0 or BQG_I4_ROW.
+ *   fmt   BQG_Q8_0, BQG_Q4_0, BQG_I4_ROW or BQG_I2_ROW (cols % 64 == 0).
  *   W     device, bqg_weight_bytes(fmt, rows, cols) bytes, 16-byte aligned.
  *   x     device fp32 [cols], 16-byte aligned.   y  device fp32 [rows], 4-byte aligned.
  *   rows  >= 1.   cols  multiple of 32, 32 <= cols <= BQG_MAX_COLS.
@@ -213,7 +217,7 @@ typedef struct {
   int top_k;         /* 1..BQG_MAX_TOPK, <= n_experts               */
   int hidden;        /* multiple of 32, <= BQG_MAX_MOE_COLS         */
   int inter;         /* multiple of 32, <= BQG_MAX_MOE_COLS         */
-  int expert_fmt;    /* BQG_Q8_0, BQG_Q4_0 or BQG_I4_ROW            */
+  int expert_fmt;    /* BQG_Q8_0, BQG_Q4_0, BQG_I4_ROW or BQG_I2_ROW  */
   int act;           /* BQG_ACT_GELU_TANH or BQG_ACT_SILU           */
   const void* gate;  /* device, 16-byte aligned                      */
   const void* up;

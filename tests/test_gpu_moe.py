@@ -19,6 +19,8 @@ SMALL = [
     wl.MoESpec("m_i4_silu", 16, 8, 256, 64, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False),
     wl.MoESpec("m_q4_odd", 5, 5, 160, 96, bqg.Q4_0, bqg.ACT_GELU_TANH, 32, bqg.Q4_0, False),
     wl.MoESpec("m_i4_shared_q8", 12, 4, 192, 128, bqg.I4_ROW, bqg.ACT_GELU_TANH, 64, bqg.Q8_0, False),
+    wl.MoESpec("m_i2_silu", 16, 8, 256, 128, bqg.I2_ROW, bqg.ACT_SILU, 0, 0, False),
+    wl.MoESpec("m_q4_shared_i2", 8, 2, 128, 64, bqg.Q4_0, bqg.ACT_GELU_TANH, 192, bqg.I2_ROW, False),
 ]
 
 
@@ -183,3 +185,15 @@ def test_binding_rejects_short_buffers():
         bqg.moe_forward(lay, x, idx, w, torch.empty(2, spec.hidden, device="cuda"))
     with pytest.raises(ValueError):
         bqg.moe_forward_noalloc(lay, x, idx, w[:1], torch.empty(3, spec.hidden, device="cuda"))
+
+
+def test_glm_like_int2_layer_full_geometry():
+    """The GLM-like layer with packed int2 experts (hidden 6144, 256 experts of 2048, SwiGLU, top-8
+    of given N(0,1) logits): every token at T = 1 and T = 8 against the oracle."""
+    need_gpu()
+    spec = wl.MoESpec("glm_i2", 256, 8, 6144, 2048, bqg.I2_ROW, bqg.ACT_SILU, 0, 0, False)
+    L = wl.build_moe_layer(spec, 0, 0, device="cuda")
+    for tokens in (1, 8):
+        _glm_layer_check(L, spec, 0, tokens)
+    del L
+    torch.cuda.empty_cache()

@@ -159,3 +159,53 @@ def test_repeated_launches_and_graph_replays():
         for y in ys:
             assert torch.equal(y, ref), f"replay {rep}"
     assert bqg.bqg_device_errors() == 0
+
+
+# ---------------------------------------------------------------- packed int2 with a per-row scale
+I2_SHAPES = [(1, 64), (37, 128), (130, 704), (300, 2112), (77, 5632), (1000, 2048), (2048, 2048),
+             (4099, 256), (64, 15360), (513, 2816)]
+
+
+@pytest.mark.parametrize("rows,cols", I2_SHAPES)
+def test_qgemv_i2_row_matches_oracle(rows, cols):
+    y, ref = _run(bqg.I2_ROW, rows, cols)
+    assert_close(y, ref, what=f"i2_row {rows}x{cols}")
+    if rows >= 64:
+        assert_close(y, ref, tol=2e-4, what=f"i2_row {rows}x{cols} (x fixed-point accuracy)")
+
+
+def test_qgemv_i2_row_unit_probes_and_determinism():
+    """x = e_j reads column j (s_r * q_rj exactly); two calls give identical bits; cols not a
+    multiple of 64 is refused."""
+    need_gpu()
+    rows, cols = 96, 1024
+    W = synth.matrix(bqg.I2_ROW, rows, cols, 5, "i2probe")
+    deq = oq.dequantize(bqg.I2_ROW, W.numpy(), rows, cols)
+    for j in (0, 1, 2, 3, 4, 63, 64, 511, 1023):
+        e = torch.zeros(cols)
+        e[j] = 1.0
+        y = bqg.qgemv(bqg.I2_ROW, W.cuda(), e.cuda(), rows, cols).cpu().numpy()
+        np.testing.assert_allclose(y, deq[:, j], rtol=1e-6, atol=1e-9)
+    x = synth.normal_f32(5, 6, cols).cuda()
+    assert torch.equal(bqg.qgemv(bqg.I2_ROW, W.cuda(), x, rows, cols), bqg.qgemv(bqg.I2_ROW, W.cuda(), x, rows, cols))
+    with pytest.raises(bqg.BQGError) as e:
+        bqg.qgemv(bqg.I2_ROW, W.cuda(), x, rows, 992)
+    assert e.value.status == -3
+
+
+def test_qgemv_batched_mixed_with_i2_row():
+    """int2 matrices inside a mixed-format batch (one launch)."""
+    need_gpu()
+    specs = [(bqg.I2_ROW, 700, 2048), (bqg.Q4_0, 300, 2048), (bqg.I2_ROW, 2048, 704), (bqg.Q8_0, 64, 128),
+             (bqg.I4_ROW, 129, 640)]
+    items, refs = [], []
+    for i, (fmt, rows, cols) in enumerate(specs):
+        W = synth.matrix(fmt, rows, cols, 0, f"mix2/{i}")
+        x = synth.normal_f32(0, 100 + i, cols)
+        y = torch.empty(rows, device="cuda")
+        items.append((fmt, W.cuda(), x.cuda(), y, rows, cols))
+        refs.append(oq.qgemv(fmt, W.numpy(), x.numpy().astype(np.float64), rows, cols))
+    bqg.qgemv_batched(items)
+    torch.cuda.synchronize()
+    for (fmt, _, _, y, rows, cols), ref in zip(items, refs):
+        assert_close(y, ref, tol=2e-4, what=f"mixed batch fmt {fmt} {rows}x{cols}")
