@@ -41,7 +41,7 @@ def test_oracle_imports_neither_the_product_nor_the_generators():
 
 
 def test_bench_reaches_the_oracle_only_from_its_cpu_legs():
-    legs = {"oracle_sample", "run_reference"}
+    legs = {"oracle_sample", "oracle_moe_sample", "oracle_prefill_sample", "run_reference"}
     for mod, func in _imports(os.path.join(ROOT, "bench.py")):
         if mod == "oracle":
             assert func in legs, f"bench.py imports the oracle in {func}"
