@@ -694,6 +694,64 @@ def time_moe_glm_i2(dev, seed, peak, layers=8):
     return out
 
 
+def time_expert_cache(dev, seed, n_host=64, n_slots=16, calls=10):
+    """GLM-like experts (hidden 6144, int4 SwiGLU 2048, top-8) in pinned host memory, 16 device
+    slots, one token per layer: us per layer and host-to-device bytes at 100 %, 50 % and 0 % hits.
+    The routing is chosen to give those hit rates: the same 8 experts every call; 4 of them kept
+    plus 4 taken in turn from the other experts; 8 new experts every call (blocks of 8 in turn,
+    of which the slots hold two)."""
+    import dataclasses
+
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    spec = dataclasses.replace(wl.GLM_MOE, name="cache_glm", n_experts=n_host)
+    L = wl.build_moe_layer(spec, seed, 0, device="cpu")
+    host = [t.pin_memory() for t in (L.gate, L.up, L.down)]
+    cache = bqg.ExpertCache(spec.n_experts, spec.top_k, spec.hidden, spec.inter, spec.expert_fmt, spec.act, *host,
+                            L.gate_stride, L.up_stride, L.down_stride, n_slots)
+    x = wl.moe_tokens(spec, seed, 1).to(dev)
+    w = torch.full((1, 8), 1.0 / 8, device=dev)
+    y = torch.empty(1, spec.hidden, device=dev)
+    ws = torch.empty(cache.workspace_size(1), dtype=torch.uint8, device=dev)
+    expert_bytes = sum(spec.mat_bytes(m) for m in ("gate", "up", "down"))
+
+    def routing(kind, i):
+        if kind == "hit100":
+            e = list(range(8))
+        elif kind == "hit50":
+            e = list(range(4)) + [8 + (4 * i + j) % (n_host - 8) for j in range(4)]
+        else:
+            e = [(8 * i + j) % n_host for j in range(8)]
+        return torch.tensor([e], dtype=torch.int32)
+
+    out = {"workload": f"glm-like experts (hidden 6144, int4 SwiGLU 2048, top-8), {n_host} on the host (pinned), "
+                       f"{n_slots} device slots, 1 token per layer; {calls} timed calls per case"}
+    stream = torch.cuda.current_stream()
+    for kind in ("hit100", "hit50", "hit0"):
+        for i in range(calls):  # warm-up: the same sequence, so the slots hold what the timed calls expect
+            cache.forward(x, routing(kind, i), w, y, ws)
+        torch.cuda.synchronize()
+        before = cache.stats()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(calls):
+            cache.forward(x, routing(kind, i + calls), w, y, ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        after = cache.stats()
+        us = e0.elapsed_time(e1) * 1e3 / calls
+        hits = after["hits"] - before["hits"]
+        misses = after["misses"] - before["misses"]
+        h2d = (after["bytes_copied"] - before["bytes_copied"]) / calls
+        out[kind] = {"us_per_layer": us, "hit_rate": hits / max(1, hits + misses), "h2d_bytes_per_layer": h2d,
+                     "h2d_GB/s": h2d / us / 1e3, "hbm_bytes_per_layer": 8 * expert_bytes}
+    del cache, host, L
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
     assert torch.cuda.is_available(), "bench.py --impl ours needs a CUDA device"
@@ -718,6 +776,7 @@ def run_ours(args, world, rank, local):
         if not args.no_glm:
             extras["moe_glm"] = time_moe_glm(dev, args.seed, peak)
             extras["moe_glm_i2"] = time_moe_glm_i2(dev, args.seed, peak)
+        extras["expert_cache_glm"] = time_expert_cache(dev, args.seed)
     extras["decode_step_without_greedy_token"] = {
         "ms_per_step": r["plain_ms"], "GB/s": step_bytes / (r["plain_ms"] * 1e-3) / 1e9,
         "argmax_cost_frac": r["launch_ms"] / r["plain_ms"] - 1.0}

@@ -24,7 +24,7 @@ __all__ = [
     "lib", "library_path", "bqg_status_string", "bqg_weight_bytes", "bqg_device_errors",
     "bqg_selftest_wait_timeout",
     "qgemv", "qgemv_batched", "GemvBatch", "qgemv_argmax", "ArgmaxState", "qgemm_prefill", "moe_router_logits",
-    "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward", "moe_forward_noalloc",
+    "moe_router_topk", "MoELayer", "moe_workspace_size", "moe_forward", "moe_forward_noalloc", "ExpertCache",
 ]
 
 Q8_0, Q4_0, I4_ROW, I2_ROW = 1, 2, 3, 4
@@ -61,6 +61,15 @@ class MoELayerC(ctypes.Structure):
                 ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp), ("path", _i)]
 
 
+class ExpertCacheDesc(ctypes.Structure):
+    _fields_ = [("layer", MoELayerC), ("n_slots", _i), ("slot_gate", _vp), ("slot_up", _vp), ("slot_down", _vp)]
+
+
+class ExpertCacheStats(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_longlong), ("hits", ctypes.c_longlong), ("misses", ctypes.c_longlong),
+                ("evictions", ctypes.c_longlong), ("bytes_copied", ctypes.c_longlong)]
+
+
 _SIGNATURES = {
     "bqg_status_string": (ctypes.c_char_p, [_i]),
     "bqg_version": (_i, []),
@@ -77,6 +86,11 @@ _SIGNATURES = {
     "moe_forward": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "moe_forward_noalloc": (_i, [ctypes.POINTER(MoELayerC), _vp, _vp, _vp, _vp, _i, _vp]),
     "bqg_selftest_wait_timeout": (_i, [_vp]),
+    "bqg_expert_cache_create": (_i, [ctypes.POINTER(ExpertCacheDesc), ctypes.POINTER(_vp)]),
+    "bqg_expert_cache_destroy": (None, [_vp]),
+    "bqg_expert_cache_workspace_size": (_sz, [_vp, _i]),
+    "bqg_expert_cache_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp, _vp]),
+    "bqg_expert_cache_get_stats": (_i, [_vp, ctypes.POINTER(ExpertCacheStats)]),
 }
 
 
@@ -383,3 +397,96 @@ def moe_forward_noalloc(layer: MoELayer, x: torch.Tensor, idx: torch.Tensor, w: 
     _check(lib().moe_forward_noalloc(ctypes.byref(layer.c), _ptr(x), _ptr(idx), _ptr(w), _ptr(y), tokens, _stream(x)),
            "moe_forward_noalloc")
     return y
+
+
+# ---------------------------------------------------------------- host-resident experts
+class ExpertCache:
+    """Routed experts of one layer in pinned host memory, `n_slots` of them resident in device
+    slots (LFU replacement with a recency tie-break).  forward() takes the routing ids on the
+    host and computes the layer exactly as moe_forward would.
+
+    gate/up/down: pinned host uint8 tensors with n_experts matrices each (expert e at
+    e * <name>_stride); shared: optional (fmt, inter, gate, up, down) DEVICE uint8 tensors."""
+
+    def __init__(self, n_experts: int, top_k: int, hidden: int, inter: int, expert_fmt: int, act: int,
+                 gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor,
+                 gate_stride: int, up_stride: int, down_stride: int, n_slots: int, shared=None, device="cuda",
+                 path: int = 0):
+        for name, t in (("gate", gate), ("up", up), ("down", down)):
+            if t.is_cuda or t.dtype != torch.uint8 or not t.is_contiguous():
+                raise TypeError(f"{name} must be a contiguous uint8 HOST tensor (pinned for asynchronous copies)")
+        if not 1 <= n_slots <= min(n_experts, MAX_EXPERTS):
+            raise ValueError(f"n_slots must be in 1..{min(n_experts, MAX_EXPERTS)}")
+        # the host stacks, described as a layer (the library checks them like any MoE layer)
+        self.host = MoELayer.__new__(MoELayer)
+        c = MoELayerC()
+        c.n_experts, c.top_k, c.hidden, c.inter, c.expert_fmt, c.act = n_experts, top_k, hidden, inter, expert_fmt, act
+        c.gate, c.up, c.down = gate.data_ptr(), up.data_ptr(), down.data_ptr()
+        c.gate_stride, c.up_stride, c.down_stride = gate_stride, up_stride, down_stride
+        c.path = path
+        for name, t, rows, cols, stride in (("gate", gate, inter, hidden, gate_stride), ("up", up, inter, hidden, up_stride),
+                                            ("down", down, hidden, inter, down_stride)):
+            nb = bqg_weight_bytes(expert_fmt, rows, cols)
+            if nb == 0 or stride < nb or t.numel() < (n_experts - 1) * stride + nb:
+                raise ValueError(f"{name}: host tensor or stride too small for {n_experts} experts")
+        self.tensors = [gate, up, down]
+        if shared is not None:
+            sfmt, sinter, sg, su, sd = shared
+            for t in (sg, su, sd):
+                _need_cuda("shared expert", t, torch.uint8)
+            c.shared_inter, c.shared_fmt = sinter, sfmt
+            c.s_gate, c.s_up, c.s_down = sg.data_ptr(), su.data_ptr(), sd.data_ptr()
+            self.tensors += [sg, su, sd]
+        self.slots = [torch.empty(n_slots * st, dtype=torch.uint8, device=device)
+                      for st in (gate_stride, up_stride, down_stride)]
+        d = ExpertCacheDesc()
+        d.layer = c
+        d.n_slots = n_slots
+        d.slot_gate, d.slot_up, d.slot_down = [t.data_ptr() for t in self.slots]
+        self.desc = d
+        h = _vp()
+        _check(lib().bqg_expert_cache_create(ctypes.byref(d), ctypes.byref(h)), "bqg_expert_cache_create")
+        self.handle = h
+        self.hidden, self.top_k, self.n_experts, self.n_slots = hidden, top_k, n_experts, n_slots
+        self.device = torch.device(device)
+        self.copy_stream = torch.cuda.Stream(device=self.device)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            lib().bqg_expert_cache_destroy(h)
+            self.handle = None
+
+    def workspace_size(self, tokens: int) -> int:
+        return int(lib().bqg_expert_cache_workspace_size(self.handle, tokens))
+
+    def forward(self, x: torch.Tensor, idx_host: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """y for routing ids idx_host (int32 HOST tensor [tokens, top_k]) and weights w (device)."""
+        _need_cuda("x", x, torch.float32)
+        _need_cuda("w", w, torch.float32)
+        if idx_host.is_cuda or idx_host.dtype != torch.int32 or not idx_host.is_contiguous():
+            raise TypeError("idx_host must be a contiguous int32 HOST tensor")
+        tokens = x.numel() // self.hidden
+        if tokens < 1 or x.numel() != tokens * self.hidden:
+            raise ValueError(f"x must hold whole tokens of hidden = {self.hidden} values")
+        if idx_host.numel() < tokens * self.top_k or w.numel() < tokens * self.top_k:
+            raise ValueError(f"idx_host and w must hold tokens x top_k = {tokens} x {self.top_k} values")
+        if y is None:
+            y = torch.empty(tokens, self.hidden, dtype=torch.float32, device=x.device)
+        _need_cuda("y", y, torch.float32)
+        if y.numel() < tokens * self.hidden:
+            raise ValueError("y too small")
+        need = self.workspace_size(tokens)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+        _need_cuda("workspace", workspace, torch.uint8)
+        _check(lib().bqg_expert_cache_forward(self.handle, _ptr(x), idx_host.data_ptr(), _ptr(w), _ptr(y), tokens,
+                                              _ptr(workspace), workspace.numel(), _stream(x),
+                                              _vp(self.copy_stream.cuda_stream)), "bqg_expert_cache_forward")
+        return y
+
+    def stats(self) -> dict:
+        st = ExpertCacheStats()
+        _check(lib().bqg_expert_cache_get_stats(self.handle, ctypes.byref(st)), "bqg_expert_cache_get_stats")
+        return {name: int(getattr(st, name)) for name, _ in ExpertCacheStats._fields_}

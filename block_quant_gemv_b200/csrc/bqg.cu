@@ -6,7 +6,10 @@
 //   qgemv.cuh        dequantize-fused GEMV kernel (single matrix and decode-step list)
 //   qgemv_api.cuh    qgemv / qgemv_batched entry points
 //   router.cuh       router logits and softmax/top-k/renormalise kernels + entry points
-//   moe.cuh          grouped MoE layer kernels + moe_forward
+//   moe.cuh          grouped MoE layer kernels (CUDA cores)
+//   moe_tc.cuh       grouped expert GEMM on tcgen05 (many tokens)
+//   moe_api.cuh      moe_forward: workspace, path choice, launches
+//   expert_cache.cuh host-resident experts with a device slot cache
 //   prefill.cuh      tcgen05 prefill-chunk GEMM + qgemm_prefill
 //   selftest.cuh     failure-detection self-test (a bounded wait that runs out)
 #include "common.cuh"
@@ -14,6 +17,7 @@
 #include "qgemv_api.cuh"
 #include "router.cuh"
 #include "moe_api.cuh"
+#include "expert_cache.cuh"
 #include "prefill.cuh"
 #include "selftest.cuh"
 

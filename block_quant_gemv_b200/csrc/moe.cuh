@@ -230,6 +230,7 @@ struct RouteWs {
   int32_t* perm;      // [T * k] pair ids (t * k + j) grouped by expert, token order inside
   uint32_t* ctr;      // [2] work item counters of the two grouped GEMV launches
   int4* act_info;     // [E] per touched expert (in active order): (expert, count, offset, first pair)
+  int skip_negative;  // 1: negative ids mark pairs left out of this call (skipped, not an error)
 };
 
 __device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int pairs, int n_experts,
@@ -245,7 +246,7 @@ __device__ __forceinline__ void moe_route(const int32_t* __restrict__ idx, int p
   for (int p = tid; p < pairs; p += kRouteThreads) {
     const int e = idx[p];
     if (e >= 0 && e < n_experts) atomicAdd(&cnt[e], 1);
-    else bad = true;
+    else if (!(ws.skip_negative && e < 0)) bad = true;
   }
   if (bad) flag_error(BQG_DEVERR_EXPERT_ID);
   __syncthreads();
@@ -675,10 +676,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_moe_gemv(const __grid_const
 
 // ---------------------------------------------------------------- 4. combine
 // y[t, c] = sum_{j<k} w[t, j] * part[t*k + j, c] in slot order (pairs with an invalid expert id
-// contribute nothing), plus the shared output.
+// contribute nothing), plus the shared output; with `accumulate`, added to y instead of stored.
 __global__ void k_moe_combine(const float* __restrict__ part, const int32_t* __restrict__ idx,
                               const float* __restrict__ w, const float* __restrict__ sout, float* __restrict__ y,
-                              int tokens, int top_k, int hidden, int n_experts) {
+                              int tokens, int top_k, int hidden, int n_experts, int accumulate) {
   griddep_wait();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)tokens * hidden) return;
@@ -702,7 +703,7 @@ __global__ void k_moe_combine(const float* __restrict__ part, const int32_t* __r
 #pragma unroll
   for (int j = 0; j < BQG_MAX_TOPK; ++j)
     if (j < top_k) acc = fmaf(wv[j], pv[j], acc);
-  y[i] = acc + s;
+  y[i] = accumulate ? y[i] + (acc + s) : acc + s;
 }
 
 }  // namespace bqg

@@ -315,7 +315,8 @@ namespace bqg {
 // The layer on the tensor-core path: route grouping (one block), fp16 activation rows, the
 // grouped gate/up GEMM with act(g) * u in its epilogue, the grouped down GEMM, the combine.
 inline int moe_forward_tc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
-                          int tokens, uint8_t* ws, int dev, const DeviceInfo* info, cudaStream_t s) {
+                          int tokens, uint8_t* ws, int dev, const DeviceInfo* info, cudaStream_t s, int skip_negative,
+                          int accumulate) {
   TcLayer TL;
   if (!tc_layer(L, &TL)) return BQG_ERR_SHAPE;
   const MoeTcLayout lay = moe_ws_layout_tc(L, tokens);
@@ -329,6 +330,7 @@ inline int moe_forward_tc(const bqg_moe_layer* L, const float* x, const int32_t*
   route.perm = reinterpret_cast<int32_t*>(ws + lay.perm);
   route.ctr = reinterpret_cast<uint32_t*>(ws + lay.ctr);
   route.act_info = reinterpret_cast<int4*>(ws + lay.act_info);
+  route.skip_negative = skip_negative;
   auto H = [&](size_t o) { return reinterpret_cast<__half*>(ws + o); };
   auto F = [&](size_t o) { return reinterpret_cast<float*>(ws + o); };
   int st;
@@ -357,7 +359,7 @@ inline int moe_forward_tc(const bqg_moe_layer* L, const float* x, const int32_t*
   const long long n = (long long)tokens * L->hidden;
   return launch_pdl(k_moe_combine, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s, (const float*)F(lay.part), idx, w,
                     sh ? (const float*)F(lay.sout) : (const float*)nullptr, y, tokens, L->top_k, L->hidden,
-                    L->n_experts);
+                    L->n_experts, accumulate);
 }
 }  // namespace bqg
 
@@ -366,9 +368,12 @@ extern "C" size_t moe_workspace_size(const bqg_moe_layer* L, int tokens) {
   return bqg::moe_ws_total(L, tokens);
 }
 
-extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
-                           int tokens, void* workspace, size_t ws_bytes, void* stream) {
-  using namespace bqg;
+namespace bqg {
+// moe_forward with two internal options: skip_negative (negative ids mark pairs that belong to
+// another call: skipped without an error) and accumulate (y += this call's sum instead of y =).
+inline int moe_forward_impl(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
+                            int tokens, void* workspace, size_t ws_bytes, void* stream, int skip_negative,
+                            int accumulate) {
   int st = check_layer(L);
   if (st != BQG_OK) return st;
   if (x == nullptr || idx == nullptr || w == nullptr || y == nullptr || tokens < 1) return BQG_ERR_ARG;
@@ -384,7 +389,8 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   if (st != BQG_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (path == BQG_MOE_PATH_TENSOR_CORES) return moe_forward_tc(L, x, idx, w, y, tokens, ws, dev, info, s);
+  if (path == BQG_MOE_PATH_TENSOR_CORES)
+    return moe_forward_tc(L, x, idx, w, y, tokens, ws, dev, info, s, skip_negative, accumulate);
   const MoeWsLayout lay = moe_ws_layout(L, tokens);
   auto F = [&](size_t o) { return reinterpret_cast<float*>(ws + o); };
   auto R = [&](size_t o) { return reinterpret_cast<uint4*>(ws + o); };
@@ -399,6 +405,7 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   route.perm = reinterpret_cast<int32_t*>(ws + lay.perm);
   route.ctr = reinterpret_cast<uint32_t*>(ws + lay.ctr);
   route.act_info = reinterpret_cast<int4*>(ws + lay.act_info);
+  route.skip_negative = skip_negative;
 
   // routed and shared matrix families
   const MgMat gate = mg_mat(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden);
@@ -497,5 +504,11 @@ extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t
   // 5. combine
   const long long n = (long long)tokens * L->hidden;
   return launch_pdl(k_moe_combine, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s, F(lay.part), idx, w,
-                    sh ? F(lay.sout) : nullptr, y, tokens, L->top_k, L->hidden, L->n_experts);
+                    sh ? F(lay.sout) : nullptr, y, tokens, L->top_k, L->hidden, L->n_experts, accumulate);
+}
+}  // namespace bqg
+
+extern "C" int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
+                           int tokens, void* workspace, size_t ws_bytes, void* stream) {
+  return bqg::moe_forward_impl(L, x, idx, w, y, tokens, workspace, ws_bytes, stream, 0, 0);
 }

@@ -259,6 +259,56 @@ BQG_API size_t moe_workspace_size(const bqg_moe_layer* L, int tokens);
 BQG_API int moe_forward(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w,
                 float* y, int tokens, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- host-resident experts, device slot cache
+ * An expert cache keeps a layer's routed experts in HOST memory (pinned, for asynchronous copies)
+ * and the ones in use in n_slots device slots.  bqg_expert_cache_forward computes exactly
+ * moe_forward's y for routing ids given on the host: it loads the missing experts into slots
+ * (replacing the least frequently used slot that this call does not need, the least recently
+ * used among equals) with cudaMemcpyAsync on copy_stream, runs the hit experts and the shared
+ * expert on stream while those copies are in flight, then the missed experts once they have
+ * landed, summed into the same y.
+ *   Source: TurboFieldfare wiki, "메모리·전문가 스트리밍" (16 expert slots per layer, LFU with a
+ *   recency tie-break, hits and misses split, loads overlapped with compute); Camelid README,
+ *   "Supported models" (SSER: host-resident experts with an adaptive VRAM expert cache); colibri
+ *   wiki summary, "구현 범위" (per-layer expert cache).
+ * bqg_expert_cache_desc.layer describes the routed experts as in moe_forward, except that gate,
+ * up and down are HOST pointers to the stacked experts (expert e at base + e * stride); the
+ * optional shared expert's pointers are DEVICE pointers.  slot_gate / slot_up / slot_down are
+ * DEVICE buffers of n_slots * {gate, up, down}_stride bytes (16-byte aligned), owned by the
+ * caller.  The cache object itself is host memory allocated by bqg_expert_cache_create.
+ *   - At most n_slots distinct experts per call (else BQG_ERR_LIMIT, nothing done).
+ *   - idx_host: HOST int32 [tokens x top_k] routing ids (as written by moe_router_topk and copied
+ *     to the host); w, x, y: device, as for moe_forward.
+ *   - workspace: device, >= bqg_expert_cache_workspace_size(cache, tokens) bytes, 256-aligned.
+ *   - Calls on one cache must be made from one host thread, in order, on the same two streams;
+ *     the cache's bookkeeping is updated before the work is enqueued, so after an error destroy
+ *     and re-create it. */
+typedef struct {
+  bqg_moe_layer layer;  /* routed experts on the HOST (gate, up, down), shared expert on the device */
+  int n_slots;          /* device slots, 1 .. min(n_experts, BQG_MAX_EXPERTS) */
+  void* slot_gate;      /* DEVICE n_slots * layer.gate_stride bytes */
+  void* slot_up;        /* DEVICE n_slots * layer.up_stride bytes */
+  void* slot_down;      /* DEVICE n_slots * layer.down_stride bytes */
+} bqg_expert_cache_desc;
+
+typedef struct {
+  long long calls;        /* completed forward calls */
+  long long hits;         /* distinct experts found in a slot, summed over calls */
+  long long misses;       /* distinct experts loaded, summed over calls */
+  long long evictions;    /* slots whose expert was replaced */
+  long long bytes_copied; /* host-to-device bytes of the loads */
+} bqg_expert_cache_stats;
+
+typedef struct bqg_expert_cache bqg_expert_cache;
+
+BQG_API int bqg_expert_cache_create(const bqg_expert_cache_desc* desc, bqg_expert_cache** cache);
+BQG_API void bqg_expert_cache_destroy(bqg_expert_cache* cache);
+BQG_API size_t bqg_expert_cache_workspace_size(const bqg_expert_cache* cache, int tokens);
+BQG_API int bqg_expert_cache_forward(bqg_expert_cache* cache, const float* x, const int32_t* idx_host,
+                                     const float* w, float* y, int tokens, void* workspace, size_t ws_bytes,
+                                     void* stream, void* copy_stream);
+BQG_API int bqg_expert_cache_get_stats(const bqg_expert_cache* cache, bqg_expert_cache_stats* stats);
+
 /* ---------------------------------------------------------------- moe_forward without allocation
  * moe_forward_noalloc: the same computation as moe_forward, for callers that cannot allocate
  * device memory around the call (a CUDA graph captured by another component, a runtime that

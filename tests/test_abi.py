@@ -33,7 +33,8 @@ def test_header_declares_the_api():
     for want in ["qgemv", "qgemv_batched", "qgemm_prefill", "moe_router_logits", "moe_router_topk",
                  "moe_workspace_size", "moe_forward", "moe_forward_noalloc", "bqg_status_string", "bqg_weight_bytes",
                  "bqg_device_errors", "bqg_version", "bqg_selftest_wait_timeout", "qgemv_argmax",
-                 "qgemv_batched_argmax"]:
+                 "qgemv_batched_argmax", "bqg_expert_cache_create", "bqg_expert_cache_destroy",
+                 "bqg_expert_cache_workspace_size", "bqg_expert_cache_forward", "bqg_expert_cache_get_stats"]:
         assert want in names
 
 
@@ -249,3 +250,26 @@ def test_argmax_argument_errors(L):
         d.fmt, d.rows, d.cols, d.W, d.x, d.y = 2, 4, 32, A, A, A
     assert g(D, 3, 3, A, None, A, None) == -1                       # index outside the batch
     assert g(D, 3, -1, A, None, A, None) == -1
+
+
+def test_expert_cache_argument_errors(L):
+    """Creation is refused for bad slot counts or a slot layer that is not a valid MoE layer,
+    before any device call."""
+    import block_quant_gemv_b200 as bqg
+    from synth import workloads as wl
+    d = bqg.ExpertCacheDesc()
+    d.layer = _layer_c(wl.GLM_MOE)
+    d.n_slots = 16
+    d.slot_gate = d.slot_up = d.slot_down = 0x40000
+    h = ctypes.c_void_p()
+    f = L.lib().bqg_expert_cache_create
+    d.n_slots = 0
+    assert f(ctypes.byref(d), ctypes.byref(h)) == -1
+    d.n_slots = 300
+    assert f(ctypes.byref(d), ctypes.byref(h)) == -8
+    d.n_slots = 16
+    d.slot_up = 0x40008                                          # slot buffer not 16-byte aligned
+    assert f(ctypes.byref(d), ctypes.byref(h)) == -4
+    d.slot_up = None
+    assert f(ctypes.byref(d), ctypes.byref(h)) == -1
+    assert L.lib().bqg_expert_cache_forward(None, 0x1000, 0x1000, 0x1000, 0x1000, 1, 0x1000, 1 << 20, None, None) == -1
