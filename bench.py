@@ -709,8 +709,11 @@ def time_expert_cache(dev, seed, n_host=64, n_slots=16, calls=10):
     spec = dataclasses.replace(wl.GLM_MOE, name="cache_glm", n_experts=n_host)
     L = wl.build_moe_layer(spec, seed, 0, device="cpu")
     host = [t.pin_memory() for t in (L.gate, L.up, L.down)]
-    cache = bqg.ExpertCache(spec.n_experts, spec.top_k, spec.hidden, spec.inter, spec.expert_fmt, spec.act, *host,
-                            L.gate_stride, L.up_stride, L.down_stride, n_slots)
+
+    def new_cache():  # each case starts from empty slots
+        return bqg.ExpertCache(spec.n_experts, spec.top_k, spec.hidden, spec.inter, spec.expert_fmt, spec.act,
+                               *host, L.gate_stride, L.up_stride, L.down_stride, n_slots)
+    cache = new_cache()
     x = wl.moe_tokens(spec, seed, 1).to(dev)
     w = torch.full((1, 8), 1.0 / 8, device=dev)
     y = torch.empty(1, spec.hidden, device=dev)
@@ -730,6 +733,7 @@ def time_expert_cache(dev, seed, n_host=64, n_slots=16, calls=10):
                        f"{n_slots} device slots, 1 token per layer; {calls} timed calls per case"}
     stream = torch.cuda.current_stream()
     for kind in ("hit100", "hit50", "hit0"):
+        cache = new_cache()
         for i in range(calls):  # warm-up: the same sequence, so the slots hold what the timed calls expect
             cache.forward(x, routing(kind, i), w, y, ws)
         torch.cuda.synchronize()

@@ -531,6 +531,59 @@ __device__ __forceinline__ bool gemv_matrix(const GemvParams<MAXP>& prm, int pi,
   return true;
 }
 
+// The CTA's problems in processing order.  A CTA holding rows of the argmax output takes that
+// matrix first, so that its share of the greedy argmax is merged early, overlapping the rest of
+// its rows, instead of adding a chain of global atomics after the last matrix.
+__device__ __forceinline__ int cta_problem(const CtaRange& cr, int am_first, int q) {
+  if (am_first < 0) return cr.p0 + q;
+  if (q == 0) return am_first;
+  const int pi = cr.p0 + q - 1;
+  return pi >= am_first ? pi + 1 : pi;
+}
+
+// Greedy argmax of y[am_p] over the CTAs that wrote its rows (called by every consumer thread of
+// such a CTA, right after those rows): warp, then CTA maximum; one 64-bit max reduction per CTA
+// on the packed key, then a release/acquire count; the last of these CTAs decodes the key into
+// the token and clears the state.
+template <int MAXP>
+__device__ __forceinline__ void argmax_merge(const GemvParams<MAXP>& prm, float am_v, int am_i) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, am_v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, am_i, o);
+    am_take(am_v, am_i, ov, oi);
+  }
+  __shared__ float am_wv[kGemvConsumerWarps];
+  __shared__ int am_wi[kGemvConsumerWarps];
+  if (lane == 0) {
+    am_wv[warp] = am_v;
+    am_wi[warp] = am_i;
+  }
+  named_bar_sync(1, kGemvCompute);
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kGemvConsumerWarps; ++w) am_take(am_v, am_i, am_wv[w], am_wi[w]);
+    unsigned int* count = reinterpret_cast<unsigned int*>(prm.am_state + 1);
+    if (am_i != 0x7fffffff)
+      asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(prm.am_state), "l"(am_pack(am_v, am_i))
+                   : "memory");
+    unsigned int prev;
+    // release: this CTA's maximum is visible before its count; acquire: the last CTA sees them all
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(count) : "memory");
+    if (prev == unsigned(prm.am_ctas) - 1u) {
+      unsigned long long key;
+      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(key) : "l"(prm.am_state) : "memory");
+      float v;
+      int i;
+      am_unpack(key, v, i);
+      *prm.am_token = i;
+      if (prm.am_value != nullptr) *prm.am_value = v;
+      prm.am_state[0] = 0ull;  // ready for the next call on this stream
+      *count = 0u;
+    }
+  }
+}
+
 template <int MAXP>
 __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant__ GemvParams<MAXP> prm) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -557,6 +610,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
 
   const CtaRange cr = prm.cta[blockIdx.x];
   const int p_last = min(cr.p1, prm.n - 1);
+  const int nprob = p_last >= cr.p0 ? p_last - cr.p0 + 1 : 0;
+  int am_first = -1;  // the argmax output, when this CTA holds rows of it
+  if (prm.am_p >= cr.p0 && prm.am_p <= p_last) {
+    int ra, rb;
+    cta_rows(cr, prm.p[prm.am_p], prm.am_p, ra, rb);
+    if (ra < rb) am_first = prm.am_p;
+  }
 
   if (warp == kGemvConsumerWarps) {
     // ------------------------------------------------ producer warp (one elected lane)
@@ -566,7 +626,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
     int s = 0;
     int xs_n = 0;  // problems whose x has been staged
     bool ok = true;
-    for (int pi = cr.p0; pi <= p_last && ok; ++pi) {
+    for (int q = 0; q < nprob && ok; ++q) {
+      const int pi = cta_problem(cr, am_first, q);
       const GemvProb& P = prm.p[pi];
       int ra, rbnd;
       cta_rows(cr, P, pi, ra, rbnd);
@@ -626,7 +687,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
   XUnit X;
   float am_v = -INFINITY;  // greedy argmax: the best (value, row) this thread has written
   int am_i = 0x7fffffff;
-  for (int pi = cr.p0; pi <= p_last; ++pi) {
+  for (int q = 0; q < nprob; ++q) {
+    const int pi = cta_problem(cr, am_first, q);
     const GemvProb& P = prm.p[pi];
     int ra, rbnd;
     cta_rows(cr, P, pi, ra, rbnd);
@@ -644,50 +706,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) k_qgemv(const __grid_constant
       case kI2x64: ok = gemv_matrix<kI2x64, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
       default: ok = gemv_matrix<kI4x32, MAXP>(prm, pi, ra, rbnd, ring, xs, red, full, xfull, xfree, empty, s, xs_n, X, am_v, am_i); break;
     }
-    if (!ok) break;  // still takes part in the argmax completion below, so its count stays whole
-  }
-  if (prm.am_p < 0) return;
-  {
-    int ra, rb;
-    cta_rows(cr, prm.p[prm.am_p], prm.am_p, ra, rb);
-    if (!(prm.am_p >= cr.p0 && prm.am_p <= p_last && ra < rb)) return;  // no rows of the argmax output
-  }
-  // Greedy argmax of y[am_p] over the CTAs that wrote its rows: warp, then CTA maximum; one
-  // 64-bit max reduction per CTA on the packed key, then a release/acquire count; the last of
-  // these CTAs decodes the key into the token and clears the state.
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, am_v, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, am_i, o);
-    am_take(am_v, am_i, ov, oi);
-  }
-  __shared__ float am_wv[kGemvConsumerWarps];
-  __shared__ int am_wi[kGemvConsumerWarps];
-  if (lane == 0) {
-    am_wv[warp] = am_v;
-    am_wi[warp] = am_i;
-  }
-  named_bar_sync(1, kGemvCompute);
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < kGemvConsumerWarps; ++w) am_take(am_v, am_i, am_wv[w], am_wi[w]);
-    unsigned int* count = reinterpret_cast<unsigned int*>(prm.am_state + 1);
-    if (am_i != 0x7fffffff)
-      asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(prm.am_state), "l"(am_pack(am_v, am_i))
-                   : "memory");
-    unsigned int prev;
-    // release: this CTA's maximum is visible before its count; acquire: the last CTA sees them all
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(count) : "memory");
-    if (prev == unsigned(prm.am_ctas) - 1u) {
-      unsigned long long key;
-      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(key) : "l"(prm.am_state) : "memory");
-      float v;
-      int i;
-      am_unpack(key, v, i);
-      *prm.am_token = i;
-      if (prm.am_value != nullptr) *prm.am_value = v;
-      prm.am_state[0] = 0ull;  // ready for the next call on this stream
-      *count = 0u;
-    }
+    // the argmax output comes first: merge this CTA's share now (also after a failed wait, so
+    // that the count of the CTAs stays whole)
+    if (q == 0 && am_first >= 0) argmax_merge(prm, am_v, am_i);
+    if (!ok) break;
   }
 }
 
