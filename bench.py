@@ -385,7 +385,9 @@ def workload_config():
     return {"workload": "tinyllama_decode: 22 layers x Q4_0 (q,o 2048x2048; k,v 256x2048; gate,up 5632x2048; "
                         "down 2048x5632) + Q8_0 LM head 32000x2048 + greedy token (argmax of the head), batch 1, "
                         "x ~ N(0,1)",
-            "weight_bytes_per_step": 614629376, "launch": "one qgemv_batched_argmax launch per step",
+            "weight_bytes_per_step": 614629376,
+            "launch": "one qgemv_batched_argmax launch per step, captured once in a CUDA graph and replayed; "
+                      "e2e calls the API eagerly",
             "l2": "inputs larger than L2 (615 MB of weights per step vs 126 MB L2); no flush",
             "parallelism": "replicas"}
 
@@ -403,8 +405,28 @@ def time_decode_step(args, world, dev):
     greedy = bqg.ArgmaxState(dev)
     head = len(specs) - 1
 
-    def step():
+    def step_eager():
         batch.run(argmax=(head, greedy))
+
+    # The decode step as an engine runs it: the public call captured once into a CUDA graph
+    # (the pages' captured decode graph) and replayed per step, so the host's per-call
+    # marshalling (155 descriptors, a 30 KB parameter block) does not starve the GPU.
+    def capture(fn):
+        cs = torch.cuda.Stream()
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cs):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            fn()
+        torch.cuda.synchronize()
+        return g
+    g_step = capture(step_eager)
+    g_plain = capture(batch.run)
+
+    def step():
+        g_step.replay()
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(physical_gpu(torch.cuda.current_device()))
     clocks.start()
@@ -434,12 +456,12 @@ def time_decode_step(args, world, dev):
     launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     total_ms = max_over_ranks(total_ms, world)
 
-    # the same step without the greedy token (the cost of the fused argmax)
+    # the same step without the greedy token (the cost of the fused argmax), same graph replay
     n_plain = max(20, min(args.steps, 500))
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     for _ in range(n_plain):
-        batch.run()
+        g_plain.replay()
     p1.record(stream)
     torch.cuda.synchronize()
     plain_ms = p0.elapsed_time(p1) / n_plain
@@ -451,9 +473,9 @@ def time_decode_step(args, world, dev):
     tok_host = torch.empty(1, dtype=torch.int32, pin_memory=True)
     val_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
 
-    def e2e_step():
+    def e2e_step():  # eager: the public call itself every step
         W.x_all.copy_(x_host, non_blocking=True)
-        step()
+        step_eager()
         tok_host.copy_(greedy.token, non_blocking=True)
         val_host.copy_(greedy.value, non_blocking=True)
     e_steps = max(10, min(args.steps, 500))
@@ -478,6 +500,7 @@ def time_decode_step(args, world, dev):
     legs = {"h2d_us": ev[1].elapsed_time(ev[2]) * 1e3 / e_steps, "d2h_us": ev[2].elapsed_time(ev[3]) * 1e3 / e_steps}
     assert int(tok_host.item()) == int(torch.argmax(W.y(head)).item())
     barrier(world)
+    del g_step, g_plain
     return dict(W=W, total_ms=total_ms, launch_ms=launch_ms, clocks=clk, e2e_ms=e2e_ms, plain_ms=plain_ms,
                 legs=legs, h2d=x_host.numel() * 4, d2h=4 + 4)
 

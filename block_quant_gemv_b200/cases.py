@@ -1,6 +1,6 @@
 """Runs one hot-path case a few times on cuda:0, for profilers (ncu) and quick timing.
 
-    python -m block_quant_gemv_b200.cases decode  [--layers 22] [--iters 5]
+    python -m block_quant_gemv_b200.cases decode  [--layers 22] [--argmax] [--iters 5]
     python -m block_quant_gemv_b200.cases prefill [--tokens 128] [--n 14336] [--k 4096] [--iters 5]
     python -m block_quant_gemv_b200.cases moe gemma|glm [--tokens 1] [--experts E] [--path P] [--iters 5]
 
@@ -46,8 +46,14 @@ def _time(fn, iters: int) -> float:
 def decode(args) -> str:
     W = wl.build_gemv_workload(wl.decode_step_specs(args.layers), seed=0, device="cuda")
     batch = bqg.GemvBatch(W.items())
-    us = _time(batch.run, args.iters)
-    return f"decode step ({args.layers} layers + head, {W.weight_bytes} weight bytes): {us:.1f} us per call"
+    if args.argmax:  # the greedy token of the LM head (the last descriptor) in the same launch
+        out = bqg.ArgmaxState("cuda")
+        head = len(W.specs) - 1
+        us = _time(lambda: batch.run(argmax=(head, out)), args.iters)
+    else:
+        us = _time(batch.run, args.iters)
+    return (f"decode step ({args.layers} layers + head{' + greedy token' if args.argmax else ''}, "
+            f"{W.weight_bytes} weight bytes): {us:.1f} us per call")
 
 
 def prefill(args) -> str:
@@ -90,6 +96,7 @@ def main(argv=None):
     sub = ap.add_subparsers(dest="case", required=True)
     d = sub.add_parser("decode")
     d.add_argument("--layers", type=int, default=22)
+    d.add_argument("--argmax", action="store_true", help="also compute the greedy token of the LM head")
     p = sub.add_parser("prefill")
     p.add_argument("--tokens", type=int, default=128)
     p.add_argument("--n", type=int, default=14336)
