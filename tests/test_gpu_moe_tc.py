@@ -2,7 +2,7 @@
 the float64 oracle, through the C ABI, and against the CUDA-core path on the same inputs.
 
 The shapes cover every weight format as routed and as shared expert, rows whose byte length
-needs 1, 2 or 4 rows per tensor-map super-row, partial 128-row tiles, experts with more than 64
+needs 1, 2 or 4 rows per tensor-map super-row, partial 128-row tiles, experts with more than 128
 tokens (several token chunks per item) and the full-size Gemma-like and GLM-like geometry.
 
 Tolerance: the benchmark spec's bound 2e-3 * max|y_ref|, and a stricter bound derived from the
@@ -52,7 +52,7 @@ def _route(spec, seed, tokens):
 
 
 @pytest.mark.parametrize("spec", TC_SPECS, ids=lambda s: s.name)
-@pytest.mark.parametrize("tokens", [1, 16, 40, 100])
+@pytest.mark.parametrize("tokens", [1, 16, 40, 100, 200])
 def test_tc_small_matches_oracle(spec, tokens):
     need_gpu()
     L, lay = _layer(spec, bqg.MOE_PATH_TENSOR_CORES)
