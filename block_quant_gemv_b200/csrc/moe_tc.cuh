@@ -8,28 +8,28 @@
 // each expert read serves every row routed to it; routed experts split from the dense shared
 // branch); Camelid README, "Gemma 4" (GeGLU experts; dense shared expert + sparse top-8 branch).
 //
-// One work item = up to 128 tokens of one expert (or of the shared expert) times two 128-row
-// weight tiles: the gate and up tiles of the same rows (gate/up phase), or two consecutive tiles
-// of the down matrix (down phase).  The tokens sit on the MMA's M side (128) and the 256 weight
-// rows on N: a tcgen05.mma instruction costs about the same whatever its N, and M = 128 x N = 256
-// x K = 16 covers twice the weights of weights-on-M.  Each CTA (one per SM) runs items claimed
-// from a counter, with warp-specialised roles:
+// One work item = up to 64 tokens of one expert (or of the shared expert) times two 128-row
+// weight tiles: the gate and up tiles of the same rows (gate/up phase), or two consecutive
+// tiles of the down matrix (down phase).  Weight rows sit on the MMA's M side (128), the item's
+// tokens on N (16..64, padded to 16), k along the matrix columns.  Each CTA (one per SM) runs
+// items claimed from a counter, with warp-specialised roles:
 //   warp 0      TMA: raw weight chunks (128 rows x 128 or 64 k of each tile, in their block
 //               format) through a ring in shared memory.  A 3-D tensor map with 8-byte elements
 //               views each family as [expert][super-row][bytes], a super-row being g = 1, 2 or 4
 //               consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of 704
 //               values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
-//   warp 14     TMA: the item's activation rows (fp16, 128-byte swizzle, k-major) per 64-k stage:
-//               the A operand.
+//   warp 14     TMA: the item's activation rows (fp16, 128-byte swizzle, k-major) per 64-k stage.
 //   warps 2-9   dequantize: thread (tile f, row r) turns its row's 64 weights of a stage into fp16
-//               and writes them into the B operand (256 rows, 128-byte swizzle, k-major).
-//   warp 1      allocates all 512 tensor-memory columns and issues tcgen05.mma (kind::f16, both
-//               operands in shared memory, fp32 accumulation): two accumulator buffers of 128
-//               lanes (tokens) x 256 columns (weight rows), so the epilogue of one item overlaps
-//               the MMAs of the next.
-//   warps 10-13 epilogue: read the accumulator rows of the item's tokens (tcgen05.ld), apply int4
-//               row scales, and write h = act(g) * u as fp16 (gate/up) or the fp32 per-pair
-//               outputs (down), one token row per thread.
+//               and stores them with tcgen05.st straight into TENSOR MEMORY (lane r), where the
+//               MMA reads its A operand.  Keeping A out of shared memory matters: 4-bit weights
+//               expanded to fp16 in shared memory would cost ~4 bytes of shared-memory traffic
+//               per weight (store + MMA read), more than the SM moves at the HBM rate.
+//   warp 1      allocates all 512 tensor-memory columns and issues tcgen05.mma (kind::f16, A from
+//               tensor memory, B from shared memory, fp32 accumulation): 4 A stages of 2 x 32
+//               columns, and two accumulator buffers of 2 x 64 columns, so the epilogue of one
+//               item overlaps the MMAs of the next.
+//   warps 10-13 epilogue: read the accumulators (tcgen05.ld), apply int4 row scales, and write
+//               h = act(g) * u as fp16 (gate/up) or the fp32 per-pair outputs (down).
 //
 // Weights become fp16 exactly as stored values allow: Q4_0 (q - 8) and Q8_0 q exactly via the
 // fp16 exponent-bias identity (0x6400 | byte = 1024 + byte), then one rounding of the product by
@@ -51,22 +51,19 @@ namespace bqg {
 constexpr int kTcThreads = 480;            // 15 warps
 constexpr int kTcWarpRaw = 0, kTcWarpMma = 1, kTcWarpDq = 2, kTcWarpEpi = 10, kTcWarpB = 14;
 constexpr int kTcDqThreads = 256;          // 2 tiles x 128 rows
-constexpr int kTcNMax = 128;               // tokens per item (MMA M)
-constexpr int kTcAStages = 3;              // activation stages (A operand)
-constexpr int kTcBStages = 2;              // dequantized weight stages (B operand)
-constexpr int kTcAStageBytes = kTcNMax * 128;  // 128 rows x 64 k fp16
-constexpr int kTcBStageBytes = 256 * 128;      // 256 weight rows x 64 k fp16
+constexpr int kTcNMax = 64;                // tokens per item (MMA N <= 64)
+constexpr int kTcAStages = 4;              // A stages in tensor memory
+constexpr int kTcBStages = 4;              // activation stages in shared memory
+constexpr int kTcBStageBytes = kTcNMax * 128;  // 64 rows x 64 k fp16
 constexpr int kTcDescs = 8;                // item descriptor ring
 constexpr int kTcRawMax = 12;              // raw weight ring depth (runtime, by window size)
-constexpr int kTcDescReaders = 1 + 1 + 8 + 4;  // A producer, MMA, dequant warps, epilogue warps
-// smem: [1 KB alignment slack][A ring][B ring][raw ring][barriers + descriptors][row scales]
+constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (A stages use 0..255)
+constexpr int kTcDescReaders = 1 + 1 + 8 + 4;  // B producer, MMA, dequant warps, epilogue warps
+// smem: [1 KB alignment slack][B ring][raw ring][barriers + descriptors]
 constexpr int kTcBarBytes = 1024;
-constexpr int kTcScaleBytes = 256 * 4;
-constexpr size_t kTcFixedSmem = 1024 + size_t(kTcAStages) * kTcAStageBytes + size_t(kTcBStages) * kTcBStageBytes +
-                                kTcBarBytes + kTcScaleBytes;
+constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBStages) * kTcBStageBytes + kTcBarBytes;
 constexpr size_t kTcMaxSmem = 227 * 1024;
-static_assert((2 * kTcRawMax + 2 * kTcAStages + 2 * kTcBStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <=
-                  kTcBarBytes,
+static_assert((2 * kTcRawMax + 4 * kTcAStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <= kTcBarBytes,
               "barrier area");
 
 // One family of stacked matrices as the kernel sees it (rows on M, cols = k).
@@ -174,21 +171,19 @@ __host__ __device__ __forceinline__ int tc_kpos(int k, int nibble) {
 
 // ---------------------------------------------------------------- the kernel
 // Item descriptor: d0 = (flags: bit0 shared, bit1 second tile present; expert; m0; tokens),
-//                  d1 = (first activation row; activation rows loaded (tokens rounded up to 16);
-//                        first output row; 64-k stages).
+//                  d1 = (first activation row; N; first output row; 64-k stages).
 __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant__ TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_s & 1023)) & 1023);
-  uint8_t* aring = smem;                                            // kTcAStages x 16 KB
-  uint8_t* bring = aring + size_t(kTcAStages) * kTcAStageBytes;    // kTcBStages x 32 KB
+  uint8_t* bring = smem;                                            // kTcBStages x 8 KB
   uint8_t* wring = bring + size_t(kTcBStages) * kTcBStageBytes;    // raw_stages x raw_stage_bytes
   uint64_t* bars = reinterpret_cast<uint64_t*>(wring + size_t(P.raw_stages) * P.raw_stage_bytes);
   uint64_t* raw_full = bars;                        // [kTcRawMax] TMA bytes
   uint64_t* raw_empty = raw_full + kTcRawMax;       // [kTcRawMax] 256 dequant threads
-  uint64_t* a_full = raw_empty + kTcRawMax;         // [kTcAStages] TMA bytes (activations)
+  uint64_t* a_full = raw_empty + kTcRawMax;         // [kTcAStages] 256 dequant threads
   uint64_t* a_empty = a_full + kTcAStages;          // [kTcAStages] MMA commit
-  uint64_t* b_full = a_empty + kTcAStages;          // [kTcBStages] 256 dequant threads
+  uint64_t* b_full = a_empty + kTcAStages;          // [kTcBStages] TMA bytes
   uint64_t* b_empty = b_full + kTcBStages;          // [kTcBStages] MMA commit
   uint64_t* acc_full = b_empty + kTcBStages;        // [2] MMA commit
   uint64_t* acc_empty = acc_full + 2;               // [2] 128 epilogue threads
@@ -198,7 +193,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int4* descs = reinterpret_cast<int4*>(bars + (kTcBarBytes - kTcDescs * 32) / 8);  // [kTcDescs][2]
-  float* scl = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kTcBarBytes);  // [256] row scales
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -207,11 +201,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       mbar_init(&raw_empty[i], kTcDqThreads);
     }
     for (int i = 0; i < kTcAStages; ++i) {
-      mbar_init(&a_full[i], 1);
+      mbar_init(&a_full[i], kTcDqThreads);
       mbar_init(&a_empty[i], 1);
     }
     for (int i = 0; i < kTcBStages; ++i) {
-      mbar_init(&b_full[i], kTcDqThreads);
+      mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -243,6 +237,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
   griddep_launch_dependents();
   griddep_wait();  // routing tables and activation rows come from earlier kernels
 
+  // Readers of the descriptor ring: wait for slot ds, copy, release (lane 0 of each reader warp).
   // Called by lane 0 of a reader warp only (the other lanes get the values by shuffles).
   auto read_desc = [&](int ds, int4& d0, int4& d1) -> bool {
     const int slot = ds % kTcDescs;
@@ -254,10 +249,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
     d1 = ld_desc(&descs[2 * slot + 1]);
     mbar_arrive(&d_empty[slot]);
     return true;
-  };
-  auto bcast = [&](int4 v) {
-    return make_int4(__shfl_sync(0xffffffffu, v.x, 0), __shfl_sync(0xffffffffu, v.y, 0),
-                     __shfl_sync(0xffffffffu, v.z, 0), __shfl_sync(0xffffffffu, v.w, 0));
   };
 
   if (warp == kTcWarpRaw) {
@@ -358,19 +349,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       }
     }
   } else if (warp == kTcWarpB) {
-    // ------------------------------------------------ activation rows (A operand) TMA
+    // ------------------------------------------------ activation rows (B operand) TMA
     if (lane == 0) {
-      int as = 0;
+      int bs = 0;
       bool ok = true;
       for (int ds = 0; ok; ++ds) {
         int4 d0, d1;
         if (!read_desc(ds, d0, d1)) break;
         if (d0.x < 0) break;
         const int sh = d0.x & 1;
-        const int rows = d1.y;
-        for (int s = 0; s < d1.w; ++s, ++as) {
-          const int slot = as % kTcAStages;
-          if (as >= kTcAStages && !mbar_wait(&a_empty[slot], uint32_t(as / kTcAStages - 1) & 1u)) {
+        const int N = d1.y;
+        for (int s = 0; s < d1.w; ++s, ++bs) {
+          const int slot = bs % kTcBStages;
+          if (bs >= kTcBStages && !mbar_wait(&b_empty[slot], uint32_t(bs / kTcBStages - 1) & 1u)) {
             ok = false;
             break;
           }
@@ -378,16 +369,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&a_full[slot], uint32_t(rows * 128));
-          uint8_t* dst = aring + size_t(slot) * kTcAStageBytes;
-          for (int nb = 0; nb < rows / 16; ++nb)
-            tma_load_2d(dst + nb * 2048, &P.bmap[sh], s * 64, d1.x + 16 * nb, &a_full[slot]);
+          mbar_arrive_expect_tx(&b_full[slot], uint32_t(N * 128));
+          uint8_t* dst = bring + size_t(slot) * kTcBStageBytes;
+          for (int nb = 0; nb < N / 16; ++nb)
+            tma_load_2d(dst + nb * 2048, &P.bmap[sh], s * 64, d1.x + 16 * nb, &b_full[slot]);
         }
       }
       if (!ok) {
         *abort_flag = 1;
-        for (int q = (as > kTcAStages ? as - kTcAStages : 0); q < as; ++q)
-          mbar_wait(&a_full[q % kTcAStages], uint32_t(q / kTcAStages) & 1u);
+        for (int q = (bs > kTcBStages ? bs - kTcBStages : 0); q < bs; ++q)
+          mbar_wait(&b_full[q % kTcBStages], uint32_t(q / kTcBStages) & 1u);
       }
     }
   } else if (warp == kTcWarpMma) {
@@ -406,8 +397,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = umma_idesc_f16(128, two ? 256 : 128);
-        const uint32_t dcol = tmem + uint32_t(buf * 256);
+        const uint32_t idesc = umma_idesc_f16(128, d1.y);
+        const uint32_t dcol = tmem + uint32_t(kTcAccCol + buf * 128);
         for (int s = 0; s < d1.w; ++s, ++as, ++bs) {
           const int aslot = as % kTcAStages, bslot = bs % kTcBStages;
           if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u) ||
@@ -416,12 +407,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             break;
           }
           tc_fence_after();
-          const uint32_t a_s = smem_u32(aring + size_t(aslot) * kTcAStageBytes);
+          const uint32_t acol = tmem + uint32_t(aslot * 64);
           const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // 16 k per MMA: 32 bytes of each 128-byte swizzled row
-            umma_f16(dcol, umma_desc_sw128(a_s + 32 * kk), umma_desc_sw128(b_s + 32 * kk), idesc,
-                     (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {  // 16 k per MMA: 8 tensor-memory columns, 32 bytes of B
+            const uint64_t bdesc = umma_desc_sw128(b_s + 32 * kk);
+            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+            umma_f16_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);
+            if (two) umma_f16_ts(dcol + 64, acol + 32 + 8 * kk, bdesc, idesc, acc);
+          }
           umma_commit(&a_empty[aslot]);
           umma_commit(&b_empty[bslot]);
         }
@@ -433,26 +427,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       mbar_wait(done, 0);
     }
   } else if (warp < kTcWarpEpi) {
-    // ------------------------------------------------ dequantize into the B operand
-    const int dw = warp - kTcWarpDq;          // 0..7
-    const int f = dw >> 2;                    // tile 0 (warps 2-5) or tile 1 (warps 6-9)
-    const int r = 32 * (dw & 3) + lane;       // row of the tile
-    const int R = f * 128 + r;                // row of the B operand (N index)
-    const uint32_t b_row = uint32_t(R >> 3) * 1024 + uint32_t(R & 7) * 128;
-    const int sw = R & 7;                     // 128-byte swizzle: chunk c of row R at chunk c ^ (R % 8)
+    // ------------------------------------------------ dequantize into tensor memory
+    const int f = (warp - kTcWarpDq) >> 2;    // tile 0 (warps 2-5) or tile 1 (warps 6-9)
+    const int qw = warp & 3;                  // tensor-memory lane quarter this warp may access
+    const int r = 32 * qw + lane;             // row of the tile = tensor-memory lane
+    const uint32_t tlane = uint32_t(32 * qw) << 16;
     const uint32_t wring_s = smem_u32(wring);
-    int rp = 0, bs = 0;
+    int rp = 0, as = 0;
     bool ok = true;
     for (int ds = 0; ok; ++ds) {
+      int4 d0, d1;
       int4 dd0 = make_int4(0, 0, 0, 0), dd1 = dd0;
       if (lane == 0 && !read_desc(ds, dd0, dd1)) dd0.x = -2;
-      const int4 d0 = bcast(dd0), d1 = bcast(dd1);
+      d0.x = __shfl_sync(0xffffffffu, dd0.x, 0);
+      d0.y = __shfl_sync(0xffffffffu, dd0.y, 0);
+      d0.z = __shfl_sync(0xffffffffu, dd0.z, 0);
+      d1.w = __shfl_sync(0xffffffffu, dd1.w, 0);
       if (d0.x < 0) break;
       const int fb = (d0.x & 1) ? 2 : 0;
       const bool tile_on = f == 0 || ((d0.x >> 1) & 1);
       const TcFam& F = P.fam[fb + f];
       const TcFam& F0 = P.fam[fb];
-      const bool row_on = tile_on && d0.z + F.m_off + r < F.rows;
+      const bool row_on = tile_on && d0.z + F.m_off + r < F.rows;  // warp-uniform (rows % 32 == 0)
       const int g = F.g, j = r % g, q = r / g;
       const uint32_t row_off = uint32_t(f * 128 * F.win + j * (128 / g) * F.win + q * F.win);
       const int spr = F0.raw_k / 64;  // MMA stages per raw chunk
@@ -465,125 +461,101 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         }
         const uint32_t mis = uint32_t(j * F.row_bytes + kc * F.cb) & 15u;
         const uint32_t rbase = wring_s + uint32_t(slot_r) * P.raw_stage_bytes + row_off + mis;
-        for (int h = 0; h < spr && kc * spr + h < d1.w; ++h, ++bs) {
-          const int bslot = bs % kTcBStages;
-          if (bs >= kTcBStages && !mbar_wait(&b_empty[bslot], uint32_t(bs / kTcBStages - 1) & 1u)) {
+        for (int h = 0; h < spr && kc * spr + h < d1.w; ++h, ++as) {
+          const int aslot = as % kTcAStages;
+          if (as >= kTcAStages && !mbar_wait(&a_empty[aslot], uint32_t(as / kTcAStages - 1) & 1u)) {
             ok = false;
             break;
           }
-          // rows past the matrix (a partial tile) or of an absent second tile are left as they
-          // are: they only feed accumulator columns that nothing reads
+          tc_fence_after();
           if (row_on) {
             uint32_t o[32];
             tc_dequant64(F.fmt, rbase + uint32_t(h * (F.cb / spr)), o);
-            const uint32_t dst = smem_u32(bring + size_t(bslot) * kTcBStageBytes) + b_row;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              sts128(dst + uint32_t((c ^ sw) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            const uint32_t taddr = tmem + tlane + uint32_t(aslot * 64 + f * 32);
+            tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(&o[0]));
+            tmem_st16(taddr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&o[16]));
+            tmem_wait_st();
           }
-          fence_proxy_async_smem();  // make the fp16 rows visible to the tensor core
-          mbar_arrive(&b_full[bslot]);
+          tc_fence_before();
+          mbar_arrive(&a_full[aslot]);
         }
         mbar_arrive(&raw_empty[slot_r]);
       }
     }
     if (!ok) *abort_flag = 1;
   } else {
-    // ------------------------------------------------ epilogue: one token row per thread
+    // ------------------------------------------------ epilogue
     const int qw = warp & 3;
-    const int t = 32 * qw + lane;            // token of the item = accumulator lane
+    const int r = 32 * qw + lane;
     const uint32_t tlane = uint32_t(32 * qw) << 16;
-    const int et = threadIdx.x - kTcWarpEpi * 32;  // 0..127
     bool ok = true;
     for (int it = 0; ok; ++it) {
+      int4 d0, d1;
       int4 dd0 = make_int4(0, 0, 0, 0), dd1 = dd0;
       if (lane == 0 && !read_desc(it, dd0, dd1)) dd0.x = -2;
-      const int4 d0 = bcast(dd0), d1 = bcast(dd1);
+      d0 = make_int4(__shfl_sync(0xffffffffu, dd0.x, 0), __shfl_sync(0xffffffffu, dd0.y, 0),
+                     __shfl_sync(0xffffffffu, dd0.z, 0), __shfl_sync(0xffffffffu, dd0.w, 0));
+      d1 = make_int4(__shfl_sync(0xffffffffu, dd1.x, 0), __shfl_sync(0xffffffffu, dd1.y, 0),
+                     __shfl_sync(0xffffffffu, dd1.z, 0), __shfl_sync(0xffffffffu, dd1.w, 0));
       if (d0.x < 0) break;
       const int sh = d0.x & 1, two = (d0.x >> 1) & 1;
       const int fb = sh ? 2 : 0;
-      const int ntok = d0.w, obase = d1.z;
+      const int ntok = d0.w, N = d1.y, obase = d1.z;
       const int buf = it & 1;
-      // int4 row scales of the item's 256 weight rows, staged once in shared memory
-      const bool i4 = P.fam[fb].fmt == BQG_I4_ROW;
-      if (i4) {
-        named_bar_sync(2, 128);  // the previous item's scales are no longer read
-        for (int i = et; i < 256; i += 128) {
-          const int f = i >> 7;
-          const TcFam& F = P.fam[fb + f];
-          const int row = d0.z + F.m_off + (i & 127);
-          float v = 0.f;
-          if ((f == 0 || two) && row < F.rows)
-            v = __ldg(reinterpret_cast<const float*>(F.base + (sh ? 0 : size_t(d0.y) * F.stride) + F.scale_off) + row);
-          scl[i] = v;
-        }
-        named_bar_sync(2, 128);
-      }
       if (!mbar_wait(&acc_full[buf], uint32_t(it / 2) & 1u)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t acc = tmem + tlane + uint32_t(buf * 256);
-      const bool on = t < ntok;
-      if (32 * qw < ntok) {  // warps whose lanes hold no token of this item skip the reads
-        if (P.phase == 0) {
-          const TcFam& G = P.fam[fb];
-          const int nrow = min(128, G.rows - d0.z);  // valid rows of the tile (a multiple of 32)
-          __half* hrow = P.hout[sh] + size_t(obase + t) * P.hstride[sh];
-          for (int c0 = 0; c0 < nrow; c0 += 8) {
-            uint32_t gv[8], uv[8];
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                : "=r"(gv[0]), "=r"(gv[1]), "=r"(gv[2]), "=r"(gv[3]), "=r"(gv[4]), "=r"(gv[5]), "=r"(gv[6]),
-                  "=r"(gv[7])
-                : "r"(acc + uint32_t(c0)));
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                : "=r"(uv[0]), "=r"(uv[1]), "=r"(uv[2]), "=r"(uv[3]), "=r"(uv[4]), "=r"(uv[5]), "=r"(uv[6]),
-                  "=r"(uv[7])
-                : "r"(acc + uint32_t(128 + c0)));
-            tmem_wait_ld();
-            if (on) {
-              float hv[8];
+      const uint32_t acc = tmem + tlane + uint32_t(kTcAccCol + buf * 128);
+      if (P.phase == 0) {
+        const TcFam& G = P.fam[fb];
+        const TcFam& U = P.fam[fb + 1];
+        const int row = d0.z + r;
+        const bool on = row < G.rows;
+        float sg = 1.f, su = 1.f;
+        if (on && G.fmt == BQG_I4_ROW) {
+          sg = __ldg(reinterpret_cast<const float*>(G.base + (sh ? 0 : size_t(d0.y) * G.stride) + G.scale_off) + row);
+          su = __ldg(reinterpret_cast<const float*>(U.base + (sh ? 0 : size_t(d0.y) * U.stride) + U.scale_off) + row);
+        }
+        __half* hrow = P.hout[sh] + tc_kpos(row, P.hperm[sh]);
+        const int hs = P.hstride[sh];
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          uint32_t gv[16], uv[16];
+          tmem_ld16_nowait(acc + uint32_t(c0), gv);
+          tmem_ld16_nowait(acc + uint32_t(64 + c0), uv);
+          tmem_wait_ld();
+          if (on) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float sg = i4 ? scl[c0 + i] : 1.f, su = i4 ? scl[128 + c0 + i] : 1.f;
-                hv[i] = act_fn(P.act, __uint_as_float(gv[i]) * sg) * (__uint_as_float(uv[i]) * su);
+            for (int i = 0; i < 16; ++i) {
+              const int n = c0 + i;
+              if (n < ntok) {
+                const float hv = act_fn(P.act, __uint_as_float(gv[i]) * sg) * (__uint_as_float(uv[i]) * su);
+                hrow[size_t(obase + n) * hs] = __float2half_rn(hv);
               }
-              // the 8 values of rows d0.z + c0 .. + 7 in the down matrix's k order
-              uint32_t o[4];
-              if (P.hperm[sh]) {  // positions 0..7 hold elements 0,4,1,5,2,6,3,7
-                o[0] = h2_bits(__floats2half2_rn(hv[0], hv[4]));
-                o[1] = h2_bits(__floats2half2_rn(hv[1], hv[5]));
-                o[2] = h2_bits(__floats2half2_rn(hv[2], hv[6]));
-                o[3] = h2_bits(__floats2half2_rn(hv[3], hv[7]));
-              } else {
-                o[0] = h2_bits(__floats2half2_rn(hv[0], hv[1]));
-                o[1] = h2_bits(__floats2half2_rn(hv[2], hv[3]));
-                o[2] = h2_bits(__floats2half2_rn(hv[4], hv[5]));
-                o[3] = h2_bits(__floats2half2_rn(hv[6], hv[7]));
-              }
-              *reinterpret_cast<uint4*>(hrow + d0.z + c0) = make_uint4(o[0], o[1], o[2], o[3]);
             }
           }
-        } else {
-          const int orow = on ? (sh ? obase + t : __ldg(P.perm + obase + t)) : 0;
-          float* yrow = P.yout[sh] + size_t(orow) * P.ystride;
-          for (int f = 0; f <= two; ++f) {
-            const TcFam& D = P.fam[fb + f];
-            const int mrow = d0.z + D.m_off;
-            const int nrow = min(128, D.rows - mrow);
-            for (int c0 = 0; c0 < nrow; c0 += 16) {
-              uint32_t v[16];
-              tmem_ld16(acc + uint32_t(f * 128 + c0), v);
-              if (on) {
-                float o[16];
+        }
+      } else {
+        for (int f = 0; f <= two; ++f) {
+          const TcFam& D = P.fam[fb + f];
+          const int row = d0.z + D.m_off + r;
+          const bool on = row < D.rows;
+          float sd = 1.f;
+          if (on && D.fmt == BQG_I4_ROW)
+            sd = __ldg(reinterpret_cast<const float*>(D.base + (sh ? 0 : size_t(d0.y) * D.stride) + D.scale_off) + row);
+          for (int c0 = 0; c0 < N; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16_nowait(acc + uint32_t(f * 64 + c0), v);
+            tmem_wait_ld();
+            if (on) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(v[i]) * (i4 ? scl[f * 128 + c0 + i] : 1.f);
-#pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                  *reinterpret_cast<float4*>(yrow + mrow + c0 + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+              for (int i = 0; i < 16; ++i) {
+                const int n = c0 + i;
+                if (n < ntok) {
+                  const int orow = sh ? obase + n : __ldg(P.perm + obase + n);
+                  P.yout[sh][size_t(orow) * P.ystride + row] = __uint_as_float(v[i]) * sd;
+                }
               }
             }
           }

@@ -2,7 +2,7 @@
 the float64 oracle, through the C ABI, and against the CUDA-core path on the same inputs.
 
 The shapes cover every weight format as routed and as shared expert, rows whose byte length
-needs 1, 2 or 4 rows per tensor-map super-row, partial 128-row tiles, experts with more than 128
+needs 1, 2 or 4 rows per tensor-map super-row, partial 128-row tiles, experts with more than 64
 tokens (several token chunks per item) and the full-size Gemma-like and GLM-like geometry.
 
 Tolerance: the benchmark spec's bound 2e-3 * max|y_ref|, and a stricter bound derived from the
