@@ -46,10 +46,11 @@ def test_peaks_come_from_the_measured_file():
 
 
 def test_committed_traffic_is_gated_by_the_kernel_source_hash(monkeypatch):
-    prof = os.path.join(bench.ROOT, "profiles", "k_qgemv_tinyllama_decode.md")
-    text = open(prof).read()
-    want = int(text.split("traffic_bytes_per_launch: `")[1].split("`")[0])
-    if f"kernel_source_hash: `{bench.kernel_source_hash()}`" in text:
+    import json
+    prof = os.path.join(bench.ROOT, "profiles", "k_qgemv_tinyllama_decode.json")
+    rec = json.load(open(prof))
+    want = int(rec["traffic_bytes_per_launch"])
+    if rec["kernel_source_hash"] == bench.kernel_source_hash():
         assert bench.committed_traffic() == want
     else:
         assert bench.committed_traffic() is None
