@@ -107,12 +107,47 @@ inline MoeWsLayout moe_ws_layout(const bqg_moe_layer* L, int tokens) {
   return o;
 }
 
-// Workspace of the tensor-core path: the same routing tables, then fp16 activation rows (x in
+// The families of a layer on the tensor-core path; false when a shape does not fit it.
+// i8: the kind::i8 variant (every family int4 or int2 with k a multiple of 128).
+struct TcLayer {
+  TcFam gate, up, down0, down1, s_gate, s_up, s_down0, s_down1;
+};
+
+inline bool tc_layer(const bqg_moe_layer* L, TcLayer* T, bool i8) {
+  TcLayer t{};
+  if (!tc_fam(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden, 0, &t.gate, i8) ||
+      !tc_fam(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden, 0, &t.up, i8) ||
+      !tc_fam(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, 0, &t.down0, i8) ||
+      !tc_fam(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, 128, &t.down1, i8))
+    return false;
+  if (L->s_gate != nullptr) {
+    if (!tc_fam(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden, 0, &t.s_gate, i8) ||
+        !tc_fam(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden, 0, &t.s_up, i8) ||
+        !tc_fam(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, 0, &t.s_down0, i8) ||
+        !tc_fam(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, 128, &t.s_down1, i8))
+      return false;
+  }
+  if (T != nullptr) *T = t;
+  return true;
+}
+
+// Which tensor-core variant takes the layer: 1 kind::i8 (int4 / int2 layers), 0 kind::f16, -1 none.
+inline int tc_variant(const bqg_moe_layer* L) {
+  if (tc_layer(L, nullptr, true)) return 1;
+  return tc_layer(L, nullptr, false) ? 0 : -1;
+}
+
+// Workspace of the tensor-core path: the same routing tables, then the activation rows (x in
 // expert-grouped order, x of the shared expert in token order, the gated hidden rows h) and the
-// fp32 per-pair and shared outputs that the combine sums.
+// fp32 per-pair and shared outputs that the combine sums.  kind::f16: fp16 rows.  kind::i8: two
+// int8 digit rows per row (the same bytes), a scale and a digit sum per row, and h in fp32 as
+// the gate/up epilogue writes it.
 struct MoeTcLayout {
+  bool i8;
   size_t counts, offsets, active, n_active, ctr, act_info, perm;
-  size_t xg, xs, hg, hs, part, sout, total;
+  size_t xg, xs, hg, hs, part, sout;
+  size_t xg_sc, xg_sum, xs_sc, xs_sum, h32g, h32s, hg_sc, hg_sum, hs_sc, hs_sum;
+  size_t total;
 };
 
 inline MoeTcLayout moe_ws_layout_tc(const bqg_moe_layer* L, int tokens) {
@@ -132,37 +167,29 @@ inline MoeTcLayout moe_ws_layout_tc(const bqg_moe_layer* L, int tokens) {
   o.ctr = take(8);
   o.act_info = take(16 * E);
   o.perm = take(4 * pairs);
+  o.i8 = tc_variant(L) == 1;
   o.xg = take(2 * pairs * L->hidden);
   o.xs = sh ? take(2 * T * L->hidden) : 0;
   o.hg = take(2 * pairs * L->inter);
   o.hs = sh ? take(2 * T * L->shared_inter) : 0;
   o.part = take(4 * pairs * L->hidden);
   o.sout = sh ? take(4 * T * L->hidden) : 0;
+  if (o.i8) {
+    o.xg_sc = take(4 * pairs);
+    o.xg_sum = take(4 * pairs);
+    o.hg_sc = take(4 * pairs);
+    o.hg_sum = take(4 * pairs);
+    o.h32g = take(4 * pairs * L->inter);
+    if (sh) {
+      o.xs_sc = take(4 * T);
+      o.xs_sum = take(4 * T);
+      o.hs_sc = take(4 * T);
+      o.hs_sum = take(4 * T);
+      o.h32s = take(4 * T * L->shared_inter);
+    }
+  }
   o.total = off;
   return o;
-}
-
-// The families of a layer on the tensor-core path; false when a shape does not fit it.
-struct TcLayer {
-  TcFam gate, up, down0, down1, s_gate, s_up, s_down0, s_down1;
-};
-
-inline bool tc_layer(const bqg_moe_layer* L, TcLayer* T) {
-  TcLayer t{};
-  if (!tc_fam(L->expert_fmt, L->gate, L->gate_stride, L->inter, L->hidden, 0, &t.gate) ||
-      !tc_fam(L->expert_fmt, L->up, L->up_stride, L->inter, L->hidden, 0, &t.up) ||
-      !tc_fam(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, 0, &t.down0) ||
-      !tc_fam(L->expert_fmt, L->down, L->down_stride, L->hidden, L->inter, 128, &t.down1))
-    return false;
-  if (L->s_gate != nullptr) {
-    if (!tc_fam(L->shared_fmt, L->s_gate, 0, L->shared_inter, L->hidden, 0, &t.s_gate) ||
-        !tc_fam(L->shared_fmt, L->s_up, 0, L->shared_inter, L->hidden, 0, &t.s_up) ||
-        !tc_fam(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, 0, &t.s_down0) ||
-        !tc_fam(L->shared_fmt, L->s_down, 0, L->hidden, L->shared_inter, 128, &t.s_down1))
-      return false;
-  }
-  if (T != nullptr) *T = t;
-  return true;
 }
 
 // The automatic choice.  A tensor-core MMA instruction (M = 128 weight rows, K = 16) costs about
@@ -180,7 +207,7 @@ inline bool moe_tc_preferred(const bqg_moe_layer* L, int tokens) {
 // Path for `tokens` tokens: BQG_MOE_PATH_CUDA_CORES or BQG_MOE_PATH_TENSOR_CORES (negative: error).
 inline int moe_path(const bqg_moe_layer* L, int tokens) {
   if (L->path == BQG_MOE_PATH_CUDA_CORES) return BQG_MOE_PATH_CUDA_CORES;
-  const bool tc = tc_layer(L, nullptr);
+  const bool tc = tc_variant(L) >= 0;
   if (L->path == BQG_MOE_PATH_TENSOR_CORES) return tc ? int(BQG_MOE_PATH_TENSOR_CORES) : int(BQG_ERR_SHAPE);
   return (tc && moe_tc_preferred(L, tokens)) ? BQG_MOE_PATH_TENSOR_CORES : BQG_MOE_PATH_CUDA_CORES;
 }
@@ -252,9 +279,17 @@ inline int quant_grid(long long threads, int cap) {
 }
 
 // One grouped-GEMM launch (phase 0 gate/up, 1 down) of the tensor-core path.
+// kind::i8 extras of one launch: per activation row scales and digit sums, fp32 h outputs.
+struct TcI8Args {
+  const float* bscale[2];
+  const int32_t* bsum[2];
+  float* h32[2];
+};
+
 inline int launch_moe_tc(const bqg_moe_layer* L, const TcLayer& TL, int phase, int tokens, const RouteWs& route,
-                         const __half* b_routed, const __half* b_shared, __half* h_routed, __half* h_shared,
-                         float* part, float* sout, int dev, const DeviceInfo* info, cudaStream_t s) {
+                         const void* b_routed, const void* b_shared, __half* h_routed, __half* h_shared,
+                         float* part, float* sout, const TcI8Args* i8, int dev, const DeviceInfo* info,
+                         cudaStream_t s) {
   const bool sh = L->s_gate != nullptr;
   const int pairs = tokens * L->top_k;
   TcParams P{};
@@ -276,12 +311,23 @@ inline int launch_moe_tc(const bqg_moe_layer* L, const TcLayer& TL, int phase, i
   }
   const int kb = phase == 0 ? L->hidden : L->inter;
   const int kbs = phase == 0 ? L->hidden : L->shared_inter;
-  if ((st = tc_encode_bmap(&P.bmap[0], b_routed, pairs, kb)) != BQG_OK) return st;
-  if (sh) {
-    if ((st = tc_encode_bmap(&P.bmap[1], b_shared, tokens, kbs)) != BQG_OK) return st;
+  if (i8 != nullptr) {
+    if ((st = tc_encode_bmap_i8(&P.bmap[0], static_cast<const int8_t*>(b_routed), 2 * pairs, kb)) != BQG_OK) return st;
+    if (sh && (st = tc_encode_bmap_i8(&P.bmap[1], static_cast<const int8_t*>(b_shared), 2 * tokens, kbs)) != BQG_OK)
+      return st;
+    for (int i = 0; i < 2; ++i) {
+      P.bscale[i] = i8->bscale[i];
+      P.bsum[i] = i8->bsum[i];
+      P.h32[i] = i8->h32[i];
+    }
+    P.nmax = kTcNMax / 2;
   } else {
-    P.bmap[1] = P.bmap[0];
+    if ((st = tc_encode_bmap(&P.bmap[0], static_cast<const __half*>(b_routed), pairs, kb)) != BQG_OK) return st;
+    if (sh && (st = tc_encode_bmap(&P.bmap[1], static_cast<const __half*>(b_shared), tokens, kbs)) != BQG_OK)
+      return st;
+    P.nmax = kTcNMax;
   }
+  if (!sh) P.bmap[1] = P.bmap[0];
   P.phase = phase;
   P.act = L->act;
   P.tokens = tokens;
@@ -304,9 +350,13 @@ inline int launch_moe_tc(const bqg_moe_layer* L, const TcLayer& TL, int phase, i
   P.yout[0] = part;
   P.yout[1] = sout;
   P.ystride = L->hidden;
-  if ((st = g_tc_attr.ensure(dev, k_moe_tc, kTcMaxSmem)) != BQG_OK) return st;
-  return launch_pdl(k_moe_tc, dim3(info->sm_count), dim3(kTcThreads), tc_smem_bytes(P.raw_stages, P.raw_stage_bytes),
-                    s, P);
+  const size_t smem = tc_smem_bytes(P.raw_stages, P.raw_stage_bytes);
+  if (i8 != nullptr) {
+    if ((st = g_tc_attr_i8.ensure(dev, k_moe_tc<true>, kTcMaxSmem)) != BQG_OK) return st;
+    return launch_pdl(k_moe_tc<true>, dim3(info->sm_count), dim3(kTcThreads), smem, s, P);
+  }
+  if ((st = g_tc_attr.ensure(dev, k_moe_tc<false>, kTcMaxSmem)) != BQG_OK) return st;
+  return launch_pdl(k_moe_tc<false>, dim3(info->sm_count), dim3(kTcThreads), smem, s, P);
 }
 
 }  // namespace bqg
@@ -317,8 +367,9 @@ namespace bqg {
 inline int moe_forward_tc(const bqg_moe_layer* L, const float* x, const int32_t* idx, const float* w, float* y,
                           int tokens, uint8_t* ws, int dev, const DeviceInfo* info, cudaStream_t s, int skip_negative,
                           int accumulate) {
+  const int variant = tc_variant(L);
   TcLayer TL;
-  if (!tc_layer(L, &TL)) return BQG_ERR_SHAPE;
+  if (variant < 0 || !tc_layer(L, &TL, variant == 1)) return BQG_ERR_SHAPE;
   const MoeTcLayout lay = moe_ws_layout_tc(L, tokens);
   const bool sh = L->s_gate != nullptr;
   const int pairs = tokens * L->top_k;
@@ -340,21 +391,63 @@ inline int moe_forward_tc(const bqg_moe_layer* L, const float* x, const int32_t*
   if ((st = launch_pdl(k_moe_prep, dim3(1), dim3(kRouteThreads), 0, s, idx, pairs, L->n_experts, route, none)) !=
       BQG_OK)
     return st;
-  // 2. activation rows in fp16 (grouped order for the routed experts, token order for the shared one)
-  const long long chunks = (long long)(pairs + (sh ? tokens : 0)) * (L->hidden / 8);
-  if ((st = launch_pdl(k_moe_xprep, dim3(quant_grid(chunks, 4 * info->sm_count)), dim3(256), 0, s, x,
-                       (const int32_t*)route.perm, (const int32_t*)route.offsets, L->n_experts, L->top_k, tokens,
-                       L->hidden, H(lay.xg), int(L->expert_fmt != BQG_Q8_0), sh ? H(lay.xs) : (__half*)nullptr,
-                       int(sh && L->shared_fmt != BQG_Q8_0))) != BQG_OK)
-    return st;
-  // 3. gate/up with h = act(g) * u in the epilogue
-  if ((st = launch_moe_tc(L, TL, 0, tokens, route, H(lay.xg), sh ? H(lay.xs) : nullptr, H(lay.hg),
-                          sh ? H(lay.hs) : nullptr, nullptr, nullptr, dev, info, s)) != BQG_OK)
-    return st;
-  // 4. down
-  if ((st = launch_moe_tc(L, TL, 1, tokens, route, H(lay.hg), sh ? H(lay.hs) : nullptr, nullptr, nullptr, F(lay.part),
-                          sh ? F(lay.sout) : nullptr, dev, info, s)) != BQG_OK)
-    return st;
+  if (lay.i8) {
+    // kind::i8: int8 digit rows of x, gate/up (h in fp32), digit rows of h, down
+    auto B = [&](size_t o) { return reinterpret_cast<int8_t*>(ws + o); };
+    auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
+    const int rows_grid = quant_grid((long long)pairs * 32, 4 * info->sm_count);
+    const int rows_grid_s = quant_grid((long long)tokens * 32, 4 * info->sm_count);
+    const int32_t* routed_rows = route.offsets + L->n_experts;
+    if ((st = launch_pdl(k_moe_digits, dim3(rows_grid), dim3(256), 0, s, x, (const int32_t*)route.perm, L->top_k,
+                         routed_rows, 0, L->hidden, L->expert_fmt, B(lay.xg), F(lay.xg_sc), I(lay.xg_sum))) != BQG_OK)
+      return st;
+    if (sh && (st = launch_pdl(k_moe_digits, dim3(rows_grid_s), dim3(256), 0, s, x, (const int32_t*)nullptr, 1,
+                               (const int32_t*)nullptr, tokens, L->hidden, L->shared_fmt, B(lay.xs), F(lay.xs_sc),
+                               I(lay.xs_sum))) != BQG_OK)
+      return st;
+    TcI8Args a0{};
+    a0.bscale[0] = F(lay.xg_sc);
+    a0.bsum[0] = I(lay.xg_sum);
+    a0.bscale[1] = sh ? F(lay.xs_sc) : nullptr;
+    a0.bsum[1] = sh ? I(lay.xs_sum) : nullptr;
+    a0.h32[0] = F(lay.h32g);
+    a0.h32[1] = sh ? F(lay.h32s) : nullptr;
+    if ((st = launch_moe_tc(L, TL, 0, tokens, route, B(lay.xg), sh ? B(lay.xs) : nullptr, nullptr, nullptr, nullptr,
+                            nullptr, &a0, dev, info, s)) != BQG_OK)
+      return st;
+    if ((st = launch_pdl(k_moe_digits, dim3(rows_grid), dim3(256), 0, s, (const float*)F(lay.h32g),
+                         (const int32_t*)nullptr, 1, routed_rows, 0, L->inter, L->expert_fmt, B(lay.hg),
+                         F(lay.hg_sc), I(lay.hg_sum))) != BQG_OK)
+      return st;
+    if (sh && (st = launch_pdl(k_moe_digits, dim3(rows_grid_s), dim3(256), 0, s, (const float*)F(lay.h32s),
+                               (const int32_t*)nullptr, 1, (const int32_t*)nullptr, tokens, L->shared_inter,
+                               L->shared_fmt, B(lay.hs), F(lay.hs_sc), I(lay.hs_sum))) != BQG_OK)
+      return st;
+    TcI8Args a1{};
+    a1.bscale[0] = F(lay.hg_sc);
+    a1.bsum[0] = I(lay.hg_sum);
+    a1.bscale[1] = sh ? F(lay.hs_sc) : nullptr;
+    a1.bsum[1] = sh ? I(lay.hs_sum) : nullptr;
+    if ((st = launch_moe_tc(L, TL, 1, tokens, route, B(lay.hg), sh ? B(lay.hs) : nullptr, nullptr, nullptr,
+                            F(lay.part), sh ? F(lay.sout) : nullptr, &a1, dev, info, s)) != BQG_OK)
+      return st;
+  } else {
+    // 2. activation rows in fp16 (grouped order for the routed experts, token order for the shared one)
+    const long long chunks = (long long)(pairs + (sh ? tokens : 0)) * (L->hidden / 8);
+    if ((st = launch_pdl(k_moe_xprep, dim3(quant_grid(chunks, 4 * info->sm_count)), dim3(256), 0, s, x,
+                         (const int32_t*)route.perm, (const int32_t*)route.offsets, L->n_experts, L->top_k, tokens,
+                         L->hidden, H(lay.xg), int(L->expert_fmt != BQG_Q8_0), sh ? H(lay.xs) : (__half*)nullptr,
+                         int(sh && L->shared_fmt != BQG_Q8_0))) != BQG_OK)
+      return st;
+    // 3. gate/up with h = act(g) * u in the epilogue
+    if ((st = launch_moe_tc(L, TL, 0, tokens, route, H(lay.xg), sh ? H(lay.xs) : nullptr, H(lay.hg),
+                            sh ? H(lay.hs) : nullptr, nullptr, nullptr, nullptr, dev, info, s)) != BQG_OK)
+      return st;
+    // 4. down
+    if ((st = launch_moe_tc(L, TL, 1, tokens, route, H(lay.hg), sh ? H(lay.hs) : nullptr, nullptr, nullptr,
+                            F(lay.part), sh ? F(lay.sout) : nullptr, nullptr, dev, info, s)) != BQG_OK)
+      return st;
+  }
   // 5. combine
   const long long n = (long long)tokens * L->hidden;
   return launch_pdl(k_moe_combine, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s, (const float*)F(lay.part), idx, w,

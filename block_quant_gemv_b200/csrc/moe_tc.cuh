@@ -13,21 +13,29 @@
 // tiles of the down matrix (down phase).  Weight rows sit on the MMA's M side (128), the item's
 // tokens on N (16..64, padded to 16), k along the matrix columns.  Each CTA (one per SM) runs
 // items claimed from a counter, with warp-specialised roles:
-//   warp 0      TMA: raw weight chunks (128 rows x 128 or 64 k of each tile, in their block
-//               format) through a ring in shared memory.  A 3-D tensor map with 8-byte elements
-//               views each family as [expert][super-row][bytes], a super-row being g = 1, 2 or 4
-//               consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of 704
-//               values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
+//   warp 0      TMA: raw weight chunks (128 rows of each tile, 144 to 256 bytes of each row, in
+//               their block format) through a ring in shared memory.  A 3-D tensor map with 8-byte
+//               elements views each family as [expert][super-row][bytes], a super-row being g = 1,
+//               2 or 4 consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of
+//               704 values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
+//               The copy engine's time grows with the number of row segments a box holds, so each
+//               chunk takes a long piece of every row (64-byte pieces measured ~7 cycles each).
+//               Rows land in shared memory an odd multiple of 16 bytes apart (176 or 208), so the
+//               dequantizing threads' 16-byte loads of consecutive rows hit distinct bank groups
+//               (a 64- or 256-byte pitch put 4 or 8 rows on the same banks).
 //   warp 14     TMA: the item's activation rows (fp16, 128-byte swizzle, k-major) per 64-k stage.
 //   warps 2-9   dequantize: thread (tile f, row r) turns its row's 64 weights of a stage into fp16
 //               and stores them with tcgen05.st straight into TENSOR MEMORY (lane r), where the
 //               MMA reads its A operand.  Keeping A out of shared memory matters: 4-bit weights
 //               expanded to fp16 in shared memory would cost ~4 bytes of shared-memory traffic
 //               per weight (store + MMA read), more than the SM moves at the HBM rate.
-//   warp 1      allocates all 512 tensor-memory columns and issues tcgen05.mma (kind::f16, A from
-//               tensor memory, B from shared memory, fp32 accumulation): 4 A stages of 2 x 32
-//               columns, and two accumulator buffers of 2 x 64 columns, so the epilogue of one
-//               item overlaps the MMAs of the next.
+//   warp 1      allocates all 512 tensor-memory columns; it and warps 15-21 issue tcgen05.mma
+//               (kind::f16, A from tensor memory, B from shared memory, fp32 accumulation): 4 A
+//               stages of 2 x 32 columns, and two accumulator buffers of 2 x 64 columns, so the
+//               epilogue of one item overlaps the MMAs of the next.  The MMAs of one thread run
+//               back to back at ~170 cycles each for any N up to 128 (measured on B200), while
+//               those of different warps overlap; so each tile's k steps are spread over up to
+//               four chains, each issued by its own warp into its own partial accumulator.
 //   warps 10-13 epilogue: read the accumulators (tcgen05.ld), apply int4 row scales, and write
 //               h = act(g) * u as fp16 (gate/up) or the fp32 per-pair outputs (down).
 //
@@ -48,17 +56,18 @@
 
 namespace bqg {
 
-constexpr int kTcThreads = 480;            // 15 warps
-constexpr int kTcWarpRaw = 0, kTcWarpMma = 1, kTcWarpDq = 2, kTcWarpEpi = 10, kTcWarpB = 14;
+constexpr int kTcThreads = 704;            // 22 warps
+constexpr int kTcWarpRaw = 0, kTcWarpMma = 1, kTcWarpDq = 2, kTcWarpEpi = 10, kTcWarpB = 14, kTcWarpMma2 = 15;
+constexpr int kTcMmaWarps = 8;             // MMA issuers: warp 1 and warps 15-21
 constexpr int kTcDqThreads = 256;          // 2 tiles x 128 rows
-constexpr int kTcNMax = 64;                // tokens per item (MMA N <= 64)
+constexpr int kTcNMax = 64;                // MMA N per item (tokens; two digit rows per token in kind::i8)
 constexpr int kTcAStages = 4;              // A stages in tensor memory
 constexpr int kTcBStages = 4;              // activation stages in shared memory
-constexpr int kTcBStageBytes = kTcNMax * 128;  // 64 rows x 64 k fp16
+constexpr int kTcBStageBytes = kTcNMax * 128;  // 64 rows x 128 bytes (64 k fp16, or 128 k int8)
 constexpr int kTcDescs = 8;                // item descriptor ring
 constexpr int kTcRawMax = 12;              // raw weight ring depth (runtime, by window size)
 constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (A stages use 0..255)
-constexpr int kTcDescReaders = 1 + 1 + 8 + 4;  // B producer, MMA, dequant warps, epilogue warps
+constexpr int kTcDescReaders = 1 + kTcMmaWarps + 8 + 4;  // B producer, MMA, dequant and epilogue warps
 // smem: [1 KB alignment slack][B ring][raw ring][barriers + descriptors]
 constexpr int kTcBarBytes = 1024;
 constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBStages) * kTcBStageBytes + kTcBarBytes;
@@ -75,7 +84,7 @@ struct TcFam {
   int g;                // rows per super-row of the tensor map
   int win;              // bytes fetched per row and raw chunk (a 16-byte-aligned window)
   int cb;               // bytes of one raw chunk of one row
-  int raw_k;            // weights per raw chunk (128, or 64 for Q8_0)
+  int raw_k;            // weights per raw chunk (int4 384, int2 768, Q4_0 256, Q8_0 128)
   int scale_off;        // int4: byte offset of the row scales in one matrix
   int m_off;            // row offset of this tile inside an item (0, or 128 for the second down tile)
 };
@@ -98,6 +107,12 @@ struct alignas(64) TcParams {
   int hperm[2];         // 1: the down matrix is a nibble format (store h in nibble order)
   float* yout[2];       // down: per-pair outputs [pairs][hidden], shared [tokens][hidden]
   int ystride;          // hidden
+  // kind::i8 variant (int4 / int2 weights): activation rows are pairs of int8 digit rows
+  // (X = 256 H + L, x ~= scale * X); per activation row its scale and the digit sum of X.
+  int nmax;             // tokens per item: kTcNMax (fp16) or kTcNMax / 2 (int8 digit rows)
+  const float* bscale[2];
+  const int32_t* bsum[2];
+  float* h32[2];        // gate/up of the kind::i8 variant: h rows in fp32 (natural order)
 };
 
 // ---------------------------------------------------------------- dequantization of one 64-k stage
@@ -130,35 +145,89 @@ __device__ __forceinline__ void tc_q8x4(uint32_t w, __half2 d2, uint32_t* o) {
   o[1] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p1), bias), d2));
 }
 
-// 64 weights of one row (two blocks, or 64 int4 values) at shared address a as 32 fp16 pairs.
+// 32 weights of one row as 16 fp16 pairs: the first (half 0) or second (half 1) block of a
+// 64-weight chunk at shared address a, or 32 of its 64 int4 values.
 // Q4_0 and Q8_0: a is 4-byte aligned (the row's blocks start there); int4: 16-byte aligned.
-__device__ __forceinline__ void tc_dequant64(int fmt, uint32_t a, uint32_t (&o)[32]) {
+__device__ __forceinline__ void tc_dequant32(int fmt, uint32_t a, int half, uint32_t (&o)[16]) {
   if (fmt == BQG_Q4_0) {  // block A: d at bytes 0-1, qs at 2..17; block B: d at 18-19, qs at 20..35
-    uint32_t v[9];
+    if (half == 0) {
+      uint32_t v[5];
 #pragma unroll
-    for (int i = 0; i < 9; ++i) v[i] = lds32(a + 4 * i);
-    const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
-    const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[4] >> 16)));
+      for (int i = 0; i < 5; ++i) v[i] = lds32(a + 4 * i);
+      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
 #pragma unroll
-    for (int m = 0; m < 4; ++m) tc_nib8(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[4 * m]);
+      for (int m = 0; m < 4; ++m) tc_nib8(__funnelshift_r(v[m], v[m + 1], 16), d, &o[4 * m]);
+    } else {
+      uint32_t v[5];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) tc_nib8(v[5 + m], dB, &o[16 + 4 * m]);
+      for (int i = 0; i < 5; ++i) v[i] = lds32(a + 16 + 4 * i);
+      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] >> 16)));
+#pragma unroll
+      for (int m = 0; m < 4; ++m) tc_nib8(v[1 + m], d, &o[4 * m]);
+    }
   } else if (fmt == BQG_Q8_0) {  // block A: d 0-1, q 2..33; block B: d 34-35, q 36..67
-    uint32_t v[17];
+    uint32_t v[9];
+    const uint32_t b = a + (half ? 32u : 0u);
 #pragma unroll
-    for (int i = 0; i < 17; ++i) v[i] = lds32(a + 4 * i);
-    const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
-    const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[8] >> 16)));
+    for (int i = 0; i < 9; ++i) v[i] = lds32(b + 4 * i);
+    if (half == 0) {
+      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
 #pragma unroll
-    for (int m = 0; m < 8; ++m) tc_q8x4(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[2 * m]);
+      for (int m = 0; m < 8; ++m) tc_q8x4(__funnelshift_r(v[m], v[m + 1], 16), d, &o[2 * m]);
+    } else {
+      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] >> 16)));
 #pragma unroll
-    for (int m = 0; m < 8; ++m) tc_q8x4(v[9 + m], dB, &o[16 + 2 * m]);
+      for (int m = 0; m < 8; ++m) tc_q8x4(v[1 + m], d, &o[2 * m]);
+    }
   } else {
+    const uint4 p = lds128(a + (half ? 16u : 0u));
+    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_i4nib8(w[m], &o[4 * m]);
+  }
+}
+
+// ---------------------------------------------------------------- kind::i8 operands (int4 / int2)
+// Weights as unsigned bytes t + 8 (int4) or t + 2 (int2): flipping the sign bit of each
+// two's-complement field adds the offset, and masks spread the fields over bytes.  The epilogue
+// removes the offset exactly: sum (t + z) X = sum t X + z sum X.
+// 64 weights at shared address a (16-byte aligned) as 16 words of 4 bytes: int4 word m yields
+// (elements 0,2,4,6) then (1,3,5,7) of its group of 8; int2 word m yields 4 words, byte j of word
+// k holding element 4j + k of its group of 16.
+__device__ __forceinline__ void tc_i8_dequant64(int fmt, uint32_t a, uint32_t (&o)[16]) {
+  if (fmt == BQG_I4_ROW) {  // 32 bytes
     const uint4 p0 = lds128(a), p1 = lds128(a + 16);
     const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-    for (int m = 0; m < 8; ++m) tc_i4nib8(w[m], &o[4 * m]);
+    for (int m = 0; m < 8; ++m) {
+      const uint32_t u = w[m] ^ 0x88888888u;
+      o[2 * m] = u & 0x0F0F0F0Fu;
+      o[2 * m + 1] = (u >> 4) & 0x0F0F0F0Fu;
+    }
+  } else {  // int2: 16 bytes
+    const uint4 p = lds128(a);
+    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t u = w[m] ^ 0xAAAAAAAAu;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[4 * m + k] = (u >> (2 * k)) & 0x03030303u;
+    }
   }
+}
+
+// Offset z of the unsigned weight bytes of a family (t + z).
+__host__ __device__ __forceinline__ int tc_i8_zero(int fmt) { return fmt == BQG_I2_ROW ? 2 : 8; }
+
+// Position of element k inside its int8 digit row: int4 groups of 8 in the order 0,2,4,6,1,3,5,7;
+// int2 groups of 16 with element 4j + k at position 4k + j.
+__host__ __device__ __forceinline__ int tc_i8_kpos(int k, int fmt) {
+  if (fmt == BQG_I2_ROW) {
+    const int i = k & 15;
+    return (k & ~15) | ((i & 3) << 2) | (i >> 2);
+  }
+  const int i = k & 7;
+  return (k & ~7) | ((i & 1) << 2) | (i >> 1);
 }
 
 // Position of element k inside its activation row: nibble formats hold each group of 8 in
@@ -169,10 +238,45 @@ __host__ __device__ __forceinline__ int tc_kpos(int k, int nibble) {
   return (k & ~7) | ((i & 3) << 1) | (i >> 2);
 }
 
+// Partial accumulators per tile for an item of N (padded) tokens: 4 x 16, 2 x 32 or 1 x N columns,
+// so that both tiles of an accumulator buffer fit its 128 columns.
+__host__ __device__ __forceinline__ int tc_partials(int N) { return N <= 16 ? 4 : N <= 32 ? 2 : 1; }
+
+// 8 accumulator columns of this warp's lanes at taddr, summed over the tile's `parts` partial
+// accumulators (stride columns apart) in a fixed order.  Warp-uniform arguments.
+__device__ __forceinline__ void tc_acc8(uint32_t taddr, int stride, int parts, float (&o)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  for (int p = 0; p < parts; ++p) {
+    uint32_t v[8];
+    tmem_ld8_nowait(taddr + uint32_t(p * stride), v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] += __uint_as_float(v[i]);
+  }
+}
+
+// The same for int32 accumulators (kind::i8): exact integer sums.
+__device__ __forceinline__ void tc_acc8i(uint32_t taddr, int stride, int parts, int (&o)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0;
+  for (int p = 0; p < parts; ++p) {
+    uint32_t v[8];
+    tmem_ld8_nowait(taddr + uint32_t(p * stride), v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] += int(v[i]);
+  }
+}
+
 // ---------------------------------------------------------------- the kernel
 // Item descriptor: d0 = (flags: bit0 shared, bit1 second tile present; expert; m0; tokens),
 //                  d1 = (first activation row; N; first output row; 64-k stages).
+// I8: kind::i8 variant (int4 / int2 weights as unsigned bytes in tensor memory, activations as
+// int8 digit rows, int32 accumulators); 128 k per stage instead of 64.
+template <bool I8>
 __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant__ TcParams P) {
+  constexpr int kStageK = I8 ? 128 : 64;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_s & 1023)) & 1023);
@@ -182,14 +286,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
   uint64_t* raw_full = bars;                        // [kTcRawMax] TMA bytes
   uint64_t* raw_empty = raw_full + kTcRawMax;       // [kTcRawMax] 256 dequant threads
   uint64_t* a_full = raw_empty + kTcRawMax;         // [kTcAStages] 256 dequant threads
-  uint64_t* a_empty = a_full + kTcAStages;          // [kTcAStages] MMA commit
+  uint64_t* a_empty = a_full + kTcAStages;          // [kTcAStages] MMA commits (one per issuer)
   uint64_t* b_full = a_empty + kTcAStages;          // [kTcBStages] TMA bytes
-  uint64_t* b_empty = b_full + kTcBStages;          // [kTcBStages] MMA commit
-  uint64_t* acc_full = b_empty + kTcBStages;        // [2] MMA commit
+  uint64_t* b_empty = b_full + kTcBStages;          // [kTcBStages] MMA commits
+  uint64_t* acc_full = b_empty + kTcBStages;        // [2] MMA commits
   uint64_t* acc_empty = acc_full + 2;               // [2] 128 epilogue threads
   uint64_t* d_full = acc_empty + 2;                 // [kTcDescs] producer
   uint64_t* d_empty = d_full + kTcDescs;            // [kTcDescs] reader warps
-  uint64_t* done = d_empty + kTcDescs;              // final MMA commit
+  uint64_t* done = d_empty + kTcDescs;              // final MMA commits
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int4* descs = reinterpret_cast<int4*>(bars + (kTcBarBytes - kTcDescs * 32) / 8);  // [kTcDescs][2]
@@ -202,21 +306,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
     }
     for (int i = 0; i < kTcAStages; ++i) {
       mbar_init(&a_full[i], kTcDqThreads);
-      mbar_init(&a_empty[i], 1);
+      mbar_init(&a_empty[i], kTcMmaWarps);
     }
     for (int i = 0; i < kTcBStages; ++i) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1);
+      mbar_init(&b_empty[i], kTcMmaWarps);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_full[i], kTcMmaWarps);
       mbar_init(&acc_empty[i], 128);
     }
     for (int i = 0; i < kTcDescs; ++i) {
       mbar_init(&d_full[i], 1);
       mbar_init(&d_empty[i], kTcDescReaders);
     }
-    mbar_init(done, 1);
+    mbar_init(done, kTcMmaWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -255,7 +359,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
     // ------------------------------------------------ item claims + raw weight TMA
     if (lane == 0) {
       const int na = *P.n_active;
-      const int nch = (P.tokens + kTcNMax - 1) / kTcNMax;
+      const int nmax = P.nmax;
+      const int nch = (P.tokens + nmax - 1) / nmax;
       const int n_sh = P.has_shared ? P.tiles_s * nch : 0;
       const int per_e = P.tiles_r * nch;
       const int n_items = n_sh + na * per_e;
@@ -287,7 +392,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             cnt = ai.y;
             off = ai.z;
           }
-          const int ntok = min(kTcNMax, cnt - c * kTcNMax);
+          const int ntok = min(nmax, cnt - c * nmax);
           if (ntok <= 0) {  // an empty token chunk of a lightly routed expert
             item = next;
             continue;
@@ -296,7 +401,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           const int m0 = t * tile_rows;
           const int two = (P.phase == 0 || m0 + 128 < P.fam[fb].rows) ? 1 : 0;
           d0 = make_int4(shared | (two << 1), e, m0, ntok);
-          d1 = make_int4(off + c * kTcNMax, (ntok + 15) & ~15, off + c * kTcNMax, P.fam[fb].cols / 64);
+          const int brow = I8 ? 2 * (off + c * nmax) : off + c * nmax;  // first B row
+          const int nb = I8 ? 2 * ntok : ntok;                                // B rows
+          d1 = make_int4(brow, (nb + 15) & ~15, off + c * nmax, P.fam[fb].cols / kStageK);
         } else {
           d0 = make_int4(-1, 0, 0, 0);
           d1 = make_int4(0, 0, 0, 0);
@@ -315,7 +422,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         const int fb = (d0.x & 1) ? 2 : 0;
         const int ntiles = 1 + ((d0.x >> 1) & 1);
         const TcFam& F0 = P.fam[fb];
-        const int nraw = (d1.w * 64 + F0.raw_k - 1) / F0.raw_k;
+        const int nraw = (d1.w * kStageK + F0.raw_k - 1) / F0.raw_k;
         for (int kc = 0; kc < nraw; ++kc, ++rp) {
           const int slot_r = rp % P.raw_stages;
           if (rp >= P.raw_stages && !mbar_wait(&raw_empty[slot_r], uint32_t(rp / P.raw_stages - 1) & 1u)) {
@@ -372,7 +479,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           mbar_arrive_expect_tx(&b_full[slot], uint32_t(N * 128));
           uint8_t* dst = bring + size_t(slot) * kTcBStageBytes;
           for (int nb = 0; nb < N / 16; ++nb)
-            tma_load_2d(dst + nb * 2048, &P.bmap[sh], s * 64, d1.x + 16 * nb, &b_full[slot]);
+            tma_load_2d(dst + nb * 2048, &P.bmap[sh], s * kStageK, d1.x + 16 * nb, &b_full[slot]);
         }
       }
       if (!ok) {
@@ -381,9 +488,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           mbar_wait(&b_full[q % kTcBStages], uint32_t(q / kTcBStages) & 1u);
       }
     }
-  } else if (warp == kTcWarpMma) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp == kTcWarpMma || warp >= kTcWarpMma2) {
+    // ------------------------------------------------ MMA issuers
+    // One thread's tcgen05.mma instructions run one after another, each taking ~170 cycles at
+    // N <= 128 whatever N is, while several issuing warps overlap theirs.  So the MMAs of a stage
+    // are spread over kTcMmaWarps issuers: issuer (tile f, partial p) owns the chain of k steps
+    // kk = p, p + P, ... of tile f into its own accumulator, P = 64 / N partial accumulators per
+    // tile (4 at N = 16, 2 at N = 32, else 1); the epilogue adds the P partials.
     if (lane == 0) {
+      const int mi = warp == kTcWarpMma ? 0 : warp - kTcWarpMma2 + 1;
+      const int f = mi & 1, p = mi >> 1;
       int as = 0, bs = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
@@ -391,14 +505,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         if (!read_desc(it, d0, d1)) break;
         if (d0.x < 0) break;
         const int two = (d0.x >> 1) & 1;
+        const int N = d1.y;
+        const int parts = tc_partials(N);
+        const bool on = p < parts && (f == 0 || two);
         const int buf = it & 1;
         if (it >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(it / 2 - 1) & 1u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = umma_idesc_f16(128, d1.y);
-        const uint32_t dcol = tmem + uint32_t(kTcAccCol + buf * 128);
+        const uint32_t idesc = I8 ? umma_idesc_i8(128, N) : umma_idesc_f16(128, N);
+        const uint32_t dcol = tmem + uint32_t(kTcAccCol + buf * 128 + f * 64 + p * N);
         for (int s = 0; s < d1.w; ++s, ++as, ++bs) {
           const int aslot = as % kTcAStages, bslot = bs % kTcBStages;
           if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u) ||
@@ -407,14 +524,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             break;
           }
           tc_fence_after();
-          const uint32_t acol = tmem + uint32_t(aslot * 64);
-          const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // 16 k per MMA: 8 tensor-memory columns, 32 bytes of B
-            const uint64_t bdesc = umma_desc_sw128(b_s + 32 * kk);
-            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-            umma_f16_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);
-            if (two) umma_f16_ts(dcol + 64, acol + 32 + 8 * kk, bdesc, idesc, acc);
+          if (on) {
+            const uint32_t acol = tmem + uint32_t(aslot * 64 + f * 32);
+            const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
+            for (int kk = p; kk < 4; kk += parts) {  // 8 tensor-memory columns, 32 bytes of B per MMA
+              const uint64_t bdesc = umma_desc_sw128(b_s + 32 * kk);
+              const uint32_t acc = (s > 0 || kk != p) ? 1u : 0u;
+              if constexpr (I8) umma_i8_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);  // 32 k
+              else umma_f16_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);               // 16 k
+            }
           }
           umma_commit(&a_empty[aslot]);
           umma_commit(&b_empty[bslot]);
@@ -423,10 +541,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         umma_commit(&acc_full[buf]);
       }
       if (!ok) *abort_flag = 1;
-      umma_commit(done);  // every MMA issued above has completed once this arrives
+      umma_commit(done);  // every MMA this thread issued has completed once all issuers' commits arrive
       mbar_wait(done, 0);
     }
-  } else if (warp < kTcWarpEpi) {
+  } else if (warp >= kTcWarpDq && warp < kTcWarpEpi) {
     // ------------------------------------------------ dequantize into tensor memory
     const int f = (warp - kTcWarpDq) >> 2;    // tile 0 (warps 2-5) or tile 1 (warps 6-9)
     const int qw = warp & 3;                  // tensor-memory lane quarter this warp may access
@@ -451,7 +569,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const bool row_on = tile_on && d0.z + F.m_off + r < F.rows;  // warp-uniform (rows % 32 == 0)
       const int g = F.g, j = r % g, q = r / g;
       const uint32_t row_off = uint32_t(f * 128 * F.win + j * (128 / g) * F.win + q * F.win);
-      const int spr = F0.raw_k / 64;  // MMA stages per raw chunk
+      const int spr = F0.raw_k / kStageK;  // MMA stages per raw chunk
       const int nraw = (d1.w + spr - 1) / spr;
       for (int kc = 0; kc < nraw && ok; ++kc, ++rp) {
         const int slot_r = rp % P.raw_stages;
@@ -469,11 +587,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           }
           tc_fence_after();
           if (row_on) {
-            uint32_t o[32];
-            tc_dequant64(F.fmt, rbase + uint32_t(h * (F.cb / spr)), o);
+            const uint32_t src = rbase + uint32_t(h * (F.cb / spr));
             const uint32_t taddr = tmem + tlane + uint32_t(aslot * 64 + f * 32);
-            tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(&o[0]));
-            tmem_st16(taddr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&o[16]));
+            uint32_t o[16];
+            if constexpr (I8) {
+              const uint32_t hb = F.fmt == BQG_I2_ROW ? 16u : 32u;  // bytes of 64 weights
+              tc_i8_dequant64(F.fmt, src, o);
+              tmem_st16(taddr, o);
+              tc_i8_dequant64(F.fmt, src + hb, o);
+              tmem_st16(taddr + 16, o);
+            } else {
+              tc_dequant32(F.fmt, src, 0, o);
+              tmem_st16(taddr, o);
+              tc_dequant32(F.fmt, src, 1, o);
+              tmem_st16(taddr + 16, o);
+            }
             tmem_wait_st();
           }
           tc_fence_before();
@@ -483,7 +611,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       }
     }
     if (!ok) *abort_flag = 1;
-  } else {
+  } else if (warp >= kTcWarpEpi && warp < kTcWarpB) {
     // ------------------------------------------------ epilogue
     const int qw = warp & 3;
     const int r = 32 * qw + lane;
@@ -501,6 +629,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const int sh = d0.x & 1, two = (d0.x >> 1) & 1;
       const int fb = sh ? 2 : 0;
       const int ntok = d0.w, N = d1.y, obase = d1.z;
+      const int parts = tc_partials(N);
       const int buf = it & 1;
       if (!mbar_wait(&acc_full[buf], uint32_t(it / 2) & 1u)) {
         ok = false;
@@ -508,7 +637,70 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       }
       tc_fence_after();
       const uint32_t acc = tmem + tlane + uint32_t(kTcAccCol + buf * 128);
-      if (P.phase == 0) {
+      if constexpr (I8) {
+        // columns 2n and 2n + 1: digit sums D_H, D_L of token n; x W^T = s (256 D_H + D_L - z SX)
+        const float* bsc = P.bscale[sh] + obase;
+        const int32_t* bsm = P.bsum[sh] + obase;
+        if (P.phase == 0) {
+          const TcFam& G = P.fam[fb];
+          const TcFam& U = P.fam[fb + 1];
+          const int row = d0.z + r;
+          const bool on = row < G.rows;
+          float sg = 0.f, su = 0.f;
+          if (on) {
+            sg = __ldg(reinterpret_cast<const float*>(G.base + (sh ? 0 : size_t(d0.y) * G.stride) + G.scale_off) + row);
+            su = __ldg(reinterpret_cast<const float*>(U.base + (sh ? 0 : size_t(d0.y) * U.stride) + U.scale_off) + row);
+          }
+          const long long z = tc_i8_zero(G.fmt);
+          float* hrow = P.h32[sh] + row;
+          const int hs = P.hstride[sh];
+          for (int c0 = 0; c0 < N; c0 += 8) {
+            int gv[8], uv[8];
+            tc_acc8i(acc + uint32_t(c0), N, parts, gv);
+            tc_acc8i(acc + uint32_t(64 + c0), N, parts, uv);
+            if (on) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int n = c0 / 2 + i;
+                if (n < ntok) {
+                  const float st = __ldg(bsc + n);
+                  const long long zx = z * __ldg(bsm + n);
+                  const float g = float(256LL * gv[2 * i] + gv[2 * i + 1] - zx) * st * sg;
+                  const float u = float(256LL * uv[2 * i] + uv[2 * i + 1] - zx) * st * su;
+                  hrow[size_t(obase + n) * hs] = act_fn(P.act, g) * u;
+                }
+              }
+            }
+          }
+        } else {
+          for (int f = 0; f <= two; ++f) {
+            const TcFam& D = P.fam[fb + f];
+            const int row = d0.z + D.m_off + r;
+            const bool on = row < D.rows;
+            float sd = 0.f;
+            if (on)
+              sd = __ldg(reinterpret_cast<const float*>(D.base + (sh ? 0 : size_t(d0.y) * D.stride) + D.scale_off) + row);
+            const long long z = tc_i8_zero(D.fmt);
+            for (int c0 = 0; c0 < N; c0 += 8) {
+              int v[8];
+              tc_acc8i(acc + uint32_t(f * 64 + c0), N, parts, v);
+              if (on) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int n = c0 / 2 + i;
+                  if (n < ntok) {
+                    const float st = __ldg(bsc + n);
+                    const long long zx = z * __ldg(bsm + n);
+                    const int orow = sh ? obase + n : __ldg(P.perm + obase + n);
+                    P.yout[sh][size_t(orow) * P.ystride + row] =
+                        float(256LL * v[2 * i] + v[2 * i + 1] - zx) * st * sd;
+                  }
+                }
+              }
+            }
+          }
+        }
+      } else if (P.phase == 0) {
         const TcFam& G = P.fam[fb];
         const TcFam& U = P.fam[fb + 1];
         const int row = d0.z + r;
@@ -520,17 +712,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         }
         __half* hrow = P.hout[sh] + tc_kpos(row, P.hperm[sh]);
         const int hs = P.hstride[sh];
-        for (int c0 = 0; c0 < N; c0 += 16) {
-          uint32_t gv[16], uv[16];
-          tmem_ld16_nowait(acc + uint32_t(c0), gv);
-          tmem_ld16_nowait(acc + uint32_t(64 + c0), uv);
-          tmem_wait_ld();
+        for (int c0 = 0; c0 < N; c0 += 8) {
+          float gv[8], uv[8];
+          tc_acc8(acc + uint32_t(c0), N, parts, gv);
+          tc_acc8(acc + uint32_t(64 + c0), N, parts, uv);
           if (on) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
               const int n = c0 + i;
               if (n < ntok) {
-                const float hv = act_fn(P.act, __uint_as_float(gv[i]) * sg) * (__uint_as_float(uv[i]) * su);
+                const float hv = act_fn(P.act, gv[i] * sg) * (uv[i] * su);
                 hrow[size_t(obase + n) * hs] = __float2half_rn(hv);
               }
             }
@@ -544,17 +735,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           float sd = 1.f;
           if (on && D.fmt == BQG_I4_ROW)
             sd = __ldg(reinterpret_cast<const float*>(D.base + (sh ? 0 : size_t(d0.y) * D.stride) + D.scale_off) + row);
-          for (int c0 = 0; c0 < N; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld16_nowait(acc + uint32_t(f * 64 + c0), v);
-            tmem_wait_ld();
+          for (int c0 = 0; c0 < N; c0 += 8) {
+            float v[8];
+            tc_acc8(acc + uint32_t(f * 64 + c0), N, parts, v);
             if (on) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
+              for (int i = 0; i < 8; ++i) {
                 const int n = c0 + i;
                 if (n < ntok) {
                   const int orow = sh ? obase + n : __ldg(P.perm + obase + n);
-                  P.yout[sh][size_t(orow) * P.ystride + row] = __uint_as_float(v[i]) * sd;
+                  P.yout[sh][size_t(orow) * P.ystride + row] = v[i] * sd;
                 }
               }
             }
@@ -620,16 +810,98 @@ __global__ void __launch_bounds__(256) k_moe_xprep(const float* __restrict__ x, 
   }
 }
 
+// ---------------------------------------------------------------- int8 digit rows (kind::i8 operand B)
+// One group of G values (G = 8 for int4, 16 for int2 weights): X = rint(v * inv), clamped to
+// |X| <= 32639, split into H = (X + 128) >> 8 and L = X - 256 H (both within [-128, 127]), placed at
+// the positions tc_i8_kpos gives.  Returns the sum of the group's X.
+template <int G>
+__device__ __forceinline__ int tc_digits_group(const float* __restrict__ v, float inv, int8_t* dh, int8_t* dl) {
+  float a[G];
+#pragma unroll
+  for (int q = 0; q < G / 4; ++q) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(v) + q);
+    a[4 * q] = t.x;
+    a[4 * q + 1] = t.y;
+    a[4 * q + 2] = t.z;
+    a[4 * q + 3] = t.w;
+  }
+  uint32_t wh[G / 4], wl[G / 4];
+#pragma unroll
+  for (int q = 0; q < G / 4; ++q) wh[q] = wl[q] = 0u;
+  int sx = 0;
+#pragma unroll
+  for (int e = 0; e < G; ++e) {
+    const int X = max(-32639, min(32639, __float2int_rn(a[e] * inv)));
+    const int H = (X + 128) >> 8;
+    const int L = X - 256 * H;
+    const int pos = tc_i8_kpos(e, G == 16 ? BQG_I2_ROW : BQG_I4_ROW);
+    wh[pos >> 2] |= uint32_t(H & 0xFF) << (8 * (pos & 3));
+    wl[pos >> 2] |= uint32_t(L & 0xFF) << (8 * (pos & 3));
+    sx += X;
+  }
+  if constexpr (G == 8) {
+    *reinterpret_cast<uint2*>(dh) = make_uint2(wh[0], wh[1]);
+    *reinterpret_cast<uint2*>(dl) = make_uint2(wl[0], wl[1]);
+  } else {
+    *reinterpret_cast<uint4*>(dh) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4*>(dl) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+  }
+  return sx;
+}
+
+// Activation rows of the kind::i8 variant, one warp per row: row i reads source row
+// gather[i] / gdiv (or i without gather) of `cols` fp32 values, takes s = max|v| / 32639 and
+// writes its digit rows 2i (H) and 2i + 1 (L) to dst [2 rows][cols] bytes, scale[i] = s and
+// sum[i] = sum of X, so that v ~= s X = s (256 H + L).  Rows: *rows_ptr if given, else rows.
+__global__ void __launch_bounds__(256) k_moe_digits(const float* __restrict__ src, const int32_t* __restrict__ gather,
+                                                  int gdiv, const int32_t* __restrict__ rows_ptr, int rows, int cols,
+                                                  int fmt, int8_t* __restrict__ dst, float* __restrict__ scale,
+                                                  int32_t* __restrict__ sum) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int n = rows_ptr != nullptr ? *rows_ptr : rows;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = int((gridDim.x * blockDim.x) >> 5);
+  for (int i = int((blockIdx.x * blockDim.x + threadIdx.x) >> 5); i < n; i += nwarps) {
+    const int sr = gather != nullptr ? __ldg(gather + i) / gdiv : i;
+    const float* v = src + size_t(sr) * cols;
+    float m = 0.f;
+    for (int k = 4 * lane; k < cols; k += 128) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(v + k));
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float inv = m > 0.f ? 32639.f / m : 0.f;
+    int8_t* dh = dst + size_t(2 * i) * cols;
+    int8_t* dl = dh + cols;
+    int sx = 0;
+    if (fmt == BQG_I2_ROW) {
+      for (int g0 = 16 * lane; g0 < cols; g0 += 512) sx += tc_digits_group<16>(v + g0, inv, dh + g0, dl + g0);
+    } else {
+      for (int g0 = 8 * lane; g0 < cols; g0 += 256) sx += tc_digits_group<8>(v + g0, inv, dh + g0, dl + g0);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    if (lane == 0) {
+      scale[i] = m / 32639.f;
+      sum[i] = sx;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- host side
 inline int tc_row_bytes(int fmt, int cols) {
-  return fmt == BQG_Q8_0 ? cols / 32 * 34 : fmt == BQG_Q4_0 ? cols / 32 * 18 : cols / 2;
+  return fmt == BQG_Q8_0 ? cols / 32 * 34 : fmt == BQG_Q4_0 ? cols / 32 * 18 : fmt == BQG_I2_ROW ? cols / 4 : cols / 2;
 }
 
 // Geometry of one family on the tensor-core path; false when the shape is not supported there
-// (k not a multiple of 64, or rows not a whole number of super-rows).
-inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols, int m_off, TcFam* out) {
-  if (fmt == BQG_I2_ROW) return false;  // the tensor-core path dequantizes Q8_0, Q4_0 and int4 only
-  if (cols % 64 != 0 || rows % 32 != 0) return false;
+// (k not a multiple of the stage, or rows not a whole number of super-rows).  i8: the kind::i8
+// variant (int4 and int2 only, k a multiple of 128); otherwise kind::f16 (Q8_0, Q4_0, int4).
+inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols, int m_off, TcFam* out,
+                   bool i8 = false) {
+  if (i8 ? (fmt != BQG_I4_ROW && fmt != BQG_I2_ROW) : fmt == BQG_I2_ROW) return false;
+  if (cols % (i8 ? 128 : 64) != 0 || rows % 32 != 0) return false;
   TcFam F{};
   F.base = static_cast<const uint8_t*>(base);
   F.stride = (long long)stride;
@@ -639,15 +911,15 @@ inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols,
   F.row_bytes = tc_row_bytes(fmt, cols);
   F.g = (F.row_bytes % 16 == 0) ? 1 : (F.row_bytes % 8 == 0) ? 2 : (F.row_bytes % 4 == 0) ? 4 : 0;
   if (F.g == 0 || rows % F.g != 0) return false;
-  if (fmt == BQG_I4_ROW) {
-    F.raw_k = 128;
-    F.cb = 64;
-    F.win = 64;  // rows are multiples of 32 bytes: every chunk starts 16-byte aligned
+  if (fmt == BQG_I4_ROW || fmt == BQG_I2_ROW) {
+    F.raw_k = fmt == BQG_I2_ROW ? 768 : 384;
+    F.cb = 192;
+    F.win = 208;  // rows are multiples of 32 (int4) or 16 (int2) bytes: chunks start 16-byte aligned
     F.scale_off = int((size_t(rows) * F.row_bytes + 15) / 16 * 16);
   } else {
-    F.raw_k = fmt == BQG_Q8_0 ? 64 : 128;
+    F.raw_k = fmt == BQG_Q8_0 ? 128 : 256;
     F.cb = F.raw_k / 32 * (fmt == BQG_Q8_0 ? 34 : 18);
-    F.win = 96;  // chunk (72 or 68 bytes) + up to 12 bytes of misalignment, rounded to 16
+    F.win = 176;  // chunk (144 or 136 bytes) + up to 12 bytes of misalignment, rounded to 16
   }
   F.m_off = m_off;
   *out = F;
@@ -688,6 +960,21 @@ inline int tc_encode_bmap(CUtensorMap* map, const __half* base, int rows, int co
   return BQG_OK;
 }
 
+// int8 digit rows [rows x cols] bytes (kind::i8 operand B), boxes of 128 k x 16 rows, 128-byte swizzle.
+inline int tc_encode_bmap_i8(CUtensorMap* map, const int8_t* base, int rows, int cols) {
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (encode == nullptr) return BQG_ERR_CUDA;
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows < 1 ? 1 : rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(cols)};
+  const cuuint32_t box[2] = {128, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return BQG_ERR_CUDA;
+  return BQG_OK;
+}
+
 inline size_t tc_smem_bytes(int raw_stages, int raw_stage_bytes) {
   return kTcFixedSmem + size_t(raw_stages) * raw_stage_bytes;
 }
@@ -699,6 +986,7 @@ inline void tc_raw_ring(int win, int* stages, int* stage_bytes) {
   *stages = n > kTcRawMax ? kTcRawMax : n;
 }
 
-inline SmemAttrOnce g_tc_attr;
+inline SmemAttrOnce g_tc_attr;     // k_moe_tc<false>
+inline SmemAttrOnce g_tc_attr_i8;  // k_moe_tc<true>
 
 }  // namespace bqg

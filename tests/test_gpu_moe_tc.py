@@ -5,12 +5,19 @@ The shapes cover every weight format as routed and as shared expert, rows whose 
 needs 1, 2 or 4 rows per tensor-map super-row, partial 128-row tiles, experts with more than 64
 tokens (several token chunks per item) and the full-size Gemma-like and GLM-like geometry.
 
+Two variants: kind::f16 (Q8_0, Q4_0 and int4 weights dequantized to fp16) and kind::i8 (layers
+whose every family is int4 or int2 with k a multiple of 128: weights as exact unsigned bytes,
+activations as 16-bit fixed-point digit pairs, int32 accumulation).
+
 Tolerance: the benchmark spec's bound 2e-3 * max|y_ref|, and a stricter bound derived from the
-arithmetic of this path.  Weights become fp16 with one rounding of (q - 8) * d or q * d
-(relative error <= 2^-11; int4 values are exact), x and h become fp16 (<= 2^-11 each), products
-accumulate in fp32.  The errors are independent per product, so a dot product's error is about
-2^-11 * sqrt(2) times the root-sum-square of its terms; through gate/up, the activation and
-down this stays near 4e-4 of max|y| (measured: see the per-test assertions), hence 1e-3.
+arithmetic of each variant.  kind::f16: weights become fp16 with one rounding of (q - 8) * d or
+q * d (relative error <= 2^-11; int4 values are exact), x and h become fp16 (<= 2^-11 each),
+products accumulate in fp32.  The errors are independent per product, so a dot product's error
+is about 2^-11 * sqrt(2) times the root-sum-square of its terms; through gate/up, the activation
+and down this stays near 4e-4 of max|y| (measured: see the per-test assertions), hence 1e-3.
+kind::i8: the sums over integers are exact; each x and h element carries a rounding error of at
+most max|row| / 65278 (16-bit fixed point per row), i.e. ~1.5e-5 of the row's largest element,
+and fp32 rounding of the scaled sums adds ~1e-7: well inside 2e-4 of max|y|.
 """
 import numpy as np
 import pytest
@@ -25,6 +32,15 @@ from tests.util import assert_close, max_rel_err, need_gpu
 pytestmark = pytest.mark.gpu
 
 TC_TOL = 1e-3
+I8_TOL = 2e-4
+
+
+def i8_variant(spec) -> bool:
+    """True when the tensor-core path takes the kind::i8 variant for this layer."""
+    fams = [(spec.expert_fmt, spec.hidden), (spec.expert_fmt, spec.inter)]
+    if spec.shared_inter:
+        fams += [(spec.shared_fmt, spec.shared_inter)]
+    return all(f in (bqg.I4_ROW, bqg.I2_ROW) and k % 128 == 0 for f, k in fams) and spec.hidden % 128 == 0
 
 TC_SPECS = [
     # hidden, inter, shared_inter multiples of 64; rows of 1584 / 216 / 72 bytes etc.
@@ -35,6 +51,14 @@ TC_SPECS = [
     wl.MoESpec("tc_q4_rows704", 5, 5, 320, 704, bqg.Q4_0, bqg.ACT_GELU_TANH, 0, 0, False),
     wl.MoESpec("tc_i4_shared_q8", 12, 4, 192, 128, bqg.I4_ROW, bqg.ACT_GELU_TANH, 128, bqg.Q8_0, False),
     wl.MoESpec("tc_q8_shared_q4", 4, 2, 128, 384, bqg.Q8_0, bqg.ACT_SILU, 448, bqg.Q4_0, False),
+    # kind::i8 layers: int2 routed; int4 with an int4 shared expert; int2 with an int4 shared expert;
+    # three 128-k stages and a down matrix of 384 rows (a 256-row item, then a one-tile item)
+    wl.MoESpec("tc8_i2_silu", 8, 2, 256, 128, bqg.I2_ROW, bqg.ACT_SILU, 0, 0, False),
+    wl.MoESpec("tc8_i4_shared_i4", 10, 3, 256, 256, bqg.I4_ROW, bqg.ACT_GELU_TANH, 128, bqg.I4_ROW, False),
+    wl.MoESpec("tc8_i2_shared_i4", 6, 2, 384, 128, bqg.I2_ROW, bqg.ACT_SILU, 256, bqg.I4_ROW, False),
+    wl.MoESpec("tc8_i4_rows384", 5, 2, 384, 384, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False),
+    # int4 with inter 192 (not a multiple of 128): the kind::f16 variant
+    wl.MoESpec("tc_i4_f16_inter192", 4, 2, 256, 192, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False),
 ]
 
 
@@ -62,7 +86,10 @@ def test_tc_small_matches_oracle(spec, tokens):
     torch.cuda.synchronize()
     ref = om.moe_layer(oracle_layer(spec, 0, 0), x.numpy(), ridx, rw)
     assert_close(y, ref, what=f"{spec.name} T={tokens}")
-    assert_close(y, ref, tol=TC_TOL, what=f"{spec.name} T={tokens} (fp16 operands)")
+    e = assert_close(y, ref, tol=TC_TOL, what=f"{spec.name} T={tokens} (fp16 operands)")
+    if i8_variant(spec):
+        assert_close(y, ref, tol=I8_TOL, what=f"{spec.name} T={tokens} (int8 digits)")
+    print(f"{spec.name} T={tokens}: max rel err {e:.2e}")
     assert bqg.bqg_device_errors() == 0
 
 
@@ -193,5 +220,6 @@ def test_glm_like_geometry_every_token_t64():
         y = bqg.moe_forward(lay.with_path(path), x.cuda(), idx, w)
         torch.cuda.synchronize()
         assert_close(y, ref, what=f"glm geometry T=64 path {path}")
-        tol = TC_TOL if path == bqg.MOE_PATH_TENSOR_CORES else 1e-4
-        assert_close(y, ref, tol=tol, what=f"glm geometry T=64 path {path} (strict)")
+        tol = I8_TOL if path == bqg.MOE_PATH_TENSOR_CORES else 1e-4
+        e = assert_close(y, ref, tol=tol, what=f"glm geometry T=64 path {path} (strict)")
+        print(f"glm geometry T=64 path {path}: max rel err {e:.2e}")
