@@ -17,7 +17,9 @@ is about 2^-11 * sqrt(2) times the root-sum-square of its terms; through gate/up
 and down this stays near 4e-4 of max|y| (measured: see the per-test assertions), hence 1e-3.
 kind::i8: the sums over integers are exact; each x and h element carries a rounding error of at
 most max|row| / 65278 (16-bit fixed point per row), i.e. ~1.5e-5 of the row's largest element,
-and fp32 rounding of the scaled sums adds ~1e-7: well inside 2e-4 of max|y|.
+and fp32 rounding of the scaled sums adds ~1e-7.  Relative to max|y| the row errors grow by the
+row's max / rms ratio, up to ~10 for the gated products h = act(g) * u, hence 3e-4 (measured up
+to 1.6e-4 over the specs below).
 """
 import numpy as np
 import pytest
@@ -32,7 +34,7 @@ from tests.util import assert_close, max_rel_err, need_gpu
 pytestmark = pytest.mark.gpu
 
 TC_TOL = 1e-3
-I8_TOL = 2e-4
+I8_TOL = 3e-4
 
 
 def i8_variant(spec) -> bool:
