@@ -56,23 +56,36 @@
 
 namespace bqg {
 
-constexpr int kTcThreads = 704;            // 22 warps
+#ifndef BQG_TC_MMA_WARPS
+#define BQG_TC_MMA_WARPS 2
+#endif
 constexpr int kTcWarpRaw = 0, kTcWarpMma = 1, kTcWarpDq = 2, kTcWarpEpi = 10, kTcWarpB = 14, kTcWarpMma2 = 15;
-constexpr int kTcMmaWarps = 8;             // MMA issuers: warp 1 and warps 15-21
+constexpr int kTcMmaWarps = BQG_TC_MMA_WARPS;  // MMA issuers: warp 1 and warps 15, 16, ...
+constexpr int kTcThreads = 32 * (14 + kTcMmaWarps);
 constexpr int kTcDqThreads = 256;          // 2 tiles x 128 rows
-constexpr int kTcNMax = 64;                // MMA N per item (tokens; two digit rows per token in kind::i8)
-constexpr int kTcAStages = 4;              // A stages in tensor memory
-constexpr int kTcBStages = 4;              // activation stages in shared memory
-constexpr int kTcBStageBytes = kTcNMax * 128;  // 64 rows x 128 bytes (64 k fp16, or 128 k int8)
+#ifndef BQG_TC_NMAX
+#define BQG_TC_NMAX 64
+#endif
+#ifndef BQG_TC_ASTAGES
+#define BQG_TC_ASTAGES 4
+#endif
+constexpr int kTcNMax = BQG_TC_NMAX;       // MMA N per item (tokens; two digit rows per token in kind::i8)
+constexpr int kTcAStages = BQG_TC_ASTAGES; // A stages in tensor memory (64 columns each: 2 tiles x 32)
+constexpr int kTcBStages = kTcAStages;     // activation stages in shared memory
+constexpr int kTcBStageBytes = kTcNMax * 128;  // N rows x 128 bytes (64 k fp16, or 128 k int8)
+constexpr int kTcAccTile = kTcNMax;        // accumulator columns per tile of one buffer
+constexpr int kTcAccBuf = 2 * kTcAccTile;  // columns per accumulator buffer (two tiles)
 constexpr int kTcDescs = 8;                // item descriptor ring
 constexpr int kTcRawMax = 12;              // raw weight ring depth (runtime, by window size)
-constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (A stages use 0..255)
+constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (after the A stages)
+static_assert(kTcAccCol + 2 * kTcAccBuf <= 512, "tensor memory: A stages + two accumulator buffers");
 constexpr int kTcDescReaders = 1 + kTcMmaWarps + 8 + 4;  // B producer, MMA, dequant and epilogue warps
 // smem: [1 KB alignment slack][B ring][raw ring][barriers + descriptors]
 constexpr int kTcBarBytes = 1024;
 constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBStages) * kTcBStageBytes + kTcBarBytes;
 constexpr size_t kTcMaxSmem = 227 * 1024;
-static_assert((2 * kTcRawMax + 4 * kTcAStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <= kTcBarBytes,
+static_assert((2 * kTcRawMax + 2 * kTcAStages + 2 * kTcBStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <=
+                  kTcBarBytes,
               "barrier area");
 
 // One family of stacked matrices as the kernel sees it (rows on M, cols = k).
@@ -240,7 +253,12 @@ __host__ __device__ __forceinline__ int tc_kpos(int k, int nibble) {
 
 // Partial accumulators per tile for an item of N (padded) tokens: 4 x 16, 2 x 32 or 1 x N columns,
 // so that both tiles of an accumulator buffer fit its 128 columns.
-__host__ __device__ __forceinline__ int tc_partials(int N) { return N <= 16 ? 4 : N <= 32 ? 2 : 1; }
+__host__ __device__ __forceinline__ int tc_partials(int N) {
+  const int cap = kTcMmaWarps >= 2 ? kTcMmaWarps / 2 : 1;  // issuers per tile
+  int p = 1;
+  while (p < 4 && p < cap && 2 * p * N <= kTcAccTile) p *= 2;
+  return p;
+}
 
 // 8 accumulator columns of this warp's lanes at taddr, summed over the tile's `parts` partial
 // accumulators (stride columns apart) in a fixed order.  Warp-uniform arguments.
@@ -269,6 +287,71 @@ __device__ __forceinline__ void tc_acc8i(uint32_t taddr, int stride, int parts, 
   }
 }
 
+// Raw chunk geometry per weight format: weights and bytes of one row per chunk, and the shared-
+// memory pitch of the rows (an odd multiple of 16 bytes; the chunk plus up to 12 bytes of
+// misalignment for the 18- and 34-byte block formats).
+__host__ __device__ constexpr int tc_raw_k(int fmt) {
+  return fmt == BQG_I2_ROW ? 768 : fmt == BQG_I4_ROW ? 384 : fmt == BQG_Q4_0 ? 256 : 128;
+}
+__host__ __device__ constexpr int tc_raw_cb(int fmt) {
+  return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? 192 : fmt == BQG_Q4_0 ? 144 : 136;
+}
+__host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? 208 : 176; }
+
+// One item's stages for this thread's row of a tile: wait for each raw chunk, dequantize every
+// 64- (kind::f16) or 128-k (kind::i8) stage of it into the A stage ring in tensor memory, and
+// hand the stages to the MMA issuers.  The format is a template argument, so the block layout
+// and every offset are constants.  Returns false when a bounded wait gave up.
+//   row_base  shared address of this row's window in raw stage 0;  mis0  j * row_bytes (the
+//   row's byte offset inside its super-row, for the 16-byte misalignment of each chunk)
+//   tcol      tensor-memory address of this lane, tile column offset included
+template <bool I8, int FMT>
+__device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_base, int mis0, int raw_stages,
+                                           int raw_stage_bytes, uint64_t* raw_full, uint64_t* raw_empty,
+                                           uint64_t* a_full, uint64_t* a_empty, uint32_t tcol, int& slot_r,
+                                           uint32_t& ph_r, int& as) {
+  constexpr int kStageK = I8 ? 128 : 64;
+  constexpr int kSpr = tc_raw_k(FMT) / kStageK;      // stages per raw chunk
+  constexpr int kCb = tc_raw_cb(FMT);
+  constexpr int kStageBytes = kCb / kSpr;
+  const int nraw = (nst + kSpr - 1) / kSpr;
+  for (int kc = 0; kc < nraw; ++kc) {
+    if (!mbar_wait(&raw_full[slot_r], ph_r)) return false;
+    const uint32_t base = row_base + uint32_t(slot_r * raw_stage_bytes) + (uint32_t(mis0 + kc * kCb) & 15u);
+    const int nh = min(kSpr, nst - kc * kSpr);
+    for (int h = 0; h < nh; ++h, ++as) {
+      const int aslot = as % kTcAStages;
+      if (as >= kTcAStages && !mbar_wait(&a_empty[aslot], uint32_t(as / kTcAStages - 1) & 1u)) return false;
+      tc_fence_after();
+      if (row_on) {
+        const uint32_t src = base + uint32_t(h * kStageBytes);
+        const uint32_t taddr = tcol + uint32_t(aslot * 64);
+        uint32_t o[16];
+        if constexpr (I8) {
+          tc_i8_dequant64(FMT, src, o);
+          tmem_st16(taddr, o);
+          tc_i8_dequant64(FMT, src + (FMT == BQG_I2_ROW ? 16u : 32u), o);
+          tmem_st16(taddr + 16, o);
+        } else {
+          tc_dequant32(FMT, src, 0, o);
+          tmem_st16(taddr, o);
+          tc_dequant32(FMT, src, 1, o);
+          tmem_st16(taddr + 16, o);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(&a_full[aslot]);
+    }
+    mbar_arrive(&raw_empty[slot_r]);
+    if (++slot_r == raw_stages) {
+      slot_r = 0;
+      ph_r ^= 1u;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- the kernel
 // Item descriptor: d0 = (flags: bit0 shared, bit1 second tile present; expert; m0; tokens),
 //                  d1 = (first activation row; N; first output row; 64-k stages).
@@ -280,7 +363,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_s & 1023)) & 1023);
-  uint8_t* bring = smem;                                            // kTcBStages x 8 KB
+  uint8_t* bring = smem;                                            // kTcBStages x N x 128 bytes
   uint8_t* wring = bring + size_t(kTcBStages) * kTcBStageBytes;    // raw_stages x raw_stage_bytes
   uint64_t* bars = reinterpret_cast<uint64_t*>(wring + size_t(P.raw_stages) * P.raw_stage_bytes);
   uint64_t* raw_full = bars;                        // [kTcRawMax] TMA bytes
@@ -497,7 +580,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
     // tile (4 at N = 16, 2 at N = 32, else 1); the epilogue adds the P partials.
     if (lane == 0) {
       const int mi = warp == kTcWarpMma ? 0 : warp - kTcWarpMma2 + 1;
-      const int f = mi & 1, p = mi >> 1;
+      constexpr int kTileStep = kTcMmaWarps >= 2 ? 2 : 1;  // one issuer per tile, or one for both
+      const int f0 = mi % kTileStep, p = mi / kTileStep;
       int as = 0, bs = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
@@ -507,7 +591,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         const int two = (d0.x >> 1) & 1;
         const int N = d1.y;
         const int parts = tc_partials(N);
-        const bool on = p < parts && (f == 0 || two);
         const int buf = it & 1;
         if (it >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(it / 2 - 1) & 1u)) {
           ok = false;
@@ -515,7 +598,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         }
         tc_fence_after();
         const uint32_t idesc = I8 ? umma_idesc_i8(128, N) : umma_idesc_f16(128, N);
-        const uint32_t dcol = tmem + uint32_t(kTcAccCol + buf * 128 + f * 64 + p * N);
+        const uint32_t dbase = tmem + uint32_t(kTcAccCol + buf * kTcAccBuf + p * N);
         for (int s = 0; s < d1.w; ++s, ++as, ++bs) {
           const int aslot = as % kTcAStages, bslot = bs % kTcBStages;
           if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u) ||
@@ -524,9 +607,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             break;
           }
           tc_fence_after();
-          if (on) {
+          const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
+          for (int f = f0; f < 1 + two && p < parts; f += kTileStep) {
             const uint32_t acol = tmem + uint32_t(aslot * 64 + f * 32);
-            const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
+            const uint32_t dcol = dbase + uint32_t(f * kTcAccTile);
             for (int kk = p; kk < 4; kk += parts) {  // 8 tensor-memory columns, 32 bytes of B per MMA
               const uint64_t bdesc = umma_desc_sw128(b_s + 32 * kk);
               const uint32_t acc = (s > 0 || kk != p) ? 1u : 0u;
@@ -551,7 +635,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
     const int r = 32 * qw + lane;             // row of the tile = tensor-memory lane
     const uint32_t tlane = uint32_t(32 * qw) << 16;
     const uint32_t wring_s = smem_u32(wring);
-    int rp = 0, as = 0;
+    const int raw_stages = P.raw_stages, raw_stage_bytes = P.raw_stage_bytes;
+    int slot_r = 0, as = 0;
+    uint32_t ph_r = 0;
     bool ok = true;
     for (int ds = 0; ok; ++ds) {
       int4 d0, d1;
@@ -565,49 +651,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const int fb = (d0.x & 1) ? 2 : 0;
       const bool tile_on = f == 0 || ((d0.x >> 1) & 1);
       const TcFam& F = P.fam[fb + f];
-      const TcFam& F0 = P.fam[fb];
       const bool row_on = tile_on && d0.z + F.m_off + r < F.rows;  // warp-uniform (rows % 32 == 0)
-      const int g = F.g, j = r % g, q = r / g;
-      const uint32_t row_off = uint32_t(f * 128 * F.win + j * (128 / g) * F.win + q * F.win);
-      const int spr = F0.raw_k / kStageK;  // MMA stages per raw chunk
-      const int nraw = (d1.w + spr - 1) / spr;
-      for (int kc = 0; kc < nraw && ok; ++kc, ++rp) {
-        const int slot_r = rp % P.raw_stages;
-        if (!mbar_wait(&raw_full[slot_r], uint32_t(rp / P.raw_stages) & 1u)) {
-          ok = false;
-          break;
-        }
-        const uint32_t mis = uint32_t(j * F.row_bytes + kc * F.cb) & 15u;
-        const uint32_t rbase = wring_s + uint32_t(slot_r) * P.raw_stage_bytes + row_off + mis;
-        for (int h = 0; h < spr && kc * spr + h < d1.w; ++h, ++as) {
-          const int aslot = as % kTcAStages;
-          if (as >= kTcAStages && !mbar_wait(&a_empty[aslot], uint32_t(as / kTcAStages - 1) & 1u)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (row_on) {
-            const uint32_t src = rbase + uint32_t(h * (F.cb / spr));
-            const uint32_t taddr = tmem + tlane + uint32_t(aslot * 64 + f * 32);
-            uint32_t o[16];
-            if constexpr (I8) {
-              const uint32_t hb = F.fmt == BQG_I2_ROW ? 16u : 32u;  // bytes of 64 weights
-              tc_i8_dequant64(F.fmt, src, o);
-              tmem_st16(taddr, o);
-              tc_i8_dequant64(F.fmt, src + hb, o);
-              tmem_st16(taddr + 16, o);
-            } else {
-              tc_dequant32(F.fmt, src, 0, o);
-              tmem_st16(taddr, o);
-              tc_dequant32(F.fmt, src, 1, o);
-              tmem_st16(taddr + 16, o);
-            }
-            tmem_wait_st();
-          }
-          tc_fence_before();
-          mbar_arrive(&a_full[aslot]);
-        }
-        mbar_arrive(&raw_empty[slot_r]);
+      const int fmt = F.fmt, win = F.win, g = F.g, j = r % g, q = r / g;
+      const uint32_t row_base = wring_s + uint32_t(f * 128 * win + j * (128 / g) * win + q * win);
+      const int mis0 = j * F.row_bytes;
+      const uint32_t tcol = tmem + tlane + uint32_t(f * 32);
+      const int nst = d1.w;
+      if constexpr (I8) {
+        ok = fmt == BQG_I2_ROW
+                 ? tc_dq_item<true, BQG_I2_ROW>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
+                                                raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as)
+                 : tc_dq_item<true, BQG_I4_ROW>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
+                                                raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as);
+      } else {
+        ok = fmt == BQG_Q4_0
+                 ? tc_dq_item<false, BQG_Q4_0>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
+                                               raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as)
+             : fmt == BQG_Q8_0
+                 ? tc_dq_item<false, BQG_Q8_0>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
+                                               raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as)
+                 : tc_dq_item<false, BQG_I4_ROW>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
+                                                 raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as);
       }
     }
     if (!ok) *abort_flag = 1;
@@ -636,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         break;
       }
       tc_fence_after();
-      const uint32_t acc = tmem + tlane + uint32_t(kTcAccCol + buf * 128);
+      const uint32_t acc = tmem + tlane + uint32_t(kTcAccCol + buf * kTcAccBuf);
       if constexpr (I8) {
         // columns 2n and 2n + 1: digit sums D_H, D_L of token n; x W^T = s (256 D_H + D_L - z SX)
         const float* bsc = P.bscale[sh] + obase;
@@ -657,7 +721,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           for (int c0 = 0; c0 < N; c0 += 8) {
             int gv[8], uv[8];
             tc_acc8i(acc + uint32_t(c0), N, parts, gv);
-            tc_acc8i(acc + uint32_t(64 + c0), N, parts, uv);
+            tc_acc8i(acc + uint32_t(kTcAccTile + c0), N, parts, uv);
             if (on) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
@@ -683,7 +747,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             const long long z = tc_i8_zero(D.fmt);
             for (int c0 = 0; c0 < N; c0 += 8) {
               int v[8];
-              tc_acc8i(acc + uint32_t(f * 64 + c0), N, parts, v);
+              tc_acc8i(acc + uint32_t(f * kTcAccTile + c0), N, parts, v);
               if (on) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -715,7 +779,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         for (int c0 = 0; c0 < N; c0 += 8) {
           float gv[8], uv[8];
           tc_acc8(acc + uint32_t(c0), N, parts, gv);
-          tc_acc8(acc + uint32_t(64 + c0), N, parts, uv);
+          tc_acc8(acc + uint32_t(kTcAccTile + c0), N, parts, uv);
           if (on) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -737,7 +801,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             sd = __ldg(reinterpret_cast<const float*>(D.base + (sh ? 0 : size_t(d0.y) * D.stride) + D.scale_off) + row);
           for (int c0 = 0; c0 < N; c0 += 8) {
             float v[8];
-            tc_acc8(acc + uint32_t(f * 64 + c0), N, parts, v);
+            tc_acc8(acc + uint32_t(f * kTcAccTile + c0), N, parts, v);
             if (on) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
@@ -912,14 +976,14 @@ inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols,
   F.g = (F.row_bytes % 16 == 0) ? 1 : (F.row_bytes % 8 == 0) ? 2 : (F.row_bytes % 4 == 0) ? 4 : 0;
   if (F.g == 0 || rows % F.g != 0) return false;
   if (fmt == BQG_I4_ROW || fmt == BQG_I2_ROW) {
-    F.raw_k = fmt == BQG_I2_ROW ? 768 : 384;
-    F.cb = 192;
-    F.win = 208;  // rows are multiples of 32 (int4) or 16 (int2) bytes: chunks start 16-byte aligned
+    F.raw_k = tc_raw_k(fmt);
+    F.cb = tc_raw_cb(fmt);
+    F.win = tc_raw_win(fmt);  // rows are multiples of 32 (int4) or 16 (int2) bytes: chunks start 16-byte aligned
     F.scale_off = int((size_t(rows) * F.row_bytes + 15) / 16 * 16);
   } else {
-    F.raw_k = fmt == BQG_Q8_0 ? 128 : 256;
-    F.cb = F.raw_k / 32 * (fmt == BQG_Q8_0 ? 34 : 18);
-    F.win = 176;  // chunk (144 or 136 bytes) + up to 12 bytes of misalignment, rounded to 16
+    F.raw_k = tc_raw_k(fmt);
+    F.cb = tc_raw_cb(fmt);
+    F.win = tc_raw_win(fmt);  // chunk (144 or 136 bytes) + up to 12 bytes of misalignment
   }
   F.m_off = m_off;
   *out = F;
