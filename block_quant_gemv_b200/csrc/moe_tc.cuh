@@ -57,7 +57,7 @@
 namespace bqg {
 
 #ifndef BQG_TC_MMA_WARPS
-#define BQG_TC_MMA_WARPS 2
+#define BQG_TC_MMA_WARPS 8
 #endif
 constexpr int kTcWarpRaw = 0, kTcWarpMma = 1, kTcWarpDq = 2, kTcWarpEpi = 10, kTcWarpB = 14, kTcWarpMma2 = 15;
 constexpr int kTcMmaWarps = BQG_TC_MMA_WARPS;  // MMA issuers: warp 1 and warps 15, 16, ...
@@ -84,7 +84,8 @@ constexpr int kTcDescReaders = 1 + kTcMmaWarps + 8 + 4;  // B producer, MMA, deq
 constexpr int kTcBarBytes = 1024;
 constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBStages) * kTcBStageBytes + kTcBarBytes;
 constexpr size_t kTcMaxSmem = 227 * 1024;
-static_assert((2 * kTcRawMax + 2 * kTcAStages + 2 * kTcBStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <=
+static_assert(kTcBStages == kTcAStages, "activation stage i shares the A stage's barriers");
+static_assert((2 * kTcRawMax + 2 * kTcAStages + kTcBStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <=
                   kTcBarBytes,
               "barrier area");
 
@@ -305,11 +306,13 @@ __host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW
 //   row_base  shared address of this row's window in raw stage 0;  mis0  j * row_bytes (the
 //   row's byte offset inside its super-row, for the 16-byte misalignment of each chunk)
 //   tcol      tensor-memory address of this lane, tile column offset included
+//   wait_b    this thread also waits for the stage's activation rows (b_full) before it arrives,
+//             so that a_full completes only once both operands of the stage are in place
 template <bool I8, int FMT>
 __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_base, int mis0, int raw_stages,
                                            int raw_stage_bytes, uint64_t* raw_full, uint64_t* raw_empty,
-                                           uint64_t* a_full, uint64_t* a_empty, uint32_t tcol, int& slot_r,
-                                           uint32_t& ph_r, int& as) {
+                                           uint64_t* a_full, uint64_t* a_empty, uint64_t* b_full, bool wait_b,
+                                           uint32_t tcol, int& slot_r, uint32_t& ph_r, int& as) {
   constexpr int kStageK = I8 ? 128 : 64;
   constexpr int kSpr = tc_raw_k(FMT) / kStageK;      // stages per raw chunk
   constexpr int kCb = tc_raw_cb(FMT);
@@ -341,6 +344,7 @@ __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_ba
         tmem_wait_st();
       }
       tc_fence_before();
+      if (wait_b && !mbar_wait(&b_full[aslot], uint32_t(as / kTcAStages) & 1u)) return false;
       mbar_arrive(&a_full[aslot]);
     }
     mbar_arrive(&raw_empty[slot_r]);
@@ -370,9 +374,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
   uint64_t* raw_empty = raw_full + kTcRawMax;       // [kTcRawMax] 256 dequant threads
   uint64_t* a_full = raw_empty + kTcRawMax;         // [kTcAStages] 256 dequant threads
   uint64_t* a_empty = a_full + kTcAStages;          // [kTcAStages] MMA commits (one per issuer)
-  uint64_t* b_full = a_empty + kTcAStages;          // [kTcBStages] TMA bytes
-  uint64_t* b_empty = b_full + kTcBStages;          // [kTcBStages] MMA commits
-  uint64_t* acc_full = b_empty + kTcBStages;        // [2] MMA commits
+  uint64_t* b_full = a_empty + kTcAStages;          // [kTcBStages] TMA bytes (B slot i is freed by a_empty[i])
+  uint64_t* acc_full = b_full + kTcBStages;         // [2] MMA commits
   uint64_t* acc_empty = acc_full + 2;               // [2] 128 epilogue threads
   uint64_t* d_full = acc_empty + 2;                 // [kTcDescs] producer
   uint64_t* d_empty = d_full + kTcDescs;            // [kTcDescs] reader warps
@@ -393,7 +396,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
     }
     for (int i = 0; i < kTcBStages; ++i) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], kTcMmaWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], kTcMmaWarps);
@@ -551,7 +553,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         const int N = d1.y;
         for (int s = 0; s < d1.w; ++s, ++bs) {
           const int slot = bs % kTcBStages;
-          if (bs >= kTcBStages && !mbar_wait(&b_empty[slot], uint32_t(bs / kTcBStages - 1) & 1u)) {
+          if (bs >= kTcBStages && !mbar_wait(&a_empty[slot], uint32_t(bs / kTcBStages - 1) & 1u)) {
             ok = false;
             break;
           }
@@ -582,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const int mi = warp == kTcWarpMma ? 0 : warp - kTcWarpMma2 + 1;
       constexpr int kTileStep = kTcMmaWarps >= 2 ? 2 : 1;  // one issuer per tile, or one for both
       const int f0 = mi % kTileStep, p = mi / kTileStep;
-      int as = 0, bs = 0;
+      int as = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
         int4 d0, d1;
@@ -599,15 +601,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         tc_fence_after();
         const uint32_t idesc = I8 ? umma_idesc_i8(128, N) : umma_idesc_f16(128, N);
         const uint32_t dbase = tmem + uint32_t(kTcAccCol + buf * kTcAccBuf + p * N);
-        for (int s = 0; s < d1.w; ++s, ++as, ++bs) {
-          const int aslot = as % kTcAStages, bslot = bs % kTcBStages;
-          if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u) ||
-              !mbar_wait(&b_full[bslot], uint32_t(bs / kTcBStages) & 1u)) {
+        for (int s = 0; s < d1.w; ++s, ++as) {
+          const int aslot = as % kTcAStages;  // B uses the same slot
+          if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u)) {  // A and B of the stage
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t b_s = smem_u32(bring + size_t(bslot) * kTcBStageBytes);
+          const uint32_t b_s = smem_u32(bring + size_t(aslot) * kTcBStageBytes);
           for (int f = f0; f < 1 + two && p < parts; f += kTileStep) {
             const uint32_t acol = tmem + uint32_t(aslot * 64 + f * 32);
             const uint32_t dcol = dbase + uint32_t(f * kTcAccTile);
@@ -618,8 +619,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
               else umma_f16_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);               // 16 k
             }
           }
-          umma_commit(&a_empty[aslot]);
-          umma_commit(&b_empty[bslot]);
+          umma_commit(&a_empty[aslot]);  // frees the A and the B stage
         }
         if (!ok) break;
         umma_commit(&acc_full[buf]);
@@ -657,21 +657,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const int mis0 = j * F.row_bytes;
       const uint32_t tcol = tmem + tlane + uint32_t(f * 32);
       const int nst = d1.w;
+      const bool wait_b = warp == kTcWarpDq && lane == 0;
       if constexpr (I8) {
         ok = fmt == BQG_I2_ROW
                  ? tc_dq_item<true, BQG_I2_ROW>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
-                                                raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as)
+                                                raw_empty, a_full, a_empty, b_full, wait_b, tcol, slot_r, ph_r, as)
                  : tc_dq_item<true, BQG_I4_ROW>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
-                                                raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as);
+                                                raw_empty, a_full, a_empty, b_full, wait_b, tcol, slot_r, ph_r, as);
       } else {
         ok = fmt == BQG_Q4_0
                  ? tc_dq_item<false, BQG_Q4_0>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
-                                               raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as)
+                                               raw_empty, a_full, a_empty, b_full, wait_b, tcol, slot_r, ph_r, as)
              : fmt == BQG_Q8_0
                  ? tc_dq_item<false, BQG_Q8_0>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
-                                               raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as)
+                                               raw_empty, a_full, a_empty, b_full, wait_b, tcol, slot_r, ph_r, as)
                  : tc_dq_item<false, BQG_I4_ROW>(nst, row_on, row_base, mis0, raw_stages, raw_stage_bytes, raw_full,
-                                                 raw_empty, a_full, a_empty, tcol, slot_r, ph_r, as);
+                                                 raw_empty, a_full, a_empty, b_full, wait_b, tcol, slot_r, ph_r, as);
       }
     }
     if (!ok) *abort_flag = 1;
