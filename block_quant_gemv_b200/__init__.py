@@ -30,7 +30,7 @@ __all__ = [
 Q8_0, Q4_0, I4_ROW, I2_ROW = 1, 2, 3, 4
 ACT_GELU_TANH, ACT_SILU = 1, 2
 MOE_PATH_AUTO, MOE_PATH_CUDA_CORES, MOE_PATH_TENSOR_CORES = 0, 1, 2
-MOE_TC_MIN_TOKENS, MOE_TC_MIN_PER_EXPERT = 16, 4
+MOE_TC_MIN_TOKENS = 8
 MAX_COLS, MAX_BATCH, MAX_EXPERTS, MAX_TOPK, MAX_MOE_COLS = 15360, 256, 256, 8, 7168
 DEVERR_TIMEOUT, DEVERR_EXPERT_ID = 0x1, 0x2
 

@@ -192,17 +192,13 @@ inline MoeTcLayout moe_ws_layout_tc(const bqg_moe_layer* L, int tokens) {
   return o;
 }
 
-// The automatic choice.  A tensor-core MMA instruction (M = 128 weight rows, K = 16) costs about
-// the same whatever the number of tokens on its N side, so that path pays per weight read,
-// while the CUDA-core path pays per (weight, token).  Measured crossovers on B200: with a
-// shared expert (its N is every token) from 16 tokens on; without one, once the routed experts
-// average 4 tokens each (GLM-like layer: T = 64 takes 2.06 ms on CUDA cores against 2.49 ms,
-// T = 128 3.96 ms against 2.88 ms).
-inline bool moe_tc_preferred(const bqg_moe_layer* L, int tokens) {
-  if (L->s_gate != nullptr && tokens >= BQG_MOE_TC_MIN_TOKENS) return true;
-  return (long long)tokens * L->top_k >= (long long)BQG_MOE_TC_MIN_PER_EXPERT * L->n_experts &&
-         tokens >= BQG_MOE_TC_MIN_TOKENS;
-}
+// The automatic choice.  A tensor-core MMA instruction (M = 128 weight rows) costs the same
+// whatever the number of tokens on its N side, so that path pays per weight read, while the
+// CUDA-core path pays per (weight, token).  Measured on B200 (us per layer, CUDA cores / tensor
+// cores): Gemma-like layer T = 4: 80 / 102, T = 8: 137 / 104; GLM-like layer T = 4: 157 / 167,
+// T = 8: 290 / 245, T = 64: 2058 / 887.  So the tensor cores from 8 tokens on, even when the
+// routed experts average well under one token each.
+inline bool moe_tc_preferred(const bqg_moe_layer*, int tokens) { return tokens >= BQG_MOE_TC_MIN_TOKENS; }
 
 // Path for `tokens` tokens: BQG_MOE_PATH_CUDA_CORES or BQG_MOE_PATH_TENSOR_CORES (negative: error).
 inline int moe_path(const bqg_moe_layer* L, int tokens) {

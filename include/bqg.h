@@ -76,20 +76,21 @@ enum bqg_act { BQG_ACT_GELU_TANH = 1, BQG_ACT_SILU = 2 };
 
 /* How moe_forward runs the experts (bqg_moe_layer.path).  Both compute the same layer.
  *   BQG_MOE_PATH_AUTO          the tensor cores (when the shapes allow it) from
- *                              BQG_MOE_TC_MIN_TOKENS tokens on if the layer has a shared expert,
- *                              else once tokens * top_k >= BQG_MOE_TC_MIN_PER_EXPERT * n_experts
- *                              (and tokens >= BQG_MOE_TC_MIN_TOKENS); the CUDA cores otherwise.
+ *                              BQG_MOE_TC_MIN_TOKENS tokens on; the CUDA cores otherwise.
  *   BQG_MOE_PATH_CUDA_CORES    grouped GEMV with integer dot products: every expert item is applied
- *                              to its tokens one at a time (best for 1..8 tokens).
+ *                              to its tokens one at a time (best for 1..7 tokens).
  *   BQG_MOE_PATH_TENSOR_CORES  grouped expert GEMM on tcgen05: weights dequantized once into tensor
  *                              memory and multiplied by all the expert's tokens at once (prefill
- *                              chunks, large decode batches).  Needs hidden, inter and shared_inter
- *                              multiples of 64, and activations (x and the gated hidden values)
- *                              within the fp16 range; returns BQG_ERR_SHAPE when the shapes do not
- *                              allow it. */
+ *                              chunks, decode batches).  Two variants:
+ *                              - kind::i8 when every family (routed, and shared if present) is
+ *                                BQG_I4_ROW or BQG_I2_ROW with hidden, inter and shared_inter
+ *                                multiples of 128: weights as exact bytes, x and the gated hidden
+ *                                values as 16-bit fixed point per row (two int8 digits), int32 sums;
+ *                              - kind::f16 otherwise (Q8_0, Q4_0, int4; no int2): hidden, inter and
+ *                                shared_inter multiples of 64, activations within the fp16 range.
+ *                              Returns BQG_ERR_SHAPE when neither variant takes the layer. */
 enum bqg_moe_path { BQG_MOE_PATH_AUTO = 0, BQG_MOE_PATH_CUDA_CORES = 1, BQG_MOE_PATH_TENSOR_CORES = 2 };
-#define BQG_MOE_TC_MIN_TOKENS 16
-#define BQG_MOE_TC_MIN_PER_EXPERT 4
+#define BQG_MOE_TC_MIN_TOKENS 8
 
 #define BQG_MAX_COLS 15360       /* largest cols (K) of the GEMV, router and prefill calls  */
 #define BQG_MAX_BATCH 256        /* largest descriptor count of one qgemv_batched call     */

@@ -39,13 +39,20 @@ def oracle_router_logits(spec: wl.MoESpec, seed: int, layer: int, x: np.ndarray)
     return om.router_logits(R, x)
 
 
-def expected_path(spec: wl.MoESpec, tokens: int) -> int:
-    """The path the library's automatic choice takes for this layer (mirrors include/bqg.h):
-    tensor cores from 16 tokens on with a shared expert, else once the routed experts average 4
-    tokens each; only shapes that are multiples of 64 can take them."""
+def tc_shapes_ok(spec: wl.MoESpec) -> bool:
+    """Whether a tensor-core variant takes the layer (mirrors include/bqg.h): kind::i8 for int4 /
+    int2 families with every dimension a multiple of 128, kind::f16 for layers without int2 with
+    every dimension a multiple of 64."""
     dims = [spec.hidden, spec.inter] + ([spec.shared_inter] if spec.shared_inter else [])
-    if any(d % 64 for d in dims) or tokens < bqg.MOE_TC_MIN_TOKENS:
-        return bqg.MOE_PATH_CUDA_CORES
-    if spec.shared_inter or tokens * spec.top_k >= bqg.MOE_TC_MIN_PER_EXPERT * spec.n_experts:
+    fmts = [spec.expert_fmt] + ([spec.shared_fmt] if spec.shared_inter else [])
+    if all(f in (bqg.I4_ROW, bqg.I2_ROW) for f in fmts) and not any(d % 128 for d in dims):
+        return True
+    return bqg.I2_ROW not in fmts and not any(d % 64 for d in dims)
+
+
+def expected_path(spec: wl.MoESpec, tokens: int) -> int:
+    """The path the library's automatic choice takes for this layer: the tensor cores from
+    MOE_TC_MIN_TOKENS tokens on when a variant takes the shapes, else the CUDA cores."""
+    if tokens >= bqg.MOE_TC_MIN_TOKENS and tc_shapes_ok(spec):
         return bqg.MOE_PATH_TENSOR_CORES
     return bqg.MOE_PATH_CUDA_CORES
