@@ -159,77 +159,10 @@ __device__ __forceinline__ void tc_q8x4(uint32_t w, __half2 d2, uint32_t* o) {
   o[1] = h2_bits(__hmul2(__hsub2(*reinterpret_cast<__half2*>(&p1), bias), d2));
 }
 
-// 32 weights of one row as 16 fp16 pairs: the first (half 0) or second (half 1) block of a
-// 64-weight chunk at shared address a, or 32 of its 64 int4 values.
-// Q4_0 and Q8_0: a is 4-byte aligned (the row's blocks start there); int4: 16-byte aligned.
-__device__ __forceinline__ void tc_dequant32(int fmt, uint32_t a, int half, uint32_t (&o)[16]) {
-  if (fmt == BQG_Q4_0) {  // block A: d at bytes 0-1, qs at 2..17; block B: d at 18-19, qs at 20..35
-    if (half == 0) {
-      uint32_t v[5];
-#pragma unroll
-      for (int i = 0; i < 5; ++i) v[i] = lds32(a + 4 * i);
-      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
-#pragma unroll
-      for (int m = 0; m < 4; ++m) tc_nib8(__funnelshift_r(v[m], v[m + 1], 16), d, &o[4 * m]);
-    } else {
-      uint32_t v[5];
-#pragma unroll
-      for (int i = 0; i < 5; ++i) v[i] = lds32(a + 16 + 4 * i);
-      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] >> 16)));
-#pragma unroll
-      for (int m = 0; m < 4; ++m) tc_nib8(v[1 + m], d, &o[4 * m]);
-    }
-  } else if (fmt == BQG_Q8_0) {  // block A: d 0-1, q 2..33; block B: d 34-35, q 36..67
-    uint32_t v[9];
-    const uint32_t b = a + (half ? 32u : 0u);
-#pragma unroll
-    for (int i = 0; i < 9; ++i) v[i] = lds32(b + 4 * i);
-    if (half == 0) {
-      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
-#pragma unroll
-      for (int m = 0; m < 8; ++m) tc_q8x4(__funnelshift_r(v[m], v[m + 1], 16), d, &o[2 * m]);
-    } else {
-      const __half2 d = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] >> 16)));
-#pragma unroll
-      for (int m = 0; m < 8; ++m) tc_q8x4(v[1 + m], d, &o[2 * m]);
-    }
-  } else {
-    const uint4 p = lds128(a + (half ? 16u : 0u));
-    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-    for (int m = 0; m < 4; ++m) tc_i4nib8(w[m], &o[4 * m]);
-  }
-}
-
 // ---------------------------------------------------------------- kind::i8 operands (int4 / int2)
 // Weights as unsigned bytes t + 8 (int4) or t + 2 (int2): flipping the sign bit of each
 // two's-complement field adds the offset, and masks spread the fields over bytes.  The epilogue
 // removes the offset exactly: sum (t + z) X = sum t X + z sum X.
-// 64 weights at shared address a (16-byte aligned) as 16 words of 4 bytes: int4 word m yields
-// (elements 0,2,4,6) then (1,3,5,7) of its group of 8; int2 word m yields 4 words, byte j of word
-// k holding element 4j + k of its group of 16.
-__device__ __forceinline__ void tc_i8_dequant64(int fmt, uint32_t a, uint32_t (&o)[16]) {
-  if (fmt == BQG_I4_ROW) {  // 32 bytes
-    const uint4 p0 = lds128(a), p1 = lds128(a + 16);
-    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const uint32_t u = w[m] ^ 0x88888888u;
-      o[2 * m] = u & 0x0F0F0F0Fu;
-      o[2 * m + 1] = (u >> 4) & 0x0F0F0F0Fu;
-    }
-  } else {  // int2: 16 bytes
-    const uint4 p = lds128(a);
-    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const uint32_t u = w[m] ^ 0xAAAAAAAAu;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) o[4 * m + k] = (u >> (2 * k)) & 0x03030303u;
-    }
-  }
-}
-
 // Offset z of the unsigned weight bytes of a family (t + z).
 __host__ __device__ __forceinline__ int tc_i8_zero(int fmt) { return fmt == BQG_I2_ROW ? 2 : 8; }
 
@@ -299,6 +232,87 @@ __host__ __device__ constexpr int tc_raw_cb(int fmt) {
 }
 __host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? 208 : 176; }
 
+// One stage of one row, loaded first and converted after: all its shared-memory words are read
+// before the first tensor-memory store, so the loads of the second half do not wait behind it.
+// Q4_0: 36 bytes (two blocks), Q8_0: 68 bytes, int4 (kind::f16, 64 k): 32 bytes.
+template <int FMT>
+__device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
+  uint32_t o[16];
+  if constexpr (FMT == BQG_Q4_0) {  // block A: d at bytes 0-1, qs 2..17; block B: d at 18-19, qs 20..35
+    uint32_t v[9];
+#pragma unroll
+    for (int i = 0; i < 9; ++i) v[i] = lds32(src + 4 * i);
+    const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
+    const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[4] >> 16)));
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_nib8(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[4 * m]);
+    tmem_st16(taddr, o);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_nib8(v[5 + m], dB, &o[4 * m]);
+    tmem_st16(taddr + 16, o);
+  } else if constexpr (FMT == BQG_Q8_0) {  // block A: d 0-1, q 2..33; block B: d 34-35, q 36..67
+    uint32_t v[17];
+#pragma unroll
+    for (int i = 0; i < 17; ++i) v[i] = lds32(src + 4 * i);
+    const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
+    const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[8] >> 16)));
+#pragma unroll
+    for (int m = 0; m < 8; ++m) tc_q8x4(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[2 * m]);
+    tmem_st16(taddr, o);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) tc_q8x4(v[9 + m], dB, &o[2 * m]);
+    tmem_st16(taddr + 16, o);
+  } else {  // int4: 16-byte aligned
+    const uint4 p0 = lds128(src), p1 = lds128(src + 16);
+    const uint32_t w0[4] = {p0.x, p0.y, p0.z, p0.w}, w1[4] = {p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_i4nib8(w0[m], &o[4 * m]);
+    tmem_st16(taddr, o);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tc_i4nib8(w1[m], &o[4 * m]);
+    tmem_st16(taddr + 16, o);
+  }
+}
+
+// kind::i8: int4 64 bytes (128 k), int2 32 bytes; 16-byte aligned.  Each int4 word yields two
+// words of bytes t + 8: elements 0,2,4,6 then 1,3,5,7 of its group of 8; each int2 word yields four
+// words of bytes t + 2, byte j of word k holding element 4j + k of its group of 16.
+__device__ __forceinline__ void tc_i4_bytes(uint4 a, uint4 b, uint32_t (&o)[16]) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const uint32_t u = w[m] ^ 0x88888888u;
+    o[2 * m] = u & 0x0F0F0F0Fu;
+    o[2 * m + 1] = (u >> 4) & 0x0F0F0F0Fu;
+  }
+}
+__device__ __forceinline__ void tc_i2_bytes(uint4 a, uint32_t (&o)[16]) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint32_t u = w[m] ^ 0xAAAAAAAAu;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[4 * m + k] = (u >> (2 * k)) & 0x03030303u;
+  }
+}
+template <int FMT>
+__device__ __forceinline__ void tc_i8_stage(uint32_t src, uint32_t taddr) {
+  uint32_t o[16];
+  if constexpr (FMT == BQG_I4_ROW) {
+    const uint4 p0 = lds128(src), p1 = lds128(src + 16), p2 = lds128(src + 32), p3 = lds128(src + 48);
+    tc_i4_bytes(p0, p1, o);
+    tmem_st16(taddr, o);
+    tc_i4_bytes(p2, p3, o);
+    tmem_st16(taddr + 16, o);
+  } else {
+    const uint4 p0 = lds128(src), p1 = lds128(src + 16);
+    tc_i2_bytes(p0, o);
+    tmem_st16(taddr, o);
+    tc_i2_bytes(p1, o);
+    tmem_st16(taddr + 16, o);
+  }
+}
+
 // One item's stages for this thread's row of a tile: wait for each raw chunk, dequantize every
 // 64- (kind::f16) or 128-k (kind::i8) stage of it into the A stage ring in tensor memory, and
 // hand the stages to the MMA issuers.  The format is a template argument, so the block layout
@@ -329,18 +343,8 @@ __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_ba
       if (row_on) {
         const uint32_t src = base + uint32_t(h * kStageBytes);
         const uint32_t taddr = tcol + uint32_t(aslot * 64);
-        uint32_t o[16];
-        if constexpr (I8) {
-          tc_i8_dequant64(FMT, src, o);
-          tmem_st16(taddr, o);
-          tc_i8_dequant64(FMT, src + (FMT == BQG_I2_ROW ? 16u : 32u), o);
-          tmem_st16(taddr + 16, o);
-        } else {
-          tc_dequant32(FMT, src, 0, o);
-          tmem_st16(taddr, o);
-          tc_dequant32(FMT, src, 1, o);
-          tmem_st16(taddr + 16, o);
-        }
+        if constexpr (I8) tc_i8_stage<FMT>(src, taddr);
+        else tc_f16_stage<FMT>(src, taddr);
         tmem_wait_st();
       }
       tc_fence_before();
