@@ -320,8 +320,9 @@ BQG_API int bqg_expert_cache_get_stats(const bqg_expert_cache* cache, bqg_expert
  * frees nothing.  Arguments are those of moe_forward without the workspace.
  *   - Returns BQG_ERR_LIMIT when moe_workspace_size(L, tokens) exceeds BQG_NOALLOC_SCRATCH_BYTES.
  *     32 MiB covers the Gemma-4-26B-A4B-like layer (hidden 2816, 128 experts, shared expert) up
- *     to 128 tokens (21.4 MB) and the GLM-like layer (hidden 6144, 256 int4 experts of 2048) up to
- *     64 tokens (21.0 MB); a GLM-like 128-token chunk (42 MB) does not fit.
+ *     to 128 tokens (21.5 MB; 25.2 MB on the CUDA cores) and the GLM-like layer (hidden 6144, 256
+ *     int4 experts of 2048) up to 64 tokens (25.2 MB); a GLM-like 128-token chunk (50 MB) does not
+ *     fit.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  *     that device current, and again after the device's context was destroyed and re-created
  *     (cudaDeviceReset); make that first call before any stream capture that includes it.
