@@ -18,8 +18,8 @@
 //               elements views each family as [expert][super-row][bytes], a super-row being g = 1,
 //               2 or 4 consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of
 //               704 values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
-//               The copy engine's time grows with the number of row segments a box holds, so each
-//               chunk takes a long piece of every row (64-byte pieces measured ~7 cycles each).
+//               Each chunk takes a long piece of every row, so that one producer/consumer round
+//               through the raw ring covers three or four MMA stages.
 //               Rows land in shared memory an odd multiple of 16 bytes apart (176 or 208), so the
 //               dequantizing threads' 16-byte loads of consecutive rows hit distinct bank groups
 //               (a 64- or 256-byte pitch put 4 or 8 rows on the same banks).
@@ -75,10 +75,15 @@ constexpr int kTcBStages = kTcAStages;     // activation stages in shared memory
 constexpr int kTcBStageBytes = kTcNMax * 128;  // N rows x 128 bytes (64 k fp16, or 128 k int8)
 constexpr int kTcAccTile = kTcNMax;        // accumulator columns per tile of one buffer
 constexpr int kTcAccBuf = 2 * kTcAccTile;  // columns per accumulator buffer (two tiles)
+#ifndef BQG_TC_ACC_BUFS
+#define BQG_TC_ACC_BUFS 2
+#endif
+constexpr int kTcAccBufs = BQG_TC_ACC_BUFS;  // accumulator buffers (2: an item's epilogue overlaps the next one's MMAs)
 constexpr int kTcDescs = 8;                // item descriptor ring
 constexpr int kTcRawMax = 12;              // raw weight ring depth (runtime, by window size)
 constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (after the A stages)
-static_assert(kTcAccCol + 2 * kTcAccBuf <= 512, "tensor memory: A stages + two accumulator buffers");
+static_assert(kTcAccBufs >= 1 && kTcAccBufs <= 2, "one or two accumulator buffers");
+static_assert(kTcAccCol + kTcAccBufs * kTcAccBuf <= 512, "tensor memory: A stages + accumulator buffers");
 constexpr int kTcDescReaders = 1 + kTcMmaWarps + 8 + 4;  // B producer, MMA, dequant and epilogue warps
 // smem: [1 KB alignment slack][B ring][raw ring][barriers + descriptors]
 constexpr int kTcBarBytes = 1024;
@@ -597,8 +602,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         const int two = (d0.x >> 1) & 1;
         const int N = d1.y;
         const int parts = tc_partials(N);
-        const int buf = it & 1;
-        if (it >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(it / 2 - 1) & 1u)) {
+        const int buf = it % kTcAccBufs;
+        if (it >= kTcAccBufs && !mbar_wait(&acc_empty[buf], uint32_t(it / kTcAccBufs - 1) & 1u)) {
           ok = false;
           break;
         }
@@ -699,8 +704,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const int fb = sh ? 2 : 0;
       const int ntok = d0.w, N = d1.y, obase = d1.z;
       const int parts = tc_partials(N);
-      const int buf = it & 1;
-      if (!mbar_wait(&acc_full[buf], uint32_t(it / 2) & 1u)) {
+      const int buf = it % kTcAccBufs;
+      if (!mbar_wait(&acc_full[buf], uint32_t(it / kTcAccBufs) & 1u)) {
         ok = false;
         break;
       }
