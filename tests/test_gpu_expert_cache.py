@@ -156,3 +156,29 @@ def test_glm_like_geometry_sixteen_slots():
         assert cache.stats() == sim.stats
     st = cache.stats()
     assert st["hits"] >= 8 and st["bytes_copied"] == st["misses"] * sim.nb
+
+
+@pytest.mark.parametrize("spec,tol", [
+    (SMALL, 1e-3),  # Q4_0 experts, Q8_0 shared expert: the kind::f16 tensor-core variant
+    (wl.MoESpec("ec_i4", 16, 4, 256, 128, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False), 3e-4),  # kind::i8
+], ids=["q4_shared_f16", "i4_i8"])
+def test_many_tokens_take_the_tensor_cores(spec, tol):
+    """Calls of 12 tokens take the tensor-core path in both passes (hits, then the misses after
+    the copies, accumulated into the same output): every call against the oracle and the policy."""
+    need_gpu()
+    assert 12 >= bqg.MOE_TC_MIN_TOKENS
+    cache, sim = _cache(spec, n_slots=spec.n_experts)
+    ref_layer = oracle_layer(spec, 0, 0)
+    for call, seed in enumerate([21, 21, 22, 23]):  # misses, all hits, then mixes
+        x = wl.moe_tokens(spec, seed, 12)
+        idx_h, w = _route(spec, seed, 12)
+        y = cache.forward(x.cuda(), idx_h, w)
+        torch.cuda.synchronize()
+        sim.step(idx_h.numpy(), spec.n_experts)
+        ref = om.moe_layer(ref_layer, x.numpy(), idx_h.numpy(), w.cpu().numpy())
+        assert_close(y, ref, what=f"{spec.name} call {call}")
+        assert_close(y, ref, tol=tol, what=f"{spec.name} call {call} (tensor cores)")
+        assert cache.stats() == sim.stats
+    st = cache.stats()
+    assert st["hits"] > 0 and st["misses"] > 0
+    assert bqg.bqg_device_errors() == 0
