@@ -19,6 +19,11 @@
 //              and store Y.
 // With several k-splits per tile (small n), the CTAs of one tile form a thread-block cluster
 // and the partial tiles are summed through distributed shared memory in a fixed order.
+// BQG_PF_ISSUERS (1, 2, 4: MMA-issuing warps, each with its own partial accumulator over a
+// share of the k steps) and BQG_PF_DQ_WARPS (4, 8: a thread per row, or per row and block) are
+// build-time choices; 1 and 4 measured best (2/4 issuers and 8 dequant warps: 32.6-35.2 us
+// against 32.9 us at n = 14336).  Launched as a dependent launch: the next kernel's prologue
+// overlaps this one's tail.
 #pragma once
 
 #include <cuda.h>
@@ -29,7 +34,19 @@
 
 namespace bqg {
 
-constexpr int kPfThreads = 192;           // 6 warps
+#ifndef BQG_PF_ISSUERS
+#define BQG_PF_ISSUERS 1
+#endif
+#ifndef BQG_PF_DQ_WARPS
+#define BQG_PF_DQ_WARPS 4
+#endif
+constexpr int kPfIssuers = BQG_PF_ISSUERS;   // MMA-issuing warps = partial accumulators (k steps split)
+constexpr int kPfDqWarps = BQG_PF_DQ_WARPS;  // 4: a thread per weight row; 8: a thread per row and block
+static_assert(kPfIssuers == 1 || kPfIssuers == 2 || kPfIssuers == 4, "1, 2 or 4 issuers");
+static_assert(kPfDqWarps == 4 || kPfDqWarps == 8, "4 or 8 dequant warps");
+constexpr int kPfDqThreads = 32 * kPfDqWarps;
+constexpr int kPfWarpIss2 = 2 + kPfDqWarps;  // first extra issuer warp
+constexpr int kPfThreads = 32 * (2 + kPfDqWarps + kPfIssuers - 1);
 constexpr int kPfTileN = 128;             // output features per CTA
 constexpr int kPfTileM = 128;             // tokens per CTA (MMA M)
 constexpr int kPfStageK = 64;             // k per stage (one 128-byte swizzle row of fp16)
@@ -54,6 +71,21 @@ struct PfParams {
   int ksplit;        // CTAs (cluster size) sharing one output tile
   int kchunks;       // k / kPfRawK; split s owns chunks [s*kchunks/ksplit, (s+1)*kchunks/ksplit)
 };
+
+// 16 accumulator columns of this warp's lanes, the kPfIssuers partials (kPfTileN columns apart)
+// added in a fixed order.
+__device__ __forceinline__ void pf_acc16(uint32_t taddr, float (&o)[16]) {
+  uint32_t v[16];
+  tmem_ld16(taddr, v);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(v[i]);
+#pragma unroll
+  for (int p = 1; p < kPfIssuers; ++p) {
+    tmem_ld16(taddr + uint32_t(p * kPfTileN), v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] += __uint_as_float(v[i]);
+  }
+}
 
 // ---------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -88,27 +120,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPfStages; ++i) {
       mbar_init(&a_full[i], 1);
-      mbar_init(&b_full[i], 128);
-      mbar_init(&st_empty[i], 1);
+      mbar_init(&b_full[i], kPfDqThreads);
+      mbar_init(&st_empty[i], kPfIssuers);
     }
     for (int i = 0; i < kPfRawStages; ++i) {
       mbar_init(&w_full[i], 1);
-      mbar_init(&w_empty[i], 128);
+      mbar_init(&w_empty[i], kPfDqThreads);
     }
-    mbar_init(done, 1);
+    mbar_init(done, kPfIssuers);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
     // 128 fp32 columns of tensor memory for the 128 x 128 accumulator
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kPfTileN));
+                 "r"(kPfIssuers * kPfTileN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Dependent launch: the next kernel on the stream may start its prologue now; every global
+  // read and write of this one waits for the previous kernel (X may be its output, Y its input).
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -142,10 +178,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mbar_wait(&w_full[q % kPfRawStages], uint32_t(q / kPfRawStages) & 1u);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp >= kPfWarpIss2) {
+    // ------------------------------------------------ MMA issuers: issuer p takes k steps p, p + I, ...
     if (lane == 0) {
+      const int p = warp == 1 ? 0 : warp - kPfWarpIss2 + 1;
       const uint32_t idesc = umma_idesc_f16(kPfTileM, kPfTileN);
+      const uint32_t acc = tmem + uint32_t(p * kPfTileN);
       for (int s = 0; s < nst; ++s) {
         const int st = s % kPfStages;
         const uint32_t par = uint32_t(s / kPfStages) & 1u;
@@ -157,16 +195,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t a_s = smem_u32(a_ring + size_t(st) * kPfABytes);
         const uint32_t b_s = smem_u32(b_ring + size_t(st) * kPfBBytes);
 #pragma unroll
-        for (int kk = 0; kk < kPfStageK / 16; ++kk)  // 16 fp16 = 32 bytes per MMA along k
-          umma_f16(tmem, umma_desc_sw128(a_s + 32 * kk), umma_desc_sw128(b_s + 32 * kk), idesc,
-                   (s > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = p; kk < kPfStageK / 16; kk += kPfIssuers)  // 16 fp16 = 32 bytes per MMA along k
+          umma_f16(acc, umma_desc_sw128(a_s + 32 * kk), umma_desc_sw128(b_s + 32 * kk), idesc,
+                   (s > 0 || kk != p) ? 1u : 0u);
         umma_commit(&st_empty[st]);  // frees the stage once these MMAs have read it
       }
       umma_commit(done);  // all MMAs issued by this thread have completed
     }
   } else {
     // ------------------------------------------------ dequantize W into the B stages
-    const int t = threadIdx.x - 64;  // 0..127: weight row n0 + t of the tile
+    const int tt = threadIdx.x - 64;     // 0 .. kPfDqThreads - 1
+    const int t = tt & 127;              // weight row n0 + t of the tile
+    const int half = kPfDqWarps == 8 ? (tt >> 7) : -1;  // 8 warps: block A (0) or B (1) of the stage
     const uint32_t b_row_base = uint32_t(t >> 3) * 1024 + uint32_t(t & 7) * 128;
     const int sw = t & 7;            // swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
     int s = 0;
@@ -185,23 +225,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           break;
         }
         // two Q4_0 blocks (36 bytes) of this row: block A at bytes 0..17, block B at 18..35
-        uint32_t v[9];
-#pragma unroll
-        for (int i = 0; i < 9; ++i) v[i] = lds32(raw_row + 36 * q + 4 * i);
-        const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
-        const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[4] >> 16)));
         const uint32_t b_s = smem_u32(b_ring + size_t(st) * kPfBBytes) + b_row_base;
+        if (half <= 0) {
+          uint32_t v[5];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {  // block A: k = 8m .. 8m+7
-          uint32_t o[4];
-          q4_word_to_f16(__funnelshift_r(v[m], v[m + 1], 16), dA, o);
-          sts128(b_s + uint32_t((m ^ sw) * 16), o[0], o[1], o[2], o[3]);
+          for (int i = 0; i < 5; ++i) v[i] = lds32(raw_row + 36 * q + 4 * i);
+          const __half2 dA = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] & 0xFFFFu)));
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {  // block A: k = 8m .. 8m+7
+            uint32_t o[4];
+            q4_word_to_f16(__funnelshift_r(v[m], v[m + 1], 16), dA, o);
+            sts128(b_s + uint32_t((m ^ sw) * 16), o[0], o[1], o[2], o[3]);
+          }
         }
+        if (half != 0) {
+          uint32_t v[5];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {  // block B: k = 32 + 8m .. 32 + 8m + 7
-          uint32_t o[4];
-          q4_word_to_f16(v[5 + m], dB, o);
-          sts128(b_s + uint32_t(((4 + m) ^ sw) * 16), o[0], o[1], o[2], o[3]);
+          for (int i = 0; i < 5; ++i) v[i] = lds32(raw_row + 36 * q + 16 + 4 * i);
+          const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[0] >> 16)));
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {  // block B: k = 32 + 8m .. 32 + 8m + 7
+            uint32_t o[4];
+            q4_word_to_f16(v[1 + m], dB, o);
+            sts128(b_s + uint32_t(((4 + m) ^ sw) * 16), o[0], o[1], o[2], o[3]);
+          }
         }
         fence_proxy_async_smem();  // make the fp16 tile visible to the tensor core
         mbar_arrive(&b_full[st]);
@@ -216,7 +263,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // k-split cluster every CTA parks its partial tile in its (now idle) A ring; rank r then sums
   // its slice of the columns over all ranks, in rank order, through distributed shared memory.
   // Every thread of every CTA takes part in the two cluster barriers.
-  const bool epi_warp = warp >= 2;
+  const bool epi_warp = warp >= 2 && warp < 6;  // the first four dequant warps: one per lane quarter
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;  // token
   bool have = false;
@@ -232,14 +279,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (epi_warp) {
 #pragma unroll 1
       for (int c = 0; c < kPfTileN; c += 16) {
-        uint32_t r16[16];
-        if (have) tmem_ld16(tm_row + uint32_t(c), r16);
+        float r16[16];
+        if (have) pf_acc16(tm_row + uint32_t(c), r16);
 #pragma unroll
         for (int i = 0; i < 16; i += 4)
           *reinterpret_cast<float4*>(&park[row * kPitch + c + i]) =
-              have ? make_float4(__uint_as_float(r16[i]), __uint_as_float(r16[i + 1]), __uint_as_float(r16[i + 2]),
-                                 __uint_as_float(r16[i + 3]))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+              have ? make_float4(r16[i], r16[i + 1], r16[i + 2], r16[i + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     __syncwarp();
@@ -279,22 +324,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int ncols = row < prm.tokens ? min(kPfTileN, prm.n - n0) : 0;
 #pragma unroll 1
     for (int c = 0; c < kPfTileN; c += 16) {
-      uint32_t r16[16];
-      tmem_ld16(tm_row + uint32_t(c), r16);
+      float r16[16];
+      pf_acc16(tm_row + uint32_t(c), r16);
       if (c < ncols) {
         uint4 pk;
-        pk.x = h2_bits(__floats2half2_rn(__uint_as_float(r16[0]), __uint_as_float(r16[1])));
-        pk.y = h2_bits(__floats2half2_rn(__uint_as_float(r16[2]), __uint_as_float(r16[3])));
-        pk.z = h2_bits(__floats2half2_rn(__uint_as_float(r16[4]), __uint_as_float(r16[5])));
-        pk.w = h2_bits(__floats2half2_rn(__uint_as_float(r16[6]), __uint_as_float(r16[7])));
+        pk.x = h2_bits(__floats2half2_rn(r16[0], r16[1]));
+        pk.y = h2_bits(__floats2half2_rn(r16[2], r16[3]));
+        pk.z = h2_bits(__floats2half2_rn(r16[4], r16[5]));
+        pk.w = h2_bits(__floats2half2_rn(r16[6], r16[7]));
         *reinterpret_cast<uint4*>(y + c) = pk;
       }
       if (c + 8 < ncols) {
         uint4 pk;
-        pk.x = h2_bits(__floats2half2_rn(__uint_as_float(r16[8]), __uint_as_float(r16[9])));
-        pk.y = h2_bits(__floats2half2_rn(__uint_as_float(r16[10]), __uint_as_float(r16[11])));
-        pk.z = h2_bits(__floats2half2_rn(__uint_as_float(r16[12]), __uint_as_float(r16[13])));
-        pk.w = h2_bits(__floats2half2_rn(__uint_as_float(r16[14]), __uint_as_float(r16[15])));
+        pk.x = h2_bits(__floats2half2_rn(r16[8], r16[9]));
+        pk.y = h2_bits(__floats2half2_rn(r16[10], r16[11]));
+        pk.z = h2_bits(__floats2half2_rn(r16[12], r16[13]));
+        pk.w = h2_bits(__floats2half2_rn(r16[14], r16[15]));
         *reinterpret_cast<uint4*>(y + c + 8) = pk;
       }
     }
@@ -303,7 +348,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPfTileN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPfIssuers * kPfTileN));
   }
 }
 
@@ -371,13 +416,15 @@ extern "C" int qgemm_prefill(int fmt, const void* W, const void* X, void* Y, int
   cfg.blockDim = dim3(kPfThreads, 1, 1);
   cfg.dynamicSmemBytes = kPfSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = unsigned(ksplit);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, k_prefill_q4, tx, tw, prm) != cudaSuccess) {
     (void)cudaGetLastError();  // not left behind for a later call's status check
     return BQG_ERR_CUDA;
