@@ -61,6 +61,30 @@ def test_moe_widest_rows():
     assert bqg.lib().moe_workspace_size(c, 1) == 0  # rejected: BQG_ERR_LIMIT on the call
 
 
+@pytest.mark.parametrize("fmt,shared_fmt,shared_inter,tol", [
+    (bqg.Q4_0, bqg.Q8_0, 192, 1e-3),  # kind::f16 variant
+    (bqg.I4_ROW, 0, 0, 3e-4),         # kind::i8 variant: int32 sums over k = 7168
+    (bqg.I2_ROW, bqg.I4_ROW, 128, 3e-4),
+], ids=["f16_q4_shared_q8", "i8_i4", "i8_i2_shared_i4"])
+def test_moe_widest_rows_tensor_cores(fmt, shared_fmt, shared_inter, tol):
+    """hidden = BQG_MAX_MOE_COLS (7168) on the tensor-core path (20 tokens, every token compared)."""
+    need_gpu()
+    spec = wl.MoESpec("lim_wide_tc", 4, 2, bqg.MAX_MOE_COLS, 256, fmt, bqg.ACT_SILU, shared_inter, shared_fmt, False)
+    L = wl.build_moe_layer(spec, 6, 0, device="cuda")
+    tokens = 20
+    assert tokens >= bqg.MOE_TC_MIN_TOKENS
+    x = wl.moe_tokens(spec, 6, tokens)
+    lg = wl.moe_logits(spec, 6, 0, tokens)
+    idx, w = bqg.moe_router_topk(lg.cuda(), spec.top_k)
+    y = bqg.moe_forward(device_layer(L).with_path(bqg.MOE_PATH_TENSOR_CORES), x.cuda(), idx, w)
+    torch.cuda.synchronize()
+    ridx, rw = om.router_topk(lg.numpy(), spec.top_k)
+    ref = om.moe_layer(oracle_layer(spec, 6, 0), x.numpy(), ridx, rw)
+    assert_close(y, ref, what=f"hidden {spec.hidden} tensor cores")
+    assert_close(y, ref, tol=tol, what=f"hidden {spec.hidden} tensor cores (strict)")
+    assert bqg.bqg_device_errors() == 0
+
+
 def test_prefill_longest_k():
     """k = BQG_MAX_COLS (15360 = 60 chunks of 256) with ragged tokens and features."""
     need_gpu()
