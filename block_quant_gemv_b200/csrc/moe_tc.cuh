@@ -242,7 +242,7 @@ __host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW
 // Q4_0: 36 bytes (two blocks), Q8_0: 68 bytes, int4 (kind::f16, 64 k): 32 bytes.
 template <int FMT>
 __device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
-  uint32_t o[16];
+  uint32_t o[32];  // both halves, stored with one tensor-memory instruction
   if constexpr (FMT == BQG_Q4_0) {  // block A: d at bytes 0-1, qs 2..17; block B: d at 18-19, qs 20..35
     uint32_t v[9];
 #pragma unroll
@@ -251,10 +251,8 @@ __device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
     const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[4] >> 16)));
 #pragma unroll
     for (int m = 0; m < 4; ++m) tc_nib8(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[4 * m]);
-    tmem_st16(taddr, o);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) tc_nib8(v[5 + m], dB, &o[4 * m]);
-    tmem_st16(taddr + 16, o);
+    for (int m = 0; m < 4; ++m) tc_nib8(v[5 + m], dB, &o[16 + 4 * m]);
   } else if constexpr (FMT == BQG_Q8_0) {  // block A: d 0-1, q 2..33; block B: d 34-35, q 36..67
     uint32_t v[17];
 #pragma unroll
@@ -263,20 +261,15 @@ __device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
     const __half2 dB = __half2half2(__ushort_as_half(static_cast<unsigned short>(v[8] >> 16)));
 #pragma unroll
     for (int m = 0; m < 8; ++m) tc_q8x4(__funnelshift_r(v[m], v[m + 1], 16), dA, &o[2 * m]);
-    tmem_st16(taddr, o);
 #pragma unroll
-    for (int m = 0; m < 8; ++m) tc_q8x4(v[9 + m], dB, &o[2 * m]);
-    tmem_st16(taddr + 16, o);
+    for (int m = 0; m < 8; ++m) tc_q8x4(v[9 + m], dB, &o[16 + 2 * m]);
   } else {  // int4: 16-byte aligned
     const uint4 p0 = lds128(src), p1 = lds128(src + 16);
-    const uint32_t w0[4] = {p0.x, p0.y, p0.z, p0.w}, w1[4] = {p1.x, p1.y, p1.z, p1.w};
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-    for (int m = 0; m < 4; ++m) tc_i4nib8(w0[m], &o[4 * m]);
-    tmem_st16(taddr, o);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) tc_i4nib8(w1[m], &o[4 * m]);
-    tmem_st16(taddr + 16, o);
+    for (int m = 0; m < 8; ++m) tc_i4nib8(w[m], &o[4 * m]);
   }
+  tmem_st32(taddr, o);
 }
 
 // kind::i8: int4 64 bytes (128 k), int2 32 bytes; 16-byte aligned.  Each int4 word yields two
@@ -302,20 +295,19 @@ __device__ __forceinline__ void tc_i2_bytes(uint4 a, uint32_t (&o)[16]) {
 }
 template <int FMT>
 __device__ __forceinline__ void tc_i8_stage(uint32_t src, uint32_t taddr) {
-  uint32_t o[16];
+  uint32_t o[32];
+  uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&o[0]);
+  uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&o[16]);
   if constexpr (FMT == BQG_I4_ROW) {
     const uint4 p0 = lds128(src), p1 = lds128(src + 16), p2 = lds128(src + 32), p3 = lds128(src + 48);
-    tc_i4_bytes(p0, p1, o);
-    tmem_st16(taddr, o);
-    tc_i4_bytes(p2, p3, o);
-    tmem_st16(taddr + 16, o);
+    tc_i4_bytes(p0, p1, lo);
+    tc_i4_bytes(p2, p3, hi);
   } else {
     const uint4 p0 = lds128(src), p1 = lds128(src + 16);
-    tc_i2_bytes(p0, o);
-    tmem_st16(taddr, o);
-    tc_i2_bytes(p1, o);
-    tmem_st16(taddr + 16, o);
+    tc_i2_bytes(p0, lo);
+    tc_i2_bytes(p1, hi);
   }
+  tmem_st32(taddr, o);  // one tensor-memory instruction per stage
 }
 
 // One item's stages for this thread's row of a tile: wait for each raw chunk, dequantize every
