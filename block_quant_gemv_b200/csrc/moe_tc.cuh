@@ -8,43 +8,53 @@
 // each expert read serves every row routed to it; routed experts split from the dense shared
 // branch); Camelid README, "Gemma 4" (GeGLU experts; dense shared expert + sparse top-8 branch).
 //
-// One work item = up to 64 tokens of one expert (or of the shared expert) times two 128-row
-// weight tiles: the gate and up tiles of the same rows (gate/up phase), or two consecutive
-// tiles of the down matrix (down phase).  Weight rows sit on the MMA's M side (128), the item's
-// tokens on N (16..64, padded to 16), k along the matrix columns.  Each CTA (one per SM) runs
-// items claimed from a counter, with warp-specialised roles:
-//   warp 0      TMA: raw weight chunks (128 rows of each tile, 144 to 256 bytes of each row, in
+// Two variants of one kernel template: kind::f16 (Q8_0, Q4_0 and int4 weights as fp16, fp16
+// activation rows, fp32 accumulation, 64 k per stage) and kind::i8 (int4 and int2 weights as
+// unsigned bytes, activations as pairs of int8 digit rows, int32 accumulation, 128 k per stage).
+//
+// One work item = up to 64 activation rows (64 tokens in kind::f16; 32 tokens of two digit rows
+// each in kind::i8) of one expert (or of the shared expert) times two 128-row weight tiles: the
+// gate and up tiles of the same rows (gate/up phase), or two consecutive tiles of the down matrix
+// (down phase).  Weight rows sit on the MMA's M side (128), the activation rows on N (16..64,
+// padded to 16), k along the matrix columns.  Each CTA (one per SM) runs items claimed from a
+// counter, with warp-specialised roles:
+//   warp 0      TMA: raw weight chunks (128 rows of each tile, 136 to 192 bytes of each row, in
 //               their block format) through a ring in shared memory.  A 3-D tensor map with 8-byte
 //               elements views each family as [expert][super-row][bytes], a super-row being g = 1,
 //               2 or 4 consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of
 //               704 values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
 //               Each chunk takes a long piece of every row, so that one producer/consumer round
-//               through the raw ring covers three or four MMA stages.
+//               through the raw ring covers two to six MMA stages.
 //               Rows land in shared memory an odd multiple of 16 bytes apart (176 or 208), so the
 //               dequantizing threads' 16-byte loads of consecutive rows hit distinct bank groups
 //               (a 64- or 256-byte pitch put 4 or 8 rows on the same banks).
-//   warp 14     TMA: the item's activation rows (fp16, 128-byte swizzle, k-major) per 64-k stage.
-//   warps 2-9   dequantize: thread (tile f, row r) turns its row's 64 weights of a stage into fp16
-//               and stores them with tcgen05.st straight into TENSOR MEMORY (lane r), where the
-//               MMA reads its A operand.  Keeping A out of shared memory matters: 4-bit weights
-//               expanded to fp16 in shared memory would cost ~4 bytes of shared-memory traffic
-//               per weight (store + MMA read), more than the SM moves at the HBM rate.
+//   warp 14     TMA: the item's activation rows (128-byte swizzle, k-major), one stage at a time
+//               into the slot of the matching A stage.
+//   warps 2-9   dequantize: thread (tile f, row r) turns its row's weights of a stage into fp16
+//               or bytes and stores them with tcgen05.st straight into TENSOR MEMORY (lane r),
+//               where the MMA reads its A operand.  Keeping A out of shared memory matters:
+//               4-bit weights expanded in shared memory would cost 2-4 bytes of shared-memory
+//               traffic per weight (store + MMA read), more than the SM moves at the HBM rate.
+//               The first of these threads also waits for the stage's activation rows before it
+//               arrives, so the stage barrier covers both operands.
 //   warp 1      allocates all 512 tensor-memory columns; it and warps 15-21 issue tcgen05.mma
-//               (kind::f16, A from tensor memory, B from shared memory, fp32 accumulation): 4 A
-//               stages of 2 x 32 columns, and two accumulator buffers of 2 x 64 columns, so the
-//               epilogue of one item overlaps the MMAs of the next.  The MMAs of one thread run
-//               back to back at ~170 cycles each for any N up to 128 (measured on B200), while
-//               those of different warps overlap; so each tile's k steps are spread over up to
-//               four chains, each issued by its own warp into its own partial accumulator.
-//   warps 10-13 epilogue: read the accumulators (tcgen05.ld), apply int4 row scales, and write
-//               h = act(g) * u as fp16 (gate/up) or the fp32 per-pair outputs (down).
+//               (A from tensor memory, B from shared memory): 4 A stages of 2 x 32 columns, and
+//               two accumulator buffers of 2 x 64 columns, so the epilogue of one item overlaps
+//               the MMAs of the next.  The MMAs of one thread run back to back (~115-200 cycles
+//               each for any N up to 128, measured on B200), while those of different warps
+//               overlap; so each tile's k steps are spread over up to four chains, each issued by
+//               its own warp into its own partial accumulator.
+//   warps 10-13 epilogue: read the accumulators (tcgen05.ld), add the partials, apply row scales
+//               (and, in kind::i8, the digit recombination), and write h = act(g) * u (gate/up)
+//               or the fp32 per-pair outputs (down).
 //
-// Weights become fp16 exactly as stored values allow: Q4_0 (q - 8) and Q8_0 q exactly via the
-// fp16 exponent-bias identity (0x6400 | byte = 1024 + byte), then one rounding of the product by
-// d; int4 values -8..7 exactly (its row scale is applied to the fp32 accumulator).  Within each
-// group of 8 k, nibble formats store the weights in the order their bytes yield them
-// (elements 0,4,1,5,2,6,3,7); the activation rows are written in the same order, which leaves
-// every dot product unchanged.
+// kind::f16 weights become fp16 exactly as stored values allow: Q4_0 (q - 8) and Q8_0 q exactly
+// via the fp16 exponent-bias identity (0x6400 | byte = 1024 + byte), then one rounding of the
+// product by d; int4 values -8..7 exactly (its row scale is applied to the fp32 accumulator).
+// Within each group of 8 k, nibble formats store the weights in the order their bytes yield them
+// (elements 0,4,1,5,2,6,3,7 in kind::f16; 0,2,4,6,1,3,5,7 in kind::i8; int2 groups of 16 in
+// kind::i8); the activation rows are written in the same order, which leaves every dot product
+// unchanged.
 #pragma once
 
 #include <cuda.h>
