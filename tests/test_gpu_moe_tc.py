@@ -225,3 +225,31 @@ def test_glm_like_geometry_every_token_t64():
         tol = I8_TOL if path == bqg.MOE_PATH_TENSOR_CORES else 1e-4
         e = assert_close(y, ref, tol=tol, what=f"glm geometry T=64 path {path} (strict)")
         print(f"glm geometry T=64 path {path}: max rel err {e:.2e}")
+
+
+def test_i8_zero_and_outlier_activations():
+    """kind::i8 with degenerate rows: tokens whose x is all zero give exactly zero (scale 0, no
+    division), and tokens with one large outlier (1e3 among N(0, 1) values, 16-bit fixed point per
+    row then spends most of its range on the outlier) stay within the bounds of max|y|."""
+    need_gpu()
+    spec = wl.MoESpec("tc8_edge", 8, 2, 256, 128, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False)
+    assert i8_variant(spec)
+    L, lay = _layer(spec, bqg.MOE_PATH_TENSOR_CORES)
+    tokens = 16
+    x = wl.moe_tokens(spec, 3, tokens).clone()
+    x[0] = 0.0
+    x[5] = 0.0
+    x[7, 17] = 1e3
+    x[9, 200] = -1e3
+    idx, w, ridx, rw = _route(spec, 3, tokens)
+    y = bqg.moe_forward(lay, x.cuda(), idx, w)
+    torch.cuda.synchronize()
+    ref = om.moe_layer(oracle_layer(spec, 0, 0), x.numpy(), ridx, rw)
+    yc = y.cpu().numpy()
+    assert np.all(yc[0] == 0.0) and np.all(yc[5] == 0.0)
+    assert_close(yc, ref, what="i8 zero / outlier rows")
+    for t in (7, 9):  # each outlier token against its own scale
+        assert_close(yc[t], ref[t], tol=I8_TOL, what=f"i8 outlier token {t}")
+    normal = [t for t in range(tokens) if t not in (0, 5, 7, 9)]
+    assert_close(yc[normal], ref[normal], tol=I8_TOL, what="i8 ordinary tokens")
+    assert bqg.bqg_device_errors() == 0
