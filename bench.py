@@ -541,6 +541,32 @@ def time_single_q8_0(dev, seed):
             "us_per_call": us, "GB/s": nbytes / us / 1e3, "bytes_per_call": nbytes}
 
 
+def time_single_row_scaled(dev, seed):
+    """Single packed int4 and int2 GEMVs with a per-row scale, 6144x2048 (the GLM-like expert's down
+    matrix): enough distinct weight copies rotated in one graph that a rotation reads >= 256 MB."""
+    import torch
+
+    import block_quant_gemv_b200 as bqg
+    import synth
+    rows, cols = 6144, 2048
+    out = {"workload": "packed int4 / int2 with fp32 row scales, 6144x2048, batch 1 (rotating copies, CUDA graph)"}
+    x = synth.normal_f32(seed, synth.stream_id("rowscaled/x"), cols).to(dev)
+    y = torch.empty(rows, device=dev)
+    for name, fmt in (("i4_row", bqg.I4_ROW), ("i2_row", bqg.I2_ROW)):
+        wb = synth.weight_bytes(fmt, rows, cols)
+        copies = max(1, -(-(256 << 20) // wb))
+        Ws = [synth.matrix(fmt, rows, cols, seed, f"rowscaled/{name}/copy{c}", device=dev) for c in range(copies)]
+
+        def fn():
+            for W in Ws:
+                bqg.qgemv(fmt, W, x, rows, cols, y)
+        us = graph_us(fn, reps=10) / copies
+        nbytes = wb + 4 * (rows + cols)
+        out[name] = {"us_per_call": us, "GB/s": nbytes / us / 1e3, "bytes_per_call": nbytes, "rotating_copies": copies}
+        del Ws
+    return out
+
+
 def graph_us(fn, reps: int = 20) -> float:
     """Device time of fn (a sequence of library calls) captured once in a CUDA graph: warm-up
     replays, then CUDA events around `reps` replays on the capture stream."""
@@ -798,6 +824,7 @@ def run_ours(args, world, rank, local):
     extras = {}
     if not args.no_extras:
         extras["q8_0_2048"] = time_single_q8_0(dev, args.seed)
+        extras["row_scaled_6144x2048"] = time_single_row_scaled(dev, args.seed)
         extras["prefill"] = time_prefill(dev, args.seed, tensor_peak())
         extras["moe_gemma"] = time_moe_gemma(dev, args.seed, peak)
         if not args.no_glm:
