@@ -76,13 +76,32 @@ constexpr int kTcDqThreads = 256;          // 2 tiles x 128 rows
 #ifndef BQG_TC_NMAX
 #define BQG_TC_NMAX 64
 #endif
-#ifndef BQG_TC_ASTAGES
-#define BQG_TC_ASTAGES 4
+#ifndef BQG_TC_I8_STAGE_K
+#define BQG_TC_I8_STAGE_K 256
 #endif
 constexpr int kTcNMax = BQG_TC_NMAX;       // MMA N per item (tokens; two digit rows per token in kind::i8)
-constexpr int kTcAStages = BQG_TC_ASTAGES; // A stages in tensor memory (64 columns each: 2 tiles x 32)
-constexpr int kTcBStages = kTcAStages;     // activation stages in shared memory
-constexpr int kTcBStageBytes = kTcNMax * 128;  // N rows x 128 bytes (64 k fp16, or 128 k int8)
+constexpr int kTcACols = 256;              // tensor-memory columns of the A stage ring
+constexpr int kTcAStages = 4;              // barrier slots (the most stages a variant uses)
+constexpr int kTcBStages = kTcAStages;
+constexpr int kTcBRing = 32 * 1024;        // shared memory of the activation ring (all variants)
+// Stage geometry of a variant.  kind::f16: 64 k per stage, 2 tiles x 32 columns, 4 stages, 4 MMAs
+// of 16 k per tile.  kind::i8: BQG_TC_I8_STAGE_K (128 or 256) k per stage, 2 tiles x 32 or 64
+// columns, 4 or 2 stages, 4 or 8 MMAs of 32 k per tile; the activation rows of a stage are one
+// or two 128-byte-swizzled blocks of 128 k, kTcNMax * 128 bytes apart.
+template <bool I8>
+struct TcCfg {
+  static constexpr int kStageK = I8 ? BQG_TC_I8_STAGE_K : 64;
+  static constexpr int kTileCols = I8 ? kStageK / 4 : 32;    // 4 bytes (or two fp16) per column
+  static constexpr int kStageCols = 2 * kTileCols;
+  static constexpr int kAStages = kTcACols / kStageCols;
+  static constexpr int kKSteps = I8 ? kStageK / 32 : 4;       // MMAs per tile and stage
+  static constexpr int kBBlocks = I8 ? kStageK / 128 : 1;     // 128-byte swizzle blocks per B row
+  static constexpr int kBStageBytes = kBBlocks * kTcNMax * 128;
+};
+static_assert(TcCfg<true>::kAStages <= kTcAStages && TcCfg<false>::kAStages <= kTcAStages, "barrier slots");
+static_assert(TcCfg<true>::kAStages * TcCfg<true>::kBStageBytes <= kTcBRing &&
+                  TcCfg<false>::kAStages * TcCfg<false>::kBStageBytes <= kTcBRing,
+              "activation ring");
 constexpr int kTcAccTile = kTcNMax;        // accumulator columns per tile of one buffer
 constexpr int kTcAccBuf = 2 * kTcAccTile;  // columns per accumulator buffer (two tiles)
 #ifndef BQG_TC_ACC_BUFS
@@ -91,13 +110,13 @@ constexpr int kTcAccBuf = 2 * kTcAccTile;  // columns per accumulator buffer (tw
 constexpr int kTcAccBufs = BQG_TC_ACC_BUFS;  // accumulator buffers (2: an item's epilogue overlaps the next one's MMAs)
 constexpr int kTcDescs = 8;                // item descriptor ring
 constexpr int kTcRawMax = 12;              // raw weight ring depth (runtime, by window size)
-constexpr int kTcAccCol = kTcAStages * 64; // first accumulator column (after the A stages)
+constexpr int kTcAccCol = kTcACols;       // first accumulator column (after the A stages)
 static_assert(kTcAccBufs >= 1 && kTcAccBufs <= 2, "one or two accumulator buffers");
 static_assert(kTcAccCol + kTcAccBufs * kTcAccBuf <= 512, "tensor memory: A stages + accumulator buffers");
 constexpr int kTcDescReaders = 1 + kTcMmaWarps + 8 + 4;  // B producer, MMA, dequant and epilogue warps
 // smem: [1 KB alignment slack][B ring][raw ring][barriers + descriptors]
 constexpr int kTcBarBytes = 1024;
-constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBStages) * kTcBStageBytes + kTcBarBytes;
+constexpr size_t kTcFixedSmem = 1024 + size_t(kTcBRing) + kTcBarBytes;
 constexpr size_t kTcMaxSmem = 227 * 1024;
 static_assert(kTcBStages == kTcAStages, "activation stage i shares the A stage's barriers");
 static_assert((2 * kTcRawMax + 2 * kTcAStages + kTcBStages + 4 + 2 * kTcDescs + 1) * 8 + 16 + kTcDescs * 32 <=
@@ -239,13 +258,15 @@ __device__ __forceinline__ void tc_acc8i(uint32_t taddr, int stride, int parts, 
 // Raw chunk geometry per weight format: weights and bytes of one row per chunk, and the shared-
 // memory pitch of the rows (an odd multiple of 16 bytes; the chunk plus up to 12 bytes of
 // misalignment for the 18- and 34-byte block formats).
+// int4 takes 512 k (256 bytes, pitch 272) when the kind::i8 stage is 256 k, else 384 k.
 __host__ __device__ constexpr int tc_raw_k(int fmt) {
-  return fmt == BQG_I2_ROW ? 768 : fmt == BQG_I4_ROW ? 384 : fmt == BQG_Q4_0 ? 256 : 128;
+  return fmt == BQG_I2_ROW ? 768 : fmt == BQG_I4_ROW ? (BQG_TC_I8_STAGE_K == 256 ? 512 : 384)
+                                 : fmt == BQG_Q4_0 ? 256 : 128;
 }
 __host__ __device__ constexpr int tc_raw_cb(int fmt) {
-  return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? 192 : fmt == BQG_Q4_0 ? 144 : 136;
+  return fmt == BQG_I2_ROW ? 192 : fmt == BQG_I4_ROW ? tc_raw_k(fmt) / 2 : fmt == BQG_Q4_0 ? 144 : 136;
 }
-__host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? 208 : 176; }
+__host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? tc_raw_cb(fmt) + 16 : 176; }
 
 // One stage of one row, loaded first and converted after: all its shared-memory words are read
 // before the first tensor-memory store, so the loads of the second half do not wait behind it.
@@ -305,19 +326,24 @@ __device__ __forceinline__ void tc_i2_bytes(uint4 a, uint32_t (&o)[16]) {
 }
 template <int FMT>
 __device__ __forceinline__ void tc_i8_stage(uint32_t src, uint32_t taddr) {
+  constexpr int kStageK = TcCfg<true>::kStageK;
   uint32_t o[32];
   uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&o[0]);
   uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&o[16]);
-  if constexpr (FMT == BQG_I4_ROW) {
-    const uint4 p0 = lds128(src), p1 = lds128(src + 16), p2 = lds128(src + 32), p3 = lds128(src + 48);
-    tc_i4_bytes(p0, p1, lo);
-    tc_i4_bytes(p2, p3, hi);
-  } else {
-    const uint4 p0 = lds128(src), p1 = lds128(src + 16);
-    tc_i2_bytes(p0, lo);
-    tc_i2_bytes(p1, hi);
+#pragma unroll
+  for (int g = 0; g < kStageK / 128; ++g) {  // 128 k = 32 tensor-memory columns per step
+    if constexpr (FMT == BQG_I4_ROW) {       // 64 bytes per 128 k
+      const uint32_t a = src + 64 * g;
+      const uint4 p0 = lds128(a), p1 = lds128(a + 16), p2 = lds128(a + 32), p3 = lds128(a + 48);
+      tc_i4_bytes(p0, p1, lo);
+      tc_i4_bytes(p2, p3, hi);
+    } else {                                 // int2: 32 bytes per 128 k
+      const uint32_t a = src + 32 * g;
+      tc_i2_bytes(lds128(a), lo);
+      tc_i2_bytes(lds128(a + 16), hi);
+    }
+    tmem_st32(taddr + 32 * g, o);
   }
-  tmem_st32(taddr, o);  // one tensor-memory instruction per stage
 }
 
 // One item's stages for this thread's row of a tile: wait for each raw chunk, dequantize every
@@ -334,8 +360,10 @@ __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_ba
                                            int raw_stage_bytes, uint64_t* raw_full, uint64_t* raw_empty,
                                            uint64_t* a_full, uint64_t* a_empty, uint64_t* b_full, bool wait_b,
                                            uint32_t tcol, int& slot_r, uint32_t& ph_r, int& as) {
-  constexpr int kStageK = I8 ? 128 : 64;
+  using C = TcCfg<I8>;
+  constexpr int kStageK = C::kStageK;
   constexpr int kSpr = tc_raw_k(FMT) / kStageK;      // stages per raw chunk
+  static_assert(tc_raw_k(FMT) % kStageK == 0, "raw chunks hold whole stages");
   constexpr int kCb = tc_raw_cb(FMT);
   constexpr int kStageBytes = kCb / kSpr;
   const int nraw = (nst + kSpr - 1) / kSpr;
@@ -344,18 +372,18 @@ __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_ba
     const uint32_t base = row_base + uint32_t(slot_r * raw_stage_bytes) + (uint32_t(mis0 + kc * kCb) & 15u);
     const int nh = min(kSpr, nst - kc * kSpr);
     for (int h = 0; h < nh; ++h, ++as) {
-      const int aslot = as % kTcAStages;
-      if (as >= kTcAStages && !mbar_wait(&a_empty[aslot], uint32_t(as / kTcAStages - 1) & 1u)) return false;
+      const int aslot = as % C::kAStages;
+      if (as >= C::kAStages && !mbar_wait(&a_empty[aslot], uint32_t(as / C::kAStages - 1) & 1u)) return false;
       tc_fence_after();
       if (row_on) {
         const uint32_t src = base + uint32_t(h * kStageBytes);
-        const uint32_t taddr = tcol + uint32_t(aslot * 64);
+        const uint32_t taddr = tcol + uint32_t(aslot * C::kStageCols);
         if constexpr (I8) tc_i8_stage<FMT>(src, taddr);
         else tc_f16_stage<FMT>(src, taddr);
         tmem_wait_st();
       }
       tc_fence_before();
-      if (wait_b && !mbar_wait(&b_full[aslot], uint32_t(as / kTcAStages) & 1u)) return false;
+      if (wait_b && !mbar_wait(&b_full[aslot], uint32_t(as / C::kAStages) & 1u)) return false;
       mbar_arrive(&a_full[aslot]);
     }
     mbar_arrive(&raw_empty[slot_r]);
@@ -374,12 +402,13 @@ __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_ba
 // int8 digit rows, int32 accumulators); 128 k per stage instead of 64.
 template <bool I8>
 __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant__ TcParams P) {
-  constexpr int kStageK = I8 ? 128 : 64;
+  using C = TcCfg<I8>;
+  constexpr int kStageK = C::kStageK;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_s & 1023)) & 1023);
-  uint8_t* bring = smem;                                            // kTcBStages x N x 128 bytes
-  uint8_t* wring = bring + size_t(kTcBStages) * kTcBStageBytes;    // raw_stages x raw_stage_bytes
+  uint8_t* bring = smem;                                            // C::kAStages x C::kBStageBytes
+  uint8_t* wring = bring + size_t(kTcBRing);                        // raw_stages x raw_stage_bytes
   uint64_t* bars = reinterpret_cast<uint64_t*>(wring + size_t(P.raw_stages) * P.raw_stage_bytes);
   uint64_t* raw_full = bars;                        // [kTcRawMax] TMA bytes
   uint64_t* raw_empty = raw_full + kTcRawMax;       // [kTcRawMax] 256 dequant threads
@@ -499,7 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           d0 = make_int4(shared | (two << 1), e, m0, ntok);
           const int brow = I8 ? 2 * (off + c * nmax) : off + c * nmax;  // first B row
           const int nb = I8 ? 2 * ntok : ntok;                                // B rows
-          d1 = make_int4(brow, (nb + 15) & ~15, off + c * nmax, P.fam[fb].cols / kStageK);
+          d1 = make_int4(brow, (nb + 15) & ~15, off + c * nmax, (P.fam[fb].cols + kStageK - 1) / kStageK);
         } else {
           d0 = make_int4(-1, 0, 0, 0);
           d1 = make_int4(0, 0, 0, 0);
@@ -563,8 +592,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         const int sh = d0.x & 1;
         const int N = d1.y;
         for (int s = 0; s < d1.w; ++s, ++bs) {
-          const int slot = bs % kTcBStages;
-          if (bs >= kTcBStages && !mbar_wait(&a_empty[slot], uint32_t(bs / kTcBStages - 1) & 1u)) {
+          const int slot = bs % C::kAStages;
+          if (bs >= C::kAStages && !mbar_wait(&a_empty[slot], uint32_t(bs / C::kAStages - 1) & 1u)) {
             ok = false;
             break;
           }
@@ -572,16 +601,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&b_full[slot], uint32_t(N * 128));
-          uint8_t* dst = bring + size_t(slot) * kTcBStageBytes;
-          for (int nb = 0; nb < N / 16; ++nb)
-            tma_load_2d(dst + nb * 2048, &P.bmap[sh], s * kStageK, d1.x + 16 * nb, &b_full[slot]);
+          mbar_arrive_expect_tx(&b_full[slot], uint32_t(N * 128 * C::kBBlocks));
+          uint8_t* dst = bring + size_t(slot) * C::kBStageBytes;
+          for (int blk = 0; blk < C::kBBlocks; ++blk)  // 128 k (kind::i8) or 64 k (fp16) per block
+            for (int nb = 0; nb < N / 16; ++nb)
+              tma_load_2d(dst + blk * (kTcNMax * 128) + nb * 2048, &P.bmap[sh],
+                          s * kStageK + blk * (I8 ? 128 : 64), d1.x + 16 * nb, &b_full[slot]);
         }
       }
       if (!ok) {
         *abort_flag = 1;
-        for (int q = (bs > kTcBStages ? bs - kTcBStages : 0); q < bs; ++q)
-          mbar_wait(&b_full[q % kTcBStages], uint32_t(q / kTcBStages) & 1u);
+        for (int q = (bs > C::kAStages ? bs - C::kAStages : 0); q < bs; ++q)
+          mbar_wait(&b_full[q % C::kAStages], uint32_t(q / C::kAStages) & 1u);
       }
     }
   } else if (warp == kTcWarpMma || warp >= kTcWarpMma2) {
@@ -603,6 +634,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         if (d0.x < 0) break;
         const int two = (d0.x >> 1) & 1;
         const int N = d1.y;
+        const int kcols = P.fam[(d0.x & 1) ? 2 : 0].cols;
         const int parts = tc_partials(N);
         const int buf = it % kTcAccBufs;
         if (it >= kTcAccBufs && !mbar_wait(&acc_empty[buf], uint32_t(it / kTcAccBufs - 1) & 1u)) {
@@ -613,18 +645,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
         const uint32_t idesc = I8 ? umma_idesc_i8(128, N) : umma_idesc_f16(128, N);
         const uint32_t dbase = tmem + uint32_t(kTcAccCol + buf * kTcAccBuf + p * N);
         for (int s = 0; s < d1.w; ++s, ++as) {
-          const int aslot = as % kTcAStages;  // B uses the same slot
-          if (!mbar_wait(&a_full[aslot], uint32_t(as / kTcAStages) & 1u)) {  // A and B of the stage
+          const int aslot = as % C::kAStages;  // B uses the same slot
+          if (!mbar_wait(&a_full[aslot], uint32_t(as / C::kAStages) & 1u)) {  // A and B of the stage
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t b_s = smem_u32(bring + size_t(aslot) * kTcBStageBytes);
+          const uint32_t b_s = smem_u32(bring + size_t(aslot) * C::kBStageBytes);
+          // k steps of this stage: all of them, or only those inside the row (a last stage of 128 k
+          // when the stage is 256 k)
+          const int ksteps = s == d1.w - 1 && (kcols % kStageK) != 0 ? (kcols % kStageK) / (I8 ? 32 : 16) : C::kKSteps;
           for (int f = f0; f < 1 + two && p < parts; f += kTileStep) {
-            const uint32_t acol = tmem + uint32_t(aslot * 64 + f * 32);
+            const uint32_t acol = tmem + uint32_t(aslot * C::kStageCols + f * C::kTileCols);
             const uint32_t dcol = dbase + uint32_t(f * kTcAccTile);
-            for (int kk = p; kk < 4; kk += parts) {  // 8 tensor-memory columns, 32 bytes of B per MMA
-              const uint64_t bdesc = umma_desc_sw128(b_s + 32 * kk);
+            for (int kk = p; kk < ksteps; kk += parts) {  // 8 tensor-memory columns, 32 bytes of B per MMA
+              const uint64_t bdesc = umma_desc_sw128(b_s + (kk >> 2) * (kTcNMax * 128) + 32 * (kk & 3));
               const uint32_t acc = (s > 0 || kk != p) ? 1u : 0u;
               if constexpr (I8) umma_i8_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);  // 32 k
               else umma_f16_ts(dcol, acol + 8 * kk, bdesc, idesc, acc);               // 16 k
@@ -666,7 +701,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
       const int fmt = F.fmt, win = F.win, g = F.g, j = r % g, q = r / g;
       const uint32_t row_base = wring_s + uint32_t(f * 128 * win + j * (128 / g) * win + q * win);
       const int mis0 = j * F.row_bytes;
-      const uint32_t tcol = tmem + tlane + uint32_t(f * 32);
+      const uint32_t tcol = tmem + tlane + uint32_t(f * C::kTileCols);
       const int nst = d1.w;
       const bool wait_b = warp == kTcWarpDq && lane == 0;
       if constexpr (I8) {
