@@ -9,8 +9,8 @@
 // branch); Camelid README, "Gemma 4" (GeGLU experts; dense shared expert + sparse top-8 branch).
 //
 // Two variants of one kernel template: kind::f16 (Q8_0, Q4_0 and int4 weights as fp16, fp16
-// activation rows, fp32 accumulation, 64 k per stage) and kind::i8 (int4 and int2 weights as
-// unsigned bytes, activations as pairs of int8 digit rows, int32 accumulation, 128 k per stage).
+// activation rows, fp32 accumulation, 128 k per stage) and kind::i8 (int4 and int2 weights as
+// unsigned bytes, activations as pairs of int8 digit rows, int32 accumulation, 256 k per stage).
 //
 // One work item = up to 64 activation rows (64 tokens in kind::f16; 32 tokens of two digit rows
 // each in kind::i8) of one expert (or of the shared expert) times two 128-row weight tiles: the
@@ -18,14 +18,14 @@
 // (down phase).  Weight rows sit on the MMA's M side (128), the activation rows on N (16..64,
 // padded to 16), k along the matrix columns.  Each CTA (one per SM) runs items claimed from a
 // counter, with warp-specialised roles:
-//   warp 0      TMA: raw weight chunks (128 rows of each tile, 136 to 192 bytes of each row, in
+//   warp 0      TMA: raw weight chunks (128 rows of each tile, 136 to 256 bytes of each row, in
 //               their block format) through a ring in shared memory.  A 3-D tensor map with 8-byte
 //               elements views each family as [expert][super-row][bytes], a super-row being g = 1,
 //               2 or 4 consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of
 //               704 values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
 //               Each chunk takes a long piece of every row, so that one producer/consumer round
 //               through the raw ring covers two to six MMA stages.
-//               Rows land in shared memory an odd multiple of 16 bytes apart (176 or 208), so the
+//               Rows land in shared memory an odd multiple of 16 bytes apart (176, 208 or 272), so the
 //               dequantizing threads' 16-byte loads of consecutive rows hit distinct bank groups
 //               (a 64- or 256-byte pitch put 4 or 8 rows on the same banks).
 //   warp 14     TMA: the item's activation rows (128-byte swizzle, k-major), one stage at a time
@@ -38,7 +38,8 @@
 //               The first of these threads also waits for the stage's activation rows before it
 //               arrives, so the stage barrier covers both operands.
 //   warp 1      allocates all 512 tensor-memory columns; it and warps 15-21 issue tcgen05.mma
-//               (A from tensor memory, B from shared memory): 4 A stages of 2 x 32 columns, and
+//               (A from tensor memory, B from shared memory): two A stages of 2 x 64 columns
+//               (128 fp16 or 256 byte weights of each row), and
 //               two accumulator buffers of 2 x 64 columns, so the epilogue of one item overlaps
 //               the MMAs of the next.  The MMAs of one thread run back to back (~115-200 cycles
 //               each for any N up to 128, measured on B200), while those of different warps
@@ -84,18 +85,23 @@ constexpr int kTcACols = 256;              // tensor-memory columns of the A sta
 constexpr int kTcAStages = 4;              // barrier slots (the most stages a variant uses)
 constexpr int kTcBStages = kTcAStages;
 constexpr int kTcBRing = 32 * 1024;        // shared memory of the activation ring (all variants)
-// Stage geometry of a variant.  kind::f16: 64 k per stage, 2 tiles x 32 columns, 4 stages, 4 MMAs
-// of 16 k per tile.  kind::i8: BQG_TC_I8_STAGE_K (128 or 256) k per stage, 2 tiles x 32 or 64
-// columns, 4 or 2 stages, 4 or 8 MMAs of 32 k per tile; the activation rows of a stage are one
-// or two 128-byte-swizzled blocks of 128 k, kTcNMax * 128 bytes apart.
+// Stage geometry of a variant.  kind::f16: BQG_TC_F16_STAGE_K (64 or 128) k per stage, 2 tiles x 32
+// or 64 columns, 4 or 2 stages, 4 or 8 MMAs of 16 k per tile; the activation rows of a stage are
+// one or two 128-byte-swizzled blocks of 64 k.  kind::i8: BQG_TC_I8_STAGE_K (128 or 256) k per
+// stage, 2 tiles x 32 or 64 columns, 4 or 2 stages, 4 or 8 MMAs of 32 k per tile; one or two
+// blocks of 128 k.  Blocks of one stage sit kTcNMax * 128 bytes apart.  Bigger stages halve the
+// handoffs through the stage barriers per weight, which bound this loop.
+#ifndef BQG_TC_F16_STAGE_K
+#define BQG_TC_F16_STAGE_K 128
+#endif
 template <bool I8>
 struct TcCfg {
-  static constexpr int kStageK = I8 ? BQG_TC_I8_STAGE_K : 64;
-  static constexpr int kTileCols = I8 ? kStageK / 4 : 32;    // 4 bytes (or two fp16) per column
+  static constexpr int kStageK = I8 ? BQG_TC_I8_STAGE_K : BQG_TC_F16_STAGE_K;
+  static constexpr int kTileCols = I8 ? kStageK / 4 : kStageK / 2;  // 4 bytes (or two fp16) per column
   static constexpr int kStageCols = 2 * kTileCols;
   static constexpr int kAStages = kTcACols / kStageCols;
-  static constexpr int kKSteps = I8 ? kStageK / 32 : 4;       // MMAs per tile and stage
-  static constexpr int kBBlocks = I8 ? kStageK / 128 : 1;     // 128-byte swizzle blocks per B row
+  static constexpr int kKSteps = I8 ? kStageK / 32 : kStageK / 16;  // MMAs per tile and stage
+  static constexpr int kBBlocks = I8 ? kStageK / 128 : kStageK / 64;  // 128-byte swizzle blocks per B row
   static constexpr int kBStageBytes = kBBlocks * kTcNMax * 128;
 };
 static_assert(TcCfg<true>::kAStages <= kTcAStages && TcCfg<false>::kAStages <= kTcAStages, "barrier slots");
@@ -132,7 +138,7 @@ struct TcFam {
   int g;                // rows per super-row of the tensor map
   int win;              // bytes fetched per row and raw chunk (a 16-byte-aligned window)
   int cb;               // bytes of one raw chunk of one row
-  int raw_k;            // weights per raw chunk (int4 384, int2 768, Q4_0 256, Q8_0 128)
+  int raw_k;            // weights per raw chunk (int4 512 or 384, int2 768, Q4_0 256, Q8_0 128)
   int scale_off;        // int4: byte offset of the row scales in one matrix
   int m_off;            // row offset of this tile inside an item (0, or 128 for the second down tile)
 };
@@ -163,7 +169,7 @@ struct alignas(64) TcParams {
   float* h32[2];        // gate/up of the kind::i8 variant: h rows in fp32 (natural order)
 };
 
-// ---------------------------------------------------------------- dequantization of one 64-k stage
+// ---------------------------------------------------------------- dequantization of one stage
 // Four fp16 pairs of the 8 nibbles of word w (element 2m = low nibble of byte m), in the order
 // the bytes yield them: (e0, e4) (e1, e5) (e2, e6) (e3, e7); values (q - 8) * d.
 __device__ __forceinline__ void tc_nib8(uint32_t w, __half2 d2, uint32_t* o) {
@@ -268,11 +274,11 @@ __host__ __device__ constexpr int tc_raw_cb(int fmt) {
 }
 __host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? tc_raw_cb(fmt) + 16 : 176; }
 
-// One stage of one row, loaded first and converted after: all its shared-memory words are read
-// before the first tensor-memory store, so the loads of the second half do not wait behind it.
-// Q4_0: 36 bytes (two blocks), Q8_0: 68 bytes, int4 (kind::f16, 64 k): 32 bytes.
+// 64 k of one row (32 tensor-memory columns), loaded first and converted after: all its shared-
+// memory words are read before the tensor-memory store, so the loads of the second half do not
+// wait behind it.  Q4_0: 36 bytes (two blocks), Q8_0: 68 bytes, int4 (kind::f16): 32 bytes.
 template <int FMT>
-__device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
+__device__ __forceinline__ void tc_f16_sub(uint32_t src, uint32_t taddr) {
   uint32_t o[32];  // both halves, stored with one tensor-memory instruction
   if constexpr (FMT == BQG_Q4_0) {  // block A: d at bytes 0-1, qs 2..17; block B: d at 18-19, qs 20..35
     uint32_t v[9];
@@ -301,6 +307,12 @@ __device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
     for (int m = 0; m < 8; ++m) tc_i4nib8(w[m], &o[4 * m]);
   }
   tmem_st32(taddr, o);
+}
+template <int FMT>
+__device__ __forceinline__ void tc_f16_stage(uint32_t src, uint32_t taddr) {
+  constexpr int kSub = FMT == BQG_Q4_0 ? 36 : FMT == BQG_Q8_0 ? 68 : 32;  // bytes per 64 k
+#pragma unroll
+  for (int g = 0; g < TcCfg<false>::kStageK / 64; ++g) tc_f16_sub<FMT>(src + kSub * g, taddr + 32 * g);
 }
 
 // kind::i8: int4 64 bytes (128 k), int2 32 bytes; 16-byte aligned.  Each int4 word yields two
@@ -347,7 +359,7 @@ __device__ __forceinline__ void tc_i8_stage(uint32_t src, uint32_t taddr) {
 }
 
 // One item's stages for this thread's row of a tile: wait for each raw chunk, dequantize every
-// 64- (kind::f16) or 128-k (kind::i8) stage of it into the A stage ring in tensor memory, and
+// stage of it (TcCfg<I8>::kStageK weights) into the A stage ring in tensor memory, and
 // hand the stages to the MMA issuers.  The format is a template argument, so the block layout
 // and every offset are constants.  Returns false when a bounded wait gave up.
 //   row_base  shared address of this row's window in raw stage 0;  mis0  j * row_bytes (the
@@ -397,9 +409,9 @@ __device__ __forceinline__ bool tc_dq_item(int nst, bool row_on, uint32_t row_ba
 
 // ---------------------------------------------------------------- the kernel
 // Item descriptor: d0 = (flags: bit0 shared, bit1 second tile present; expert; m0; tokens),
-//                  d1 = (first activation row; N; first output row; 64-k stages).
+//                  d1 = (first activation row; N; first output row; stages).
 // I8: kind::i8 variant (int4 / int2 weights as unsigned bytes in tensor memory, activations as
-// int8 digit rows, int32 accumulators); 128 k per stage instead of 64.
+// int8 digit rows, int32 accumulators); the stage geometry of each variant is TcCfg<I8>.
 template <bool I8>
 __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant__ TcParams P) {
   using C = TcCfg<I8>;
@@ -603,7 +615,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_tc(const __grid_constant_
           }
           mbar_arrive_expect_tx(&b_full[slot], uint32_t(N * 128 * C::kBBlocks));
           uint8_t* dst = bring + size_t(slot) * C::kBStageBytes;
-          for (int blk = 0; blk < C::kBBlocks; ++blk)  // 128 k (kind::i8) or 64 k (fp16) per block
+          for (int blk = 0; blk < C::kBBlocks; ++blk)  // 128 k (kind::i8) or 64 k (fp16) per swizzle block
             for (int nb = 0; nb < N / 16; ++nb)
               tma_load_2d(dst + blk * (kTcNMax * 128) + nb * 2048, &P.bmap[sh],
                           s * kStageK + blk * (I8 ? 128 : 64), d1.x + 16 * nb, &b_full[slot]);
