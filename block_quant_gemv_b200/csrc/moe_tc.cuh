@@ -18,14 +18,14 @@
 // (down phase).  Weight rows sit on the MMA's M side (128), the activation rows on N (16..64,
 // padded to 16), k along the matrix columns.  Each CTA (one per SM) runs items claimed from a
 // counter, with warp-specialised roles:
-//   warp 0      TMA: raw weight chunks (128 rows of each tile, 136 to 256 bytes of each row, in
+//   warp 0      TMA: raw weight chunks (128 rows of each tile, 192 to 288 bytes of each row, in
 //               their block format) through a ring in shared memory.  A 3-D tensor map with 8-byte
 //               elements views each family as [expert][super-row][bytes], a super-row being g = 1,
 //               2 or 4 consecutive rows so that its byte length is a multiple of 16 (Q4_0 rows of
 //               704 values are 396 bytes); each row's chunk is fetched in a 16-byte-aligned window.
 //               Each chunk takes a long piece of every row, so that one producer/consumer round
-//               through the raw ring covers two to six MMA stages.
-//               Rows land in shared memory an odd multiple of 16 bytes apart (176, 208 or 272), so the
+//               through the raw ring covers two to four MMA stages.
+//               Rows land in shared memory an odd multiple of 16 bytes apart (208, 272 or 304), so the
 //               dequantizing threads' 16-byte loads of consecutive rows hit distinct bank groups
 //               (a 64- or 256-byte pitch put 4 or 8 rows on the same banks).
 //   warp 14     TMA: the item's activation rows (128-byte swizzle, k-major), one stage at a time
@@ -138,7 +138,7 @@ struct TcFam {
   int g;                // rows per super-row of the tensor map
   int win;              // bytes fetched per row and raw chunk (a 16-byte-aligned window)
   int cb;               // bytes of one raw chunk of one row
-  int raw_k;            // weights per raw chunk (int4 512 or 384, int2 768, Q4_0 256, Q8_0 128)
+  int raw_k;            // weights per raw chunk (int4 512 or 384, int2 768, Q4_0 512, Q8_0 256)
   int scale_off;        // int4: byte offset of the row scales in one matrix
   int m_off;            // row offset of this tile inside an item (0, or 128 for the second down tile)
 };
@@ -267,12 +267,12 @@ __device__ __forceinline__ void tc_acc8i(uint32_t taddr, int stride, int parts, 
 // int4 takes 512 k (256 bytes, pitch 272) when the kind::i8 stage is 256 k, else 384 k.
 __host__ __device__ constexpr int tc_raw_k(int fmt) {
   return fmt == BQG_I2_ROW ? 768 : fmt == BQG_I4_ROW ? (BQG_TC_I8_STAGE_K == 256 ? 512 : 384)
-                                 : fmt == BQG_Q4_0 ? 256 : 128;
+                                 : fmt == BQG_Q4_0 ? 512 : 256;
 }
 __host__ __device__ constexpr int tc_raw_cb(int fmt) {
-  return fmt == BQG_I2_ROW ? 192 : fmt == BQG_I4_ROW ? tc_raw_k(fmt) / 2 : fmt == BQG_Q4_0 ? 144 : 136;
+  return fmt == BQG_I2_ROW ? 192 : fmt == BQG_I4_ROW ? tc_raw_k(fmt) / 2 : fmt == BQG_Q4_0 ? 288 : 272;
 }
-__host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? tc_raw_cb(fmt) + 16 : 176; }
+__host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? tc_raw_cb(fmt) + 16 : 304; }
 
 // 64 k of one row (32 tensor-memory columns), loaded first and converted after: all its shared-
 // memory words are read before the tensor-memory store, so the loads of the second half do not
@@ -1042,7 +1042,7 @@ inline bool tc_fam(int fmt, const void* base, size_t stride, int rows, int cols,
   } else {
     F.raw_k = tc_raw_k(fmt);
     F.cb = tc_raw_cb(fmt);
-    F.win = tc_raw_win(fmt);  // chunk (144 or 136 bytes) + up to 12 bytes of misalignment
+    F.win = tc_raw_win(fmt);  // chunk (288 or 272 bytes) + up to 12 bytes of misalignment
   }
   F.m_off = m_off;
   *out = F;
