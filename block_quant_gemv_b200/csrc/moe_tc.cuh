@@ -273,6 +273,22 @@ __host__ __device__ constexpr int tc_raw_cb(int fmt) {
   return fmt == BQG_I2_ROW ? 192 : fmt == BQG_I4_ROW ? tc_raw_k(fmt) / 2 : fmt == BQG_Q4_0 ? 288 : 272;
 }
 __host__ __device__ constexpr int tc_raw_win(int fmt) { return fmt == BQG_I2_ROW || fmt == BQG_I4_ROW ? tc_raw_cb(fmt) + 16 : 304; }
+// Geometry checks per format: the window holds the chunk plus the largest misalignment (12 bytes
+// for the block formats, whose rows are multiples of 4 bytes; none for int4 / int2, whose chunks
+// start 16-byte aligned), its pitch is an odd multiple of 16 bytes, chunks hold whole stages of
+// both variants, and at least two raw stages of the widest window fit beside the fixed areas.
+constexpr bool tc_raw_geometry_ok(int fmt, int stage_k, int fixed_smem, int max_smem) {
+  return tc_raw_win(fmt) >= tc_raw_cb(fmt) + (fmt == BQG_Q4_0 || fmt == BQG_Q8_0 ? 12 : 0) &&
+         tc_raw_win(fmt) % 16 == 0 && (tc_raw_win(fmt) / 16) % 2 == 1 && tc_raw_k(fmt) % stage_k == 0 &&
+         fixed_smem + 2 * (2 * 128 * tc_raw_win(fmt)) <= max_smem;
+}
+
+static_assert(tc_raw_geometry_ok(BQG_Q4_0, TcCfg<false>::kStageK, int(kTcFixedSmem), int(kTcMaxSmem)) &&
+                  tc_raw_geometry_ok(BQG_Q8_0, TcCfg<false>::kStageK, int(kTcFixedSmem), int(kTcMaxSmem)) &&
+                  tc_raw_geometry_ok(BQG_I4_ROW, TcCfg<false>::kStageK, int(kTcFixedSmem), int(kTcMaxSmem)) &&
+                  tc_raw_geometry_ok(BQG_I4_ROW, TcCfg<true>::kStageK, int(kTcFixedSmem), int(kTcMaxSmem)) &&
+                  tc_raw_geometry_ok(BQG_I2_ROW, TcCfg<true>::kStageK, int(kTcFixedSmem), int(kTcMaxSmem)),
+              "raw chunk geometry");
 
 // 64 k of one row (32 tensor-memory columns), loaded first and converted after: all its shared-
 // memory words are read before the tensor-memory store, so the loads of the second half do not
