@@ -226,11 +226,17 @@ __host__ __device__ __forceinline__ int tc_kpos(int k, int nibble) {
 }
 
 // Partial accumulators per tile for an item of N (padded) tokens: 4 x 16, 2 x 32 or 1 x N columns,
-// so that both tiles of an accumulator buffer fit its 128 columns.
+// so that both tiles of an accumulator buffer fit its 128 columns.  Partial p takes the k steps
+// p, p + parts, ... and is initialised by its first one, so every partial needs at least one k step
+// in an item's first stage: the shortest possible stage (a matrix of 64 columns in kind::f16, 128
+// in kind::i8, the smallest widths either variant accepts) has 4 k steps, the most partials used.
+constexpr int kTcMaxPartials = 4;
+static_assert(64 / 16 >= kTcMaxPartials && 128 / 32 >= kTcMaxPartials,
+              "every partial accumulator gets a k step of the first stage");
 __host__ __device__ __forceinline__ int tc_partials(int N) {
   const int cap = kTcMmaWarps >= 2 ? kTcMmaWarps / 2 : 1;  // issuers per tile
   int p = 1;
-  while (p < 4 && p < cap && 2 * p * N <= kTcAccTile) p *= 2;
+  while (p < kTcMaxPartials && p < cap && 2 * p * N <= kTcAccTile) p *= 2;
   return p;
 }
 
