@@ -61,6 +61,9 @@ TC_SPECS = [
     wl.MoESpec("tc8_i4_rows384", 5, 2, 384, 384, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False),
     # int4 with inter 192 (not a multiple of 128): the kind::f16 variant
     wl.MoESpec("tc_i4_f16_inter192", 4, 2, 256, 192, bqg.I4_ROW, bqg.ACT_SILU, 0, 0, False),
+    # inter 64: the down matrix's only stage is half a 128-k stage (four k steps, one per partial
+    # accumulator); Q4_0 rows of 64 values are 36 bytes (4 rows per super-row)
+    wl.MoESpec("tc_q4_inter64", 6, 2, 128, 64, bqg.Q4_0, bqg.ACT_SILU, 0, 0, False),
 ]
 
 
